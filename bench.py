@@ -1,0 +1,485 @@
+"""Benchmark of one decode step of load-balanced split-KV attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload extreme] [--impl ours|reference]
+
+A step is the whole hot path over one batch: the per-step device planner, the persistent
+attention kernel and the log-sum-exp merge, plus the fused prologue for the FP8
+workload. The default workload is the mixed-length batch the dynamic scheduler targets:
+1 x 131072 + 31 x 4096 tokens, 64 q / 8 kv heads, head dim 128, page 64, bf16 KV. The
+KV cache (1.06 GB) is larger than L2, so there is no flush between steps.
+
+Rank 0 prints one JSON line. ``value`` is the effective GB/s over the algorithmic bytes
+(valid KV + q + out), summed over ranks. The timed region is K eager steps on one stream,
+bracketed by a barrier and synchronize, timed with CUDA events. Under torchrun, each rank
+runs an independent replica: the workload has no cross-GPU exchange.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from load_balanced_split_step_b200 import workloads as W  # noqa: E402
+
+WORKLOAD_TEXT = {
+    "tiny": "tiny: 4 requests {17,64,200,513}, 8 q / 2 kv heads, D 64, page 16, bf16 KV",
+    "uniform": "uniform: 32 x 4096 tokens, 64 q / 8 kv heads, D 128, page 64, bf16 KV",
+    "extreme": "extreme mixed: 1 x 131072 + 31 x 4096 tokens, 64 q / 8 kv heads, D 128, page 64, bf16 KV",
+    "heavy": "heavy-tailed: 64 requests, L log-uniform [512, 65536), +1 per step over 8 steps, 64/8 heads, D 128, "
+             "page 64, bf16 KV",
+    "fp8": "large batch FP8: 256 requests, L ~ U[1024, 16384], 64/8 heads, D 128, page 64, E4M3 KV + fused "
+           "RoPE/QK-RMSNorm/KV-write prologue",
+}
+METRIC = "decode-attention KV-read GB/s (effective, algorithmic KV+Q+O bytes / step time) on mixed-length batches"
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="extreme", choices=list(WORKLOAD_TEXT))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--tile-len", type=int, default=0)
+    ap.add_argument("--ctas-per-sm", type=int, default=1)
+    ap.add_argument("--no-extras", action="store_true", help="skip static split-k, e2e and CPU baseline legs")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------------- distributed
+
+def dist_init(args):
+    """Returns (rank, world, local_rank). One process per GPU under torchrun."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+        return dist.get_rank(), world, local
+    return 0, 1, 0
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_done(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Step:
+    """One decode step through the binding, with buffers allocated once."""
+
+    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None):
+        self.B, self.spec, self.dc = B, spec, dc
+        self.tl = tile_len
+        dev = dc["seq_lens"].device
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_seq = dc["block_table"].shape[1] * spec.page_size
+        if static_splits:
+            self.plan = B.plan_static(dc["seq_lens"], spec.num_heads, spec.kv_heads, tile_len, static_splits,
+                                      self.max_seq, self.status)
+            self.static_splits = static_splits
+        else:
+            self.plan = B.plan(dc["seq_lens"], spec.num_heads, spec.kv_heads, tile_len, num_ctas, self.max_seq,
+                               self.status)
+            self.static_splits = None
+        self.num_ctas = num_ctas
+        self.po, self.pml = B.partial_buffers(self.plan, spec.num_heads, spec.head_dim, dev)
+        self.out = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.float32, device=dev)
+        self.q = dc["q"]
+        if spec.prologue:
+            self.q = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.bfloat16, device=dev)
+
+    def __call__(self, seq_lens=None, ev=None):
+        B, s, dc = self.B, self.spec, self.dc
+        seq = dc["seq_lens"] if seq_lens is None else seq_lens
+        if s.prologue:
+            B.prologue(dc["qkv"], dc["q_norm_w"], dc["k_norm_w"], dc["k_pages"], dc["v_pages"], dc["block_table"],
+                       seq, s.num_heads, s.kv_heads, kv_dtype=s.kv_dtype, k_scale=dc["k_scale"],
+                       v_scale=dc["v_scale"], eps=s.rms_eps, rope_theta=s.rope_theta, q_out=self.q,
+                       status=self.status)
+        if self.static_splits:
+            B.plan_static(seq, s.num_heads, s.kv_heads, self.tl, self.static_splits, self.max_seq, self.status,
+                          workspace=self.plan.workspace)
+        else:
+            B.plan(seq, s.num_heads, s.kv_heads, self.tl, self.num_ctas, self.max_seq, self.status,
+                   workspace=self.plan.workspace)
+        if ev is not None:
+            ev[0].record()
+        B.attention(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, self.plan, kv_dtype=s.kv_dtype,
+                    k_scale=dc["k_scale"], v_scale=dc["v_scale"], out=self.out, partial_o=self.po,
+                    partial_ml=self.pml, status=self.status)
+        if ev is not None:
+            ev[1].record()
+        B.merge(self.plan, self.po, self.pml, self.out, s.num_heads, self.status)
+        return self.out
+
+    @property
+    def launches(self):
+        return 4 if self.spec.prologue else 3
+
+
+def step_lengths(dc, spec):
+    """Device length vectors for each decode step (heavy-tailed grows by one per step)."""
+    return [dc["seq_lens"] + i for i in range(spec.steps)]
+
+
+def time_steps(step, lens, K, W_, world, kernel_events=True):
+    for i in range(W_):
+        step(lens[i % len(lens)])
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)] \
+        if kernel_events else [None] * K
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K):
+        step(lens[i % len(lens)], ev[i])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t0.elapsed_time(t1)
+    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in ev])) if kernel_events else None
+    return total_ms, kern_ms
+
+
+def static_leg(B, spec, dc, tl, steps, sms):
+    S0 = max(1, -(-2 * sms // (spec.batch * spec.kv_heads)))
+    res = {}
+    lens = step_lengths(dc, spec)
+    for S in sorted({S0, 1, 2, 4, 8, 16, 32}):
+        st = Step(B, spec, dc, None, tl, static_splits=S)
+        ms, _ = time_steps(st, lens, steps, 3, 1, kernel_events=False)
+        res[S] = 1000.0 * ms / steps
+    best = min(res, key=res.get)
+    return {"splits_rule": "S = max(1, ceil(2*SMs/(B*Hkv)))", "S": S0, "us_per_step": round(res[S0], 2),
+            "best_S": best, "best_us_per_step": round(res[best], 2),
+            "sweep_us": {str(k): round(v, 2) for k, v in res.items()}}
+
+
+def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world):
+    """Same metric through the public call with per-step H2D of the step inputs (q or qkv,
+    seq_lens, block_table) from pinned host memory and D2H of the output. The KV cache is
+    device-resident decode state and is not copied."""
+    dev = dc["seq_lens"].device
+    src = {"seq_lens": case.seq_lens.pin_memory(), "block_table": case.block_table.pin_memory()}
+    qname = "qkv" if spec.prologue else "q"
+    src[qname] = getattr(case, qname).pin_memory()
+    dst = {k: torch.empty_like(v, device=dev) for k, v in src.items()}
+    out_host = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in src.values())
+    d2h = out_host.numel() * out_host.element_size()
+    ddc = dict(dc)
+
+    def one():
+        for k in src:
+            dst[k].copy_(src[k], non_blocking=True)
+        ddc.update(dst)
+        q = ddc["q"]
+        if spec.prologue:
+            q = B.prologue(ddc["qkv"], ddc["q_norm_w"], ddc["k_norm_w"], ddc["k_pages"], ddc["v_pages"],
+                           ddc["block_table"], ddc["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype,
+                           k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], eps=spec.rms_eps,
+                           rope_theta=spec.rope_theta)
+        out, _, _ = B.decode_step(q, ddc["k_pages"], ddc["v_pages"], ddc["block_table"], ddc["seq_lens"],
+                                  spec.num_heads, spec.kv_heads, tl, kv_dtype=spec.kv_dtype, k_scale=ddc["k_scale"],
+                                  v_scale=ddc["v_scale"], num_ctas=num_ctas)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return t0.elapsed_time(t1), h2d, d2h
+
+
+def cpu_baseline(spec, case, target_s):
+    """The fp64 oracle, as it stands, over whole passes of the workload on the host cores,
+    until target_s seconds have been spent. Returns (GB/s, description, threads)."""
+    from oracle import attention as OA
+    from oracle import prologue as OR
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    bytes_step = W.algorithmic_bytes(spec)
+    # bounded sample: whole requests, drawn round-robin from the batch, until the target is met
+    order = list(range(spec.batch))
+    t0 = time.perf_counter()
+    done_bytes, n_req = 0, 0
+    per_req_kv = {r: spec.seq_lens[r] * spec.kv_heads * spec.head_dim * 2 * (1 if spec.kv_dtype == "e4m3" else 2)
+                  for r in order}
+    i = 0
+    while time.perf_counter() - t0 < target_s and n_req < 100000:
+        r = order[i % len(order)]
+        i += 1
+        if spec.prologue:
+            sub = W.extract_requests(case, [r])
+            kp, vp = sub.k_pages.numpy().copy(), sub.v_pages.numpy().copy()
+            q = OR.decode_prologue(sub.qkv, sub.q_norm_w, sub.k_norm_w, spec.rms_eps, spec.rope_theta,
+                                   sub.seq_lens.numpy(), sub.block_table.numpy(), kp, vp, spec.kv_dtype,
+                                   sub.k_scale, sub.v_scale, spec.num_heads, spec.kv_heads)[0]
+            OA.decode_attention(q, kp, vp, sub.block_table, sub.seq_lens, kv_dtype=spec.kv_dtype,
+                                k_scale=sub.k_scale, v_scale=sub.v_scale)
+        else:
+            OA.decode_attention(case.q[r:r + 1], case.k_pages, case.v_pages, case.block_table[r:r + 1],
+                                case.seq_lens[r:r + 1], kv_dtype=spec.kv_dtype, k_scale=case.k_scale,
+                                v_scale=case.v_scale)
+        done_bytes += per_req_kv[r] + spec.num_heads * spec.head_dim * 6
+        n_req += 1
+    el = time.perf_counter() - t0
+    frac = done_bytes / bytes_step
+    desc = (f"{n_req} whole requests of the workload taken round-robin "
+            f"({frac:.2f} of one step's algorithmic bytes) in {el:.1f} s")
+    return done_bytes / el / 1e9, desc, threads, el
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def load_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", f"attention_{workload}_traffic.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("traffic_bytes_per_launch")
+    return None
+
+
+def run_ours(args, rank, world, local):
+    from load_balanced_split_step_b200 import binding as B
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec = W.config_spec(args.workload)
+    case = W.make_case(spec)
+    dc = {k: (getattr(case, k).to(dev) if getattr(case, k) is not None else None)
+          for k in ("q", "qkv", "k_pages", "v_pages", "block_table", "seq_lens", "k_scale", "v_scale", "q_norm_w",
+                    "k_norm_w")}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tl = args.tile_len or spec.tile_len
+    G = sms * args.ctas_per_sm
+    step = Step(B, spec, dc, G, tl)
+    lens = step_lengths(dc, spec)
+    K, W_ = args.steps, max(3, args.warmup)
+
+    with ClockSampler(local) as clk:
+        total_ms, kern_ms = time_steps(step, lens, K, W_, world)
+    st = int(step.status.item())
+    if st:
+        raise RuntimeError(f"device status {st:#x} during the timed region")
+    total_ms = max_over_ranks(total_ms, world)
+    kern_ms = max_over_ranks(kern_ms, world)
+    bytes_step = float(np.mean([W.algorithmic_bytes(spec, i % spec.steps) for i in range(spec.steps)]))
+    value = world * bytes_step * K / (total_ms / 1e3) / 1e9
+    ms_step = total_ms / K
+    peak, peak_kind = load_peaks()
+    achieved = bytes_step / (kern_ms / 1e3) / 1e9
+    clocks = clk.summary()
+
+    extra = {}
+    if not args.no_extras:
+        # graph replay of the same step (host launch overhead removed)
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            step(lens[0])
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            step(lens[0])
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(K):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        extra["graph_us_per_step"] = round(1000.0 * a.elapsed_time(b) / K, 2)
+        del g
+        extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms)
+        extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step), 3)
+    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_steps = max(50, K // 4)
+    e2e_val = world * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        v, desc, threads, _ = cpu_baseline(spec, case, args.cpu_seconds)
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W_,
+        "ms_per_step": round(ms_step, 5), "us_per_step": round(1000 * ms_step, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if spec.kv_dtype == "bf16" else "e4m3/f16",
+        "data": "synthetic (seeded N(0,1), bf16-rounded; random page permutation)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "tile_len": tl, "num_ctas": G,
+                   "plan": "dynamic (re-planned on the device every step)",
+                   "l2": f"inputs larger than L2 ({bytes_step / 1e9:.2f} GB per step), no flush",
+                   "parallelism": f"{world} independent replica(s), no collective"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "frac_of_nominal_8000": round(achieved / 8000.0, 4),
+                     "kernel": "decode_attention_kernel", "kernel_us": round(1000 * kern_ms, 2),
+                     "traffic": load_traffic(args.workload)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_step": round(1000 * e2e_ms / e2e_steps, 2)},
+        "gpu_launches": step.launches * K,
+        "clocks": clocks,
+    }
+    line.update(extra)
+    return line
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle as it stands, timed on the host cores."""
+    if rank != 0:
+        return None
+    spec = W.config_spec(args.workload)
+    case = W.make_case(spec)
+    K, W_ = max(1, min(args.steps, 3)), 0
+    target = args.cpu_seconds
+    vals, descs, threads = [], [], 1
+    for _ in range(K):
+        v, desc, threads, _ = cpu_baseline(spec, case, target / K)
+        vals.append(v)
+        descs.append(desc)
+    v = float(np.mean(vals))
+    bytes_step = W.algorithmic_bytes(spec)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": W_, "ms_per_step": round(1000 * bytes_step / (v * 1e9), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "tile_len": spec.tile_len, "plan": "none (exact)",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": descs[0]},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_init(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

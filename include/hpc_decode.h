@@ -1,0 +1,234 @@
+/*
+ * hpc_decode.h: C ABI of libhpcdecode.so, load-balanced split-KV decode attention for
+ * B200 (sm_100a).
+ *
+ * One decode step runs four stages, all asynchronous on the caller's stream:
+ *
+ *   hpc_decode_prologue   (optional) RMSNorm + RoPE on the new token's q and k, and the
+ *                         K/V page write of the new token;
+ *   hpc_decode_plan       the per-step tile planner (a device kernel; no host sync);
+ *   hpc_decode_attention  the persistent attention kernel; it consumes the plan;
+ *   hpc_merge_states      the log-sum-exp merge of split (request, kv head) pairs.
+ *
+ * Sources: "Tencent HPC llega a SGLang y desafía a los kernels de inferencia
+ * predeterminados" (remio.ai), section "Por qué Tencent HPC importa para el serving de
+ * modelos en línea": uniform KV tiles spread over CTAs by current load, and a mapping
+ * rebuilt as lengths change. "腾讯混元三算子杀入 SGLang" (AREX), Dynamic Attention
+ * paragraph under "Router GEMM：精度不丢，速度翻三倍": a persistent kernel that assigns
+ * tiles every decode step by actual KV length. "vLLM × HPC-Ops: High-Performance
+ * Attention and MoE Backends from Tencent Hunyuan" (8sync News summary): a fused
+ * RoPE + QK-Norm + KV-write prologue, and a dynamic scheduler that replaces fixed
+ * split-KV.
+ *
+ * Conventions, for every entry point:
+ *  - Ownership: the caller owns every buffer. Device pointers must point to memory of
+ *    the current CUDA device. The library allocates no device memory and never
+ *    synchronises the stream.
+ *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Return value: hpc_status. A non-zero return means nothing was launched. Host-
+ *    checkable problems are reported this way: null pointers, unsupported shapes or
+ *    dtypes, misaligned pointers, too-small workspaces, launch failures.
+ *    hpc_last_error() gives a message for the calling thread.
+ *  - Device-detected problems are OR-ed into the caller's device word *status (uint32,
+ *    HPC_DEV_* bits). These depend on data the host does not read: seq_lens, page
+ *    ids, and wait timeouts. The kernels never trap. After a non-zero status the
+ *    outputs of the affected requests are unspecified (but no out-of-bounds access
+ *    happens). Clear *status before the step.
+ *  - Cache layout (HND): k_pages / v_pages are [num_pages][kv_heads][page_size][head_dim],
+ *    row-major, with elements bf16 or E4M3 codes. block_table is int32
+ *    [batch][max_pages_per_req]. block_table[r][j] is the page that holds tokens
+ *    [j*page_size, (j+1)*page_size) of request r. seq_lens is int32 [batch]: the number
+ *    of valid tokens, including the one being decoded.
+ *  - Query head h reads kv head h / (num_heads / kv_heads) (contiguous GQA groups).
+ */
+#ifndef HPC_DECODE_H_
+#define HPC_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HPC_DECODE_ABI_VERSION 1
+
+/* Symbols of the library are hidden by default; the entry points below are exported. */
+#if defined(__GNUC__)
+#define HPC_API __attribute__((visibility("default")))
+#else
+#define HPC_API
+#endif
+
+typedef enum {
+  HPC_OK = 0,
+  HPC_ERR_ARG = 1,      /* null pointer or out-of-range scalar argument */
+  HPC_ERR_SHAPE = 2,    /* unsupported head_dim / page_size / tile_len / group size */
+  HPC_ERR_DTYPE = 3,    /* unsupported dtype combination */
+  HPC_ERR_ALIGN = 4,    /* a pointer is not 16-byte aligned */
+  HPC_ERR_CUDA = 5,     /* a CUDA runtime/driver call failed */
+  HPC_ERR_CAPACITY = 6  /* a caller buffer is smaller than required */
+} hpc_status;
+
+typedef enum { HPC_BF16 = 0, HPC_FP32 = 1, HPC_E4M3 = 2 } hpc_dtype;
+
+/* Bits the kernels OR into the caller's device status word. */
+#define HPC_DEV_BAD_SEQLEN 0x1u /* seq_len < 0 or > max tokens; the request gets no tiles and a zero output */
+#define HPC_DEV_BAD_PAGE 0x2u   /* a block_table entry outside [0, num_pages); reads there return zeros */
+#define HPC_DEV_CAPACITY 0x4u   /* more work items than the plan can hold (cannot happen for a valid plan) */
+#define HPC_DEV_TIMEOUT 0x8u    /* a bounded pipeline wait expired; the kernel gave up and returned */
+
+/* One unit of a CTA's work: tiles [tile_begin, tile_end) of one (request, kv head). */
+typedef struct {
+  int32_t req;
+  int16_t kv_head;
+  int16_t flags; /* HPC_ITEM_DIRECT: the item covers its whole (req, kv_head); the attention
+                    kernel writes the final output for it, with no partial state or merge */
+  int32_t tile_begin;
+  int32_t tile_end;
+} hpc_work_item;
+
+#define HPC_ITEM_DIRECT 1
+
+/* A plan is a host struct of device pointers into one caller-owned workspace. Layout:
+ *   counts       int64[4]             n_items, n_merge, n_units, chunk (written on the device)
+ *   items        hpc_work_item[max_items]
+ *   cta_indptr   int32[num_ctas + 1]  CTA g owns items [cta_indptr[g], cta_indptr[g+1])
+ *   merge_indptr int32[batch*kv_heads + 1]  items of segment s = r*kv_heads + kvh are
+ *                                      [merge_indptr[s], merge_indptr[s+1]) (contiguous)
+ *   merge_list   int32[batch*kv_heads] segments whose item count != 1 (first n_merge valid)
+ * Item k writes partial slot k. */
+typedef struct {
+  int32_t batch, kv_heads, tile_len, num_ctas, max_items, merge_capacity, is_static, reserved;
+  int64_t* counts;
+  hpc_work_item* items;
+  int32_t* cta_indptr;
+  int32_t* merge_indptr;
+  int32_t* merge_list;
+} hpc_plan;
+
+/* ---- planning ------------------------------------------------------------------------ */
+
+/* Bytes of workspace a dynamic plan needs (max_items = num_ctas + batch*kv_heads). */
+HPC_API size_t hpc_plan_workspace_bytes(int32_t batch, int32_t kv_heads, int32_t num_ctas);
+
+/* Bytes of workspace a static split-k plan needs (num_ctas = batch*kv_heads*splits). */
+HPC_API size_t hpc_plan_static_workspace_bytes(int32_t batch, int32_t kv_heads, int32_t splits);
+
+/* The load-balanced per-step planner (remio "Por qué …"; AREX Dynamic Attention paragraph).
+ * It runs as one device kernel on `stream` and reads seq_lens from device memory.
+ * For request r, nt_r = ceil(L_r / tile_len) tiles per kv head. Units are enumerated
+ * request-major, then kv head, then tile: T units in total. With chunk = ceil(T / num_ctas),
+ * CTA g owns units [g*chunk, min((g+1)*chunk, T)), cut into items at (request, kv head)
+ * boundaries.
+ *   seq_lens:    device int32 [batch].
+ *   num_heads:   query heads; must be a multiple of kv_heads (checked only).
+ *   tile_len:    tokens per tile, a multiple of 16.
+ *   num_ctas:    persistent CTAs, normally (#SMs x resident CTAs per SM).
+ *   max_seq_len: L_r above this (or below 0) sets HPC_DEV_BAD_SEQLEN and plans no tiles
+ *                for r (<= 0: no upper check).
+ *   workspace:   device buffer of >= hpc_plan_workspace_bytes(), 256-byte aligned.
+ *   plan:        host struct filled with pointers into workspace. The attention and merge
+ *                calls read it.
+ *   status:      device uint32 status word. */
+HPC_API int hpc_decode_plan(const int32_t* seq_lens, int32_t batch, int32_t num_heads, int32_t kv_heads,
+                    int32_t tile_len, int32_t num_ctas, int32_t max_seq_len, void* workspace,
+                    size_t workspace_bytes, hpc_plan* plan, uint32_t* status, void* stream);
+
+/* Static split-k plan: the fixed split that remio ("Por qué …") describes as leaving units
+ * idle or launching empty chunks for short requests. CTA (r*kv_heads + kvh)*splits + j takes
+ * tiles [j*ceil(nt/splits), min((j+1)*ceil(nt/splits), nt)) of (r, kvh), possibly none.
+ * num_ctas of the plan = batch*kv_heads*splits. The attention kernel runs it unchanged,
+ * one launch wave per CTA group. Arguments as hpc_decode_plan. */
+HPC_API int hpc_decode_plan_static(const int32_t* seq_lens, int32_t batch, int32_t num_heads, int32_t kv_heads,
+                           int32_t tile_len, int32_t splits, int32_t max_seq_len, void* workspace,
+                           size_t workspace_bytes, hpc_plan* plan, uint32_t* status, void* stream);
+
+/* Host twin of hpc_decode_plan. It reads seq_lens from host memory and writes the same
+ * bytes into a host buffer of hpc_plan_workspace_bytes(). *status is a host word.
+ * plan receives host pointers. */
+HPC_API int hpc_plan_cpu(const int32_t* seq_lens, int32_t batch, int32_t num_heads, int32_t kv_heads,
+                 int32_t tile_len, int32_t num_ctas, int32_t max_seq_len, void* workspace,
+                 size_t workspace_bytes, hpc_plan* plan, uint32_t* status);
+
+/* ---- attention ----------------------------------------------------------------------- */
+
+/* Bytes of partial state a plan needs: partial_o is float[max_items][group][head_dim],
+ * partial_ml is float[max_items][group][2] (m, l). group = num_heads / kv_heads. */
+HPC_API size_t hpc_partial_o_bytes(const hpc_plan* plan, int32_t num_heads, int32_t head_dim);
+HPC_API size_t hpc_partial_ml_bytes(const hpc_plan* plan, int32_t num_heads);
+
+/* Persistent split-KV decode attention (AREX Dynamic Attention paragraph).
+ * grid = plan->num_ctas CTAs. Each CTA streams its items' KV pages through a shared-memory
+ * ring filled by TMA, with tensor-core QK^T and PV on the GQA group.
+ *   q:        device bf16 [batch][num_heads][head_dim].
+ *   k_pages, v_pages: device cache, see the layout above. kv_dtype is HPC_BF16 or HPC_E4M3.
+ *             Base addresses must be 16-byte aligned.
+ *   k_scale, v_scale: device float [kv_heads], required for HPC_E4M3 (value = code * scale),
+ *             ignored for HPC_BF16.
+ *   page_size: 16, 32, 64 or 128.  head_dim: 64 or 128 for bf16, 128 for E4M3.
+ *   num_heads / kv_heads in {1, 2, 4, 8}.
+ *   plan:     from hpc_decode_plan(_static) for the same seq_lens; its tile_len must be a
+ *             multiple of page_size or divide it.
+ *   sm_scale: score scale, normally 1/sqrt(head_dim).
+ *   partial_o, partial_ml: device scratch of hpc_partial_*_bytes(). Non-DIRECT item k
+ *             writes slot k with natural-log state m = max score, l = sum exp(s - m),
+ *             o = sum exp(s - m) v.
+ *   out:      device [batch][num_heads][head_dim], out_dtype HPC_FP32 or HPC_BF16. DIRECT
+ *             items write it here; hpc_merge_states writes the rest. */
+HPC_API int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                         const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                         int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                         int32_t max_pages_per_req, const int32_t* seq_lens, const hpc_plan* plan,
+                         float sm_scale, float* partial_o, float* partial_ml, void* out,
+                         hpc_dtype out_dtype, uint32_t* status, void* stream);
+
+/* ---- merge --------------------------------------------------------------------------- */
+
+/* Log-sum-exp merge of the partial states of every (request, kv head) that the plan split
+ * across items: M = max m_i, L = sum exp(m_i - M) l_i, out = sum exp(m_i - M) o_i / L.
+ * A (request, kv head) with no items (L_r = 0) gets a zero output. Arguments as in
+ * hpc_decode_attention. */
+HPC_API int hpc_merge_states(const float* partial_o, const float* partial_ml, const hpc_plan* plan,
+                     int32_t num_heads, int32_t head_dim, void* out, hpc_dtype out_dtype,
+                     uint32_t* status, void* stream);
+
+/* ---- prologue ------------------------------------------------------------------------ */
+
+/* Fused decode prologue (vllm summary: "RoPE + QK-Norm + KV-write"). For each request r
+ * with pos = seq_lens[r] - 1:
+ *   q heads:  RMSNorm (q_norm_w, eps), then NeoX RoPE at pos (pairs (i, i+D/2),
+ *             angle pos * theta^(-2i/D), computed in fp64), written as bf16 to q_out.
+ *   k heads:  RMSNorm (k_norm_w), RoPE, then stored to page block_table[r][pos/page_size],
+ *             slot pos % page_size, as bf16 or as E4M3 code of x / k_scale[g] (RNE,
+ *             saturating to +-448).
+ *   v heads:  stored as is (bf16) or as E4M3 of v / v_scale[g].
+ *   qkv:      device bf16 [batch][num_heads + 2*kv_heads][head_dim] (q heads, then k, then v).
+ *   q_norm_w, k_norm_w: device float [head_dim].
+ *   q_out:    device bf16 [batch][num_heads][head_dim].
+ * seq_lens[r] < 1 or beyond the block table sets HPC_DEV_BAD_SEQLEN, and request r's
+ * q_out row is zeroed. */
+HPC_API int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,
+                        float rope_theta, void* q_out, void* k_pages, void* v_pages, hpc_dtype kv_dtype,
+                        const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                        const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
+                        int32_t batch, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
+                        uint32_t* status, void* stream);
+
+/* ---- misc ---------------------------------------------------------------------------- */
+
+/* Launch shape the attention kernel would use: pipeline stages, dynamic shared memory
+ * bytes and threads per CTA. For introspection and benchmarking. */
+HPC_API int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, int32_t page_size, int32_t tile_len,
+                              int32_t ctas_per_sm, int32_t* stages, int32_t* smem_bytes,
+                              int32_t* threads);
+
+HPC_API const char* hpc_status_string(int status);
+HPC_API const char* hpc_last_error(void); /* message of the calling thread's last failure ("" if none) */
+HPC_API int hpc_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HPC_DECODE_H_ */

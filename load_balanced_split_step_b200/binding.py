@@ -1,0 +1,325 @@
+"""Thin Python binding of libhpcdecode.so (C ABI declared in include/hpc_decode.h).
+
+This module only marshals arguments. It checks tensor dtypes and devices and passes
+``data_ptr()`` and the current CUDA stream to the library. Every step of the decode path
+runs in the library's kernels. If the library is missing, importing this module raises
+``HpcError``: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from .build import LIB
+
+HPC_OK, HPC_ERR_ARG, HPC_ERR_SHAPE, HPC_ERR_DTYPE, HPC_ERR_ALIGN, HPC_ERR_CUDA, HPC_ERR_CAPACITY = range(7)
+HPC_BF16, HPC_FP32, HPC_E4M3 = 0, 1, 2
+DEV_STATUS = {"bad_seqlen": 0x1, "bad_page": 0x2, "capacity": 0x4, "timeout": 0x8}
+ITEM_DTYPE = np.dtype([("req", "<i4"), ("kv_head", "<i2"), ("flags", "<i2"),
+                       ("tile_begin", "<i4"), ("tile_end", "<i4")])
+
+EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_decode_plan",
+           "hpc_decode_plan_static", "hpc_plan_cpu", "hpc_partial_o_bytes", "hpc_partial_ml_bytes",
+           "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue", "hpc_attention_launch_info",
+           "hpc_status_string", "hpc_last_error", "hpc_abi_version")
+
+
+class HpcError(RuntimeError):
+    pass
+
+
+class CPlan(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("kv_heads", ctypes.c_int32), ("tile_len", ctypes.c_int32),
+                ("num_ctas", ctypes.c_int32), ("max_items", ctypes.c_int32), ("merge_capacity", ctypes.c_int32),
+                ("is_static", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("counts", ctypes.c_void_p), ("items", ctypes.c_void_p), ("cta_indptr", ctypes.c_void_p),
+                ("merge_indptr", ctypes.c_void_p), ("merge_list", ctypes.c_void_p)]
+
+
+def library_path() -> str:
+    return LIB
+
+
+def _load():
+    if not os.path.exists(LIB):
+        raise HpcError(f"{LIB} is missing; build it with `python -m load_balanced_split_step_b200.build` "
+                       "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB)
+    i32, vp, sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+    fp = ctypes.c_float
+    P = ctypes.POINTER(CPlan)
+    sig = {
+        "hpc_plan_workspace_bytes": (sz, [i32, i32, i32]),
+        "hpc_plan_static_workspace_bytes": (sz, [i32, i32, i32]),
+        "hpc_decode_plan": (ctypes.c_int, [vp, i32, i32, i32, i32, i32, i32, vp, sz, P, vp, vp]),
+        "hpc_decode_plan_static": (ctypes.c_int, [vp, i32, i32, i32, i32, i32, i32, vp, sz, P, vp, vp]),
+        "hpc_plan_cpu": (ctypes.c_int, [vp, i32, i32, i32, i32, i32, i32, vp, sz, P, vp]),
+        "hpc_partial_o_bytes": (sz, [P, i32, i32]),
+        "hpc_partial_ml_bytes": (sz, [P, i32]),
+        "hpc_decode_attention": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp, i32,
+                                                vp, P, fp, vp, vp, vp, ctypes.c_int, vp, vp]),
+        "hpc_merge_states": (ctypes.c_int, [vp, vp, P, i32, i32, vp, ctypes.c_int, vp, vp]),
+        "hpc_decode_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, vp,
+                                               i32, vp, i32, i32, i32, i32, vp, vp]),
+        "hpc_attention_launch_info": (ctypes.c_int, [i32, ctypes.c_int, i32, i32, i32, ctypes.POINTER(i32),
+                                                     ctypes.POINTER(i32), ctypes.POINTER(i32)]),
+        "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hpc_last_error": (ctypes.c_char_p, []),
+        "hpc_abi_version": (ctypes.c_int, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    return lib
+
+
+_lib = _load()
+
+
+def status_string(code: int) -> str:
+    return _lib.hpc_status_string(code).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != HPC_OK:
+        raise HpcError(f"{what}: {status_string(rc)} ({rc}): {_lib.hpc_last_error().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None, cuda=True):
+    if not isinstance(t, torch.Tensor):
+        raise HpcError(f"{name} must be a torch.Tensor")
+    if cuda and not t.is_cuda:
+        raise HpcError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise HpcError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise HpcError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise HpcError(f"{name} must be contiguous")
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+@dataclass
+class Plan:
+    """A plan bound to its workspace. ``raw`` is the C struct passed to the library."""
+
+    raw: CPlan
+    workspace: torch.Tensor
+    host: bool = False
+
+    @property
+    def num_ctas(self) -> int:
+        return int(self.raw.num_ctas)
+
+    @property
+    def max_items(self) -> int:
+        return int(self.raw.max_items)
+
+    def _view(self, ptr, dtype, count):
+        base = self.workspace.data_ptr()
+        off = int(ptr) - base
+        nbytes = np.dtype(dtype).itemsize * count
+        return self.workspace[off:off + nbytes]
+
+    def to_numpy(self) -> dict:
+        """Copy the plan to host: counts, the valid items, and the index arrays."""
+        r = self.raw
+        counts = self._view(r.counts, np.int64, 4).cpu().numpy().view(np.int64)
+        n_items, n_merge = int(counts[0]), int(counts[1])
+        items = self._view(r.items, ITEM_DTYPE, n_items).cpu().numpy().view(ITEM_DTYPE)
+        segs = r.batch * r.kv_heads
+        return {
+            "n_items": n_items, "n_merge": n_merge, "n_units": int(counts[2]), "chunk": int(counts[3]),
+            "items": items,
+            "cta_indptr": self._view(r.cta_indptr, np.int32, r.num_ctas + 1).cpu().numpy().view(np.int32),
+            "merge_indptr": self._view(r.merge_indptr, np.int32, segs + 1).cpu().numpy().view(np.int32),
+            "merge_list": self._view(r.merge_list, np.int32, n_merge).cpu().numpy().view(np.int32),
+        }
+
+
+def plan(seq_lens: torch.Tensor, num_heads: int, kv_heads: int, tile_len: int, num_ctas: int | None = None,
+         max_seq_len: int = 0, status: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> Plan:
+    """Load-balanced per-step plan on the device (``hpc_decode_plan``)."""
+    _need(seq_lens, "seq_lens", torch.int32)
+    dev = seq_lens.device
+    if num_ctas is None:
+        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    B = seq_lens.numel()
+    nbytes = _lib.hpc_plan_workspace_bytes(B, kv_heads, num_ctas)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    raw = CPlan()
+    _check(_lib.hpc_decode_plan(_ptr(seq_lens), B, num_heads, kv_heads, tile_len, num_ctas, max_seq_len,
+                                _ptr(workspace), workspace.numel(), ctypes.byref(raw), _ptr(status),
+                                _stream(dev)), "hpc_decode_plan")
+    return Plan(raw, workspace)
+
+
+def plan_static(seq_lens: torch.Tensor, num_heads: int, kv_heads: int, tile_len: int, splits: int,
+                max_seq_len: int = 0, status: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None) -> Plan:
+    """Static split-k plan on the device (``hpc_decode_plan_static``)."""
+    _need(seq_lens, "seq_lens", torch.int32)
+    dev = seq_lens.device
+    B = seq_lens.numel()
+    nbytes = _lib.hpc_plan_static_workspace_bytes(B, kv_heads, splits)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    status = new_status(dev) if status is None else status
+    raw = CPlan()
+    _check(_lib.hpc_decode_plan_static(_ptr(seq_lens), B, num_heads, kv_heads, tile_len, splits, max_seq_len,
+                                       _ptr(workspace), workspace.numel(), ctypes.byref(raw), _ptr(status),
+                                       _stream(dev)), "hpc_decode_plan_static")
+    return Plan(raw, workspace)
+
+
+def plan_host(seq_lens, num_heads: int, kv_heads: int, tile_len: int, num_ctas: int,
+              max_seq_len: int = 0) -> tuple[Plan, int]:
+    """Host twin of ``plan`` (``hpc_plan_cpu``). Returns (plan, status word)."""
+    lens = torch.as_tensor(seq_lens, dtype=torch.int32).contiguous().cpu()
+    B = lens.numel()
+    nbytes = _lib.hpc_plan_workspace_bytes(B, kv_heads, num_ctas)
+    # 256-byte aligned host buffer
+    buf = torch.empty(nbytes + 256, dtype=torch.uint8)
+    off = (-buf.data_ptr()) % 256
+    ws = buf[off:off + nbytes]
+    st = ctypes.c_uint32(0)
+    raw = CPlan()
+    _check(_lib.hpc_plan_cpu(_ptr(lens), B, num_heads, kv_heads, tile_len, num_ctas, max_seq_len, _ptr(ws),
+                             nbytes, ctypes.byref(raw), ctypes.byref(st)), "hpc_plan_cpu")
+    p = Plan(raw, ws, host=True)
+    p._keep = buf
+    return p, int(st.value)
+
+
+def partial_buffers(p: Plan, num_heads: int, head_dim: int, device):
+    no = _lib.hpc_partial_o_bytes(ctypes.byref(p.raw), num_heads, head_dim) // 4
+    nml = _lib.hpc_partial_ml_bytes(ctypes.byref(p.raw), num_heads) // 4
+    return (torch.empty(max(no, 4), dtype=torch.float32, device=device),
+            torch.empty(max(nml, 4), dtype=torch.float32, device=device))
+
+
+_KV_DTYPES = {"bf16": HPC_BF16, "e4m3": HPC_E4M3}
+
+
+def _kv_code(kv_dtype: str, t: torch.Tensor) -> int:
+    if kv_dtype not in _KV_DTYPES:
+        raise HpcError(f"kv_dtype must be one of {list(_KV_DTYPES)}")
+    want = (torch.bfloat16,) if kv_dtype == "bf16" else (torch.uint8, torch.float8_e4m3fn)
+    if t.dtype not in want:
+        raise HpcError(f"cache dtype {t.dtype} does not match kv_dtype {kv_dtype}")
+    return _KV_DTYPES[kv_dtype]
+
+
+def attention(q, k_pages, v_pages, block_table, seq_lens, p: Plan, *, kv_dtype="bf16", k_scale=None,
+              v_scale=None, sm_scale=None, out=None, out_dtype=torch.float32, partial_o=None, partial_ml=None,
+              status=None):
+    """Persistent split-KV attention (``hpc_decode_attention``). Returns (out, partial_o, partial_ml)."""
+    _need(q, "q", torch.bfloat16)
+    dev = q.device
+    for name, t in (("k_pages", k_pages), ("v_pages", v_pages)):
+        _need(t, name, device=dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    code = _kv_code(kv_dtype, k_pages)
+    _kv_code(kv_dtype, v_pages)
+    B, Hq, D = q.shape
+    num_pages, Hkv, P, D2 = k_pages.shape
+    if D2 != D or v_pages.shape != k_pages.shape:
+        raise HpcError("cache shape does not match q")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
+    _need(out, "out", (torch.float32, torch.bfloat16), dev)
+    if partial_o is None or partial_ml is None:
+        partial_o, partial_ml = partial_buffers(p, Hq, D, dev)
+    status = new_status(dev) if status is None else status
+    if code == HPC_E4M3:
+        _need(k_scale, "k_scale", torch.float32, dev)
+        _need(v_scale, "v_scale", torch.float32, dev)
+    scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    _check(_lib.hpc_decode_attention(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), ctypes.byref(p.raw), scale, _ptr(partial_o),
+        _ptr(partial_ml), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
+        _stream(dev)), "hpc_decode_attention")
+    return out, partial_o, partial_ml
+
+
+def merge(p: Plan, partial_o, partial_ml, out, num_heads: int, status=None):
+    """Log-sum-exp merge of split (request, kv head) pairs (``hpc_merge_states``)."""
+    dev = out.device
+    _need(partial_o, "partial_o", torch.float32, dev)
+    _need(partial_ml, "partial_ml", torch.float32, dev)
+    _need(out, "out", (torch.float32, torch.bfloat16), dev)
+    status = new_status(dev) if status is None else status
+    D = out.shape[-1]
+    _check(_lib.hpc_merge_states(_ptr(partial_o), _ptr(partial_ml), ctypes.byref(p.raw), num_heads, D, _ptr(out),
+                                 HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
+                                 _stream(dev)), "hpc_merge_states")
+    return out
+
+
+def prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, *,
+             kv_dtype="bf16", k_scale=None, v_scale=None, eps=1e-6, rope_theta=1e6, q_out=None, status=None):
+    """Fused RMSNorm + RoPE + KV-page write of the new token (``hpc_decode_prologue``). Returns q_out."""
+    _need(qkv, "qkv", torch.bfloat16)
+    dev = qkv.device
+    _need(q_norm_w, "q_norm_w", torch.float32, dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    code = _kv_code(kv_dtype, k_pages)
+    B, H, D = qkv.shape
+    if H != num_heads + 2 * kv_heads:
+        raise HpcError("qkv must hold num_heads + 2*kv_heads heads")
+    num_pages, Hkv, P, _ = k_pages.shape
+    if q_out is None:
+        q_out = torch.empty((B, num_heads, D), dtype=torch.bfloat16, device=dev)
+    status = new_status(dev) if status is None else status
+    _check(_lib.hpc_decode_prologue(
+        _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(q_out), _ptr(k_pages),
+        _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, _ptr(block_table), block_table.shape[1],
+        _ptr(seq_lens), B, num_heads, kv_heads, D, _ptr(status), _stream(dev)), "hpc_decode_prologue")
+    return q_out
+
+
+def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",
+                k_scale=None, v_scale=None, num_ctas=None, out=None, out_dtype=torch.float32, status=None,
+                static_splits=None):
+    """plan -> attention -> merge for one decode step; returns (out, plan, status)."""
+    dev = q.device
+    status = new_status(dev) if status is None else status
+    max_seq = block_table.shape[1] * k_pages.shape[2]
+    if static_splits:
+        p = plan_static(seq_lens, num_heads, kv_heads, tile_len, static_splits, max_seq, status)
+    else:
+        p = plan(seq_lens, num_heads, kv_heads, tile_len, num_ctas, max_seq, status)
+    out, po, pml = attention(q, k_pages, v_pages, block_table, seq_lens, p, kv_dtype=kv_dtype, k_scale=k_scale,
+                             v_scale=v_scale, out=out, out_dtype=out_dtype, status=status)
+    merge(p, po, pml, out, num_heads, status)
+    return out, p, status
+
+
+def launch_info(head_dim, kv_dtype, page_size, tile_len, ctas_per_sm=1):
+    st, sm, th = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.hpc_attention_launch_info(head_dim, _KV_DTYPES[kv_dtype], page_size, tile_len, ctas_per_sm,
+                                          ctypes.byref(st), ctypes.byref(sm), ctypes.byref(th)),
+           "hpc_attention_launch_info")
+    return {"stages": st.value, "smem_bytes": sm.value, "threads": th.value}

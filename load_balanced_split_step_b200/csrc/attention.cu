@@ -1,0 +1,582 @@
+// Persistent split-KV decode attention for sm_100a.
+//
+// "腾讯混元三算子杀入 SGLang" (AREX), Dynamic Attention paragraph under "Router GEMM：精度不丢，
+// 速度翻三倍": a persistent kernel takes the tiles that the per-step plan assigns by actual KV
+// length. Each CTA runs its items (request, kv head, tile range) back to back. An item
+// that covers a whole (request, kv head) writes the final output. Any other item writes
+// its partial softmax state (m, l, o) for the log-sum-exp merge.
+//
+// Design for B200. The kernel is bound by HBM bandwidth: 8 flop per byte of bf16 K+V,
+// against a tensor-core ridge near 250 flop/B.
+//  * Warp 8 is the producer. One lane streams each (page, kv head) block of K and V into
+//    a ring of shared-memory stages with 4-D TMA tensor loads (SWIZZLE_128B). Each stage
+//    completes on an mbarrier with the transferred byte count. Whole pages travel as a
+//    few bulk copies, with an evict-first L2 policy: each byte is read once.
+//  * Warps 0..7 are consumers. They take 16-token blocks of the stream round-robin. Each
+//    keeps its own online-softmax state for the GQA group of the item's kv head.
+//  * QK^T runs as S^T = K * Q^T on mma.m16n8k16: M = 16 tokens, N = 8 query heads, K = head
+//    dim. PV runs as O^T = V^T * P^T: M = 16 head-dim rows, N = 8 heads, K = 16 tokens. Both
+//    shapes fit the group without padding. The S^T accumulator becomes the P^T operand
+//    through two movmatrix transposes. The 128-byte swizzle keeps ldmatrix free of bank
+//    conflicts.
+//  * E4M3 cache: codes are widened to f16 in registers (cvt.f16x2.e4m3x2, exact). V needs
+//    the k = token orientation: it is loaded untransposed and transposed with movmatrix
+//    after widening. k_scale folds into the score scale, v_scale into the output.
+//  * At the end of an item, the 8 consumer warps merge their states through shared memory.
+//  * Every wait is bounded (2 s). On expiry the kernel sets HPC_DEV_TIMEOUT, stops waiting,
+//    drains its outstanding copies (bounded too) and returns.
+#include <math.h>
+
+#include <mutex>
+
+#include "hpc_common.cuh"
+
+namespace hpc {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxStages = 8;
+constexpr int kSmemLimit = 232448;  // 227 KB per block on sm_100
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnParams {
+  const __nv_bfloat16* q;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const hpc_work_item* items;
+  const int32_t* cta_indptr;
+  const float* k_scale;
+  const float* v_scale;
+  float* partial_o;
+  float* partial_ml;
+  void* out;
+  uint32_t* status;
+  int64_t max_pages;
+  int32_t num_pages, page_size, tile_len, chunk_tokens, num_heads, group;
+  int32_t stages, out_bf16;
+  uint32_t plane_bytes, stage_bytes;
+  float score_scale;  // sm_scale * log2(e)
+};
+
+template <int D, bool FP8>
+struct Shape {
+  static constexpr int kElt = FP8 ? 1 : 2;
+  static constexpr int kPlanes = D * kElt / 128;  // 128-byte swizzle planes per token row
+  static constexpr int kRedStride = D + 4;        // floats per (warp, head) row of the reduce buffer
+};
+
+// Output row index of accumulator register `half` (0: c0/c1, 1: c2/c3) for lane row g
+// inside a 16-row block. bf16 V comes from ldmatrix.trans in natural order. E4M3 V comes
+// from movmatrix in pairs: rows g -> 4*(g/2) + g%2, and the second half two further on.
+template <bool FP8>
+__device__ __forceinline__ int out_row(int g, int half) {
+  if (FP8) return 4 * (g >> 1) + (g & 1) + 2 * half;
+  return g + 8 * half;
+}
+
+// One past the last token of an item: its last tile, clipped to the request length and to
+// what the block table can address (a plan built for other lengths cannot read past it).
+__device__ __forceinline__ int64_t item_end(const hpc_work_item& w, int32_t L, int tl, int64_t capacity) {
+  int64_t e = static_cast<int64_t>(w.tile_end) * tl;
+  if (e > L) e = L;
+  if (e > capacity) e = capacity;
+  return e;
+}
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            const AttnParams p) {
+  using S = Shape<D, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int stages = p.stages;
+  uint8_t* ring = smem;
+  float* red_o = reinterpret_cast<float*>(smem + static_cast<size_t>(stages) * p.stage_bytes);
+  float* red_m = red_o + kConsumerWarps * 8 * S::kRedStride;
+  float* red_l = red_m + kConsumerWarps * 8;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * 8);  // full[stages], empty[stages]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ring_u32 = smem_u32(ring);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + stages);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int it_begin = p.cta_indptr[blockIdx.x], it_end = p.cta_indptr[blockIdx.x + 1];
+  const int C = p.chunk_tokens;
+  const int tl = p.tile_len, P = p.page_size;
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------------ producer
+    if (lane != 0) return;
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    const uint64_t policy = l2_policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    uint32_t bad = 0;
+    for (int it = it_begin; it < it_end && ok; ++it) {
+      const hpc_work_item w = p.items[it];
+      const int32_t L = p.seq_lens[w.req];
+      const int64_t tok0 = static_cast<int64_t>(w.tile_begin) * tl;
+      const int64_t tok1 = item_end(w, L, tl, p.max_pages * P);
+      const int32_t* bt = p.block_table + w.req * p.max_pages;
+      for (int64_t t = tok0; t < tok1; t += C) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
+          ok = false;
+          bad |= HPC_DEV_TIMEOUT;
+          break;
+        }
+        const int32_t page = bt[t / P];
+        const int32_t off = static_cast<int32_t>(t % P);
+        if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
+        const uint32_t full = full0 + 8 * stage;
+        const uint32_t dst = ring_u32 + stage * p.stage_bytes;
+        mbar_arrive_expect_tx(full, p.stage_bytes);
+#pragma unroll
+        for (int pl = 0; pl < S::kPlanes; ++pl)
+          tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, w.kv_head, page, policy);
+#pragma unroll
+        for (int pl = 0; pl < S::kPlanes; ++pl)
+          tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off, w.kv_head,
+                      page, policy);
+        ++issued;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    // Drain: the last fill of every slot must have landed before the CTA may exit.
+    const int64_t n = issued < stages ? issued : stages;
+    for (int64_t k = 1; k <= n; ++k) {
+      int s = stage - static_cast<int>(k);
+      uint32_t ph = phase;
+      if (s < 0) {
+        s += stages;
+        ph ^= 1;
+      }
+      if (!mbar_wait(full0 + 8 * s, ph)) bad |= HPC_DEV_TIMEOUT;
+    }
+    if (bad) atomicOr(p.status, bad);
+    return;
+  }
+
+  // -------------------------------------------------------------------- consumers
+  const int g = lane >> 2, c = lane & 3;  // MMA fragment row / column pair
+  constexpr int KSTEPS = D / 16;
+  int stage = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+
+  for (int it = it_begin; it < it_end; ++it) {
+    const hpc_work_item w = p.items[it];
+    const int32_t L = p.seq_lens[w.req];
+    const int64_t tok0 = static_cast<int64_t>(w.tile_begin) * tl;
+    const int64_t tok1 = item_end(w, L, tl, p.max_pages * P);
+    const int kvh = w.kv_head;
+    const int head0 = kvh * p.group;
+
+    // Q^T fragments (B operand): lane (g, c) holds query head head0 + g.
+    uint32_t qf[KSTEPS][2];
+    {
+      const bool live = g < p.group;
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          p.q + (static_cast<int64_t>(w.req) * p.num_heads + head0 + (live ? g : 0)) * D);
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        if (!FP8) {
+          qf[ks][0] = live ? qrow[8 * ks + c] : 0u;
+          qf[ks][1] = live ? qrow[8 * ks + 4 + c] : 0u;
+        } else {
+          // k-slots (2c, 2c+1) and (8+2c, 9+2c) of chunk ks hold d = 16ks + 4c + {0,1} and {2,3}
+          qf[ks][0] = live ? bf16x2_to_f16x2(qrow[8 * ks + 2 * c]) : 0u;
+          qf[ks][1] = live ? bf16x2_to_f16x2(qrow[8 * ks + 2 * c + 1]) : 0u;
+        }
+      }
+    }
+    float score_scale = p.score_scale;
+    if (FP8) score_scale *= p.k_scale[kvh];
+
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2c, 2c+1
+    float o[KSTEPS][4];
+#pragma unroll
+    for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+    int64_t blk = 0;  // 16-token block counter inside the item
+    const int blocks_per_chunk = C / 16;
+    for (int64_t t = tok0; t < tok1; t += C) {
+      if (ok && !mbar_wait(full0 + 8 * stage, phase)) {
+        ok = false;
+        if (lane == 0) atomicOr(p.status, HPC_DEV_TIMEOUT);
+      }
+      if (ok) {
+        const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
+        const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
+        for (int j = 0; j < blocks_per_chunk; ++j) {
+          if (((blk + j) % kConsumerWarps) != warp) continue;
+          const int64_t tb = t + 16 * j;  // first token of this block
+          if (tb >= tok1) break;
+          const int rb = 16 * j;  // first row of this block inside the stage
+
+          // ---- S^T = K * Q^T (16 tokens x 8 heads)
+          float s[4] = {0.f, 0.f, 0.f, 0.f};
+          if (!FP8) {
+            const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+              const int chunk = 2 * ks + (lane >> 4);
+              const uint32_t addr = kbase + (chunk >> 3) * p.plane_bytes + swz128(row, chunk & 7);
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4(addr, a0, a1, a2, a3);
+              mma_bf16_16816(s, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+            }
+          } else {
+            const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+              const int chunk = 2 * kp + (lane >> 4);
+              uint32_t x0, x1, x2, x3;  // rows 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
+              ldsm_x4(kbase + swz128(row, chunk), x0, x1, x2, x3);
+              mma_f16_16816(s, e4m3x2_to_f16x2(x0 & 0xffff), e4m3x2_to_f16x2(x1 & 0xffff),
+                            e4m3x2_to_f16x2(x0 >> 16), e4m3x2_to_f16x2(x1 >> 16), qf[2 * kp][0], qf[2 * kp][1]);
+              mma_f16_16816(s, e4m3x2_to_f16x2(x2 & 0xffff), e4m3x2_to_f16x2(x3 & 0xffff),
+                            e4m3x2_to_f16x2(x2 >> 16), e4m3x2_to_f16x2(x3 >> 16), qf[2 * kp + 1][0],
+                            qf[2 * kp + 1][1]);
+            }
+          }
+
+          // ---- online softmax (base 2) over this block, per head
+          const bool tail = tb + 16 > tok1;
+          s[0] *= score_scale;
+          s[1] *= score_scale;
+          s[2] *= score_scale;
+          s[3] *= score_scale;
+          if (tail) {
+            if (tb + g >= tok1) s[0] = s[1] = -INFINITY;
+            if (tb + g + 8 >= tok1) s[2] = s[3] = -INFINITY;
+          }
+          float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+          }
+          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+          const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+          const float p0 = exp2f(s[0] - mn0), p1 = exp2f(s[1] - mn1);
+          const float p2 = exp2f(s[2] - mn0), p3 = exp2f(s[3] - mn1);
+          m0 = mn0;
+          m1 = mn1;
+          l0 = l0 * al0 + (p0 + p2);
+          l1 = l1 * al1 + (p1 + p3);
+#pragma unroll
+          for (int i = 0; i < KSTEPS; ++i) {
+            o[i][0] *= al0;
+            o[i][1] *= al1;
+            o[i][2] *= al0;
+            o[i][3] *= al1;
+          }
+          // P^T fragments: rows = tokens, cols = heads -> transpose to (k = token, n = head)
+          const uint32_t pa = FP8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+          const uint32_t pb = FP8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
+          const uint32_t b0 = movmatrix_trans(pa), b1 = movmatrix_trans(pb);
+
+          // tokens held in the A-operand halves: (2c, 2c+1) and (8+2c, 9+2c)
+          uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+          if (tail) {
+            mlo = (tb + 2 * c < tok1 ? 0x0000ffffu : 0u) | (tb + 2 * c + 1 < tok1 ? 0xffff0000u : 0u);
+            mhi = (tb + 2 * c + 8 < tok1 ? 0x0000ffffu : 0u) | (tb + 2 * c + 9 < tok1 ? 0xffff0000u : 0u);
+          }
+
+          // ---- O^T += V^T * P^T
+          if (!FP8) {
+            const int row = rb + (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+            for (int mi = 0; mi < KSTEPS; ++mi) {
+              const int chunk = 2 * mi + ((lane >> 3) & 1);
+              const uint32_t addr = vbase + (chunk >> 3) * p.plane_bytes + swz128(row, chunk & 7);
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_trans(addr, a0, a1, a2, a3);
+              mma_bf16_16816(o[mi], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0, b1);
+            }
+          } else {
+            const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+              const int chunk = 2 * kp + (lane >> 4);
+              uint32_t x0, x1, x2, x3;  // tokens 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
+              ldsm_x4(vbase + swz128(row, chunk), x0, x1, x2, x3);
+              {
+                const uint32_t lo0 = movmatrix_trans(e4m3x2_to_f16x2(x0 & 0xffff));
+                const uint32_t hi0 = movmatrix_trans(e4m3x2_to_f16x2(x0 >> 16));
+                const uint32_t lo1 = movmatrix_trans(e4m3x2_to_f16x2(x1 & 0xffff));
+                const uint32_t hi1 = movmatrix_trans(e4m3x2_to_f16x2(x1 >> 16));
+                mma_f16_16816(o[2 * kp], lo0 & mlo, hi0 & mlo, lo1 & mhi, hi1 & mhi, b0, b1);
+              }
+              {
+                const uint32_t lo0 = movmatrix_trans(e4m3x2_to_f16x2(x2 & 0xffff));
+                const uint32_t hi0 = movmatrix_trans(e4m3x2_to_f16x2(x2 >> 16));
+                const uint32_t lo1 = movmatrix_trans(e4m3x2_to_f16x2(x3 & 0xffff));
+                const uint32_t hi1 = movmatrix_trans(e4m3x2_to_f16x2(x3 >> 16));
+                mma_f16_16816(o[2 * kp + 1], lo0 & mlo, hi0 & mlo, lo1 & mhi, hi1 & mhi, b0, b1);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      blk += blocks_per_chunk;
+      if (++stage == stages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+
+    // ---- merge the 8 warps' states for this item
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    if (g == 0) {
+      red_m[warp * 8 + 2 * c] = m0;
+      red_m[warp * 8 + 2 * c + 1] = m1;
+      red_l[warp * 8 + 2 * c] = l0;
+      red_l[warp * 8 + 2 * c + 1] = l1;
+    }
+    {
+      float* r0 = red_o + (warp * 8 + 2 * c) * S::kRedStride;
+      float* r1 = r0 + S::kRedStride;
+#pragma unroll
+      for (int i = 0; i < KSTEPS; ++i) {
+        const int d0 = 16 * i + out_row<FP8>(g, 0), d1 = 16 * i + out_row<FP8>(g, 1);
+        r0[d0] = o[i][0];
+        r1[d0] = o[i][1];
+        r0[d1] = o[i][2];
+        r1[d1] = o[i][3];
+      }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);
+    const bool direct = (w.flags & HPC_ITEM_DIRECT) != 0;
+    const float vs = FP8 ? p.v_scale[kvh] : 1.f;
+    for (int idx = threadIdx.x; idx < p.group * D; idx += kConsumerWarps * 32) {
+      const int h = idx / D, d = idx - h * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int wq = 0; wq < kConsumerWarps; ++wq) M = fmaxf(M, red_m[wq * 8 + h]);
+      float Ls = 0.f, acc = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int wq = 0; wq < kConsumerWarps; ++wq) {
+          const float e = exp2f(red_m[wq * 8 + h] - M);
+          Ls += e * red_l[wq * 8 + h];
+          acc += e * red_o[(wq * 8 + h) * S::kRedStride + d];
+        }
+      }
+      acc *= vs;
+      if (direct) {
+        const float val = Ls > 0.f ? acc / Ls : 0.f;
+        const int64_t oi = (static_cast<int64_t>(w.req) * p.num_heads + head0 + h) * D + d;
+        if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
+        else reinterpret_cast<float*>(p.out)[oi] = val;
+      } else {
+        const int64_t pi = static_cast<int64_t>(it) * p.group + h;
+        p.partial_o[pi * D + d] = acc;
+        if (d == 0) {
+          p.partial_ml[2 * pi] = M * kLn2;  // natural-log units
+          p.partial_ml[2 * pi + 1] = Ls;
+        }
+      }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);  // reduce buffers are reused by the next item
+  }
+}
+
+// ----------------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Tensor map of a page pool [num_pages][Hkv][P][D]. Each box is 128 bytes of one token
+// row x `box_tokens` tokens of one (page, kv head), stored with the 128-byte swizzle.
+int make_pool_map(CUtensorMap* map, const void* base, bool fp8, int D, int P, int Hkv, int num_pages,
+                  int box_tokens) {
+  auto fn = encode_fn();
+  if (!fn) return fail(HPC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const int elt = fp8 ? 1 : 2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(Hkv),
+                        static_cast<cuuint64_t>(num_pages)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * elt, static_cast<cuuint64_t>(P) * D * elt,
+                           static_cast<cuuint64_t>(Hkv) * P * D * elt};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elt), static_cast<cuuint32_t>(box_tokens), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HPC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return HPC_OK;
+}
+
+struct LaunchShape {
+  int stages, smem, plane_bytes, stage_bytes;
+};
+
+int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
+  const int elt = fp8 ? 1 : 2;
+  const int planes = D * elt / 128;
+  const int plane_bytes = C * 128;
+  const int stage_bytes = 2 * planes * plane_bytes;
+  const int red = kConsumerWarps * 8 * (D + 4) * 4 + 2 * kConsumerWarps * 8 * 4;
+  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm);
+  const int fixed = red + 2 * kMaxStages * 8 + 1024;  // reduce buffers, barriers, alignment slack
+  int stages = (budget - fixed) / stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return fail(HPC_ERR_SHAPE, "page chunk of %d tokens does not fit two pipeline stages", C);
+  ls->stages = stages;
+  ls->plane_bytes = plane_bytes;
+  ls->stage_bytes = stage_bytes;
+  ls->smem = stages * stage_bytes + fixed;
+  return HPC_OK;
+}
+
+template <int D, bool FP8>
+int launch(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid, int smem,
+           cudaStream_t stream) {
+  auto kern = decode_attention_kernel<D, FP8>;
+  static int configured[64] = {0};  // per device: largest dynamic smem already allowed
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && configured[dev] < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(decode_attention_kernel)");
+    configured[dev] = smem;
+  }
+  kern<<<grid, kThreads, smem, stream>>>(mk, mv, prm);
+  return check_launch("decode_attention_kernel");
+}
+
+}  // namespace
+}  // namespace hpc
+
+using namespace hpc;
+
+extern "C" size_t hpc_partial_o_bytes(const hpc_plan* plan, int32_t num_heads, int32_t head_dim) {
+  if (!plan || plan->kv_heads < 1) return 0;
+  return static_cast<size_t>(plan->max_items) * (num_heads / plan->kv_heads) * head_dim * sizeof(float);
+}
+
+extern "C" size_t hpc_partial_ml_bytes(const hpc_plan* plan, int32_t num_heads) {
+  if (!plan || plan->kv_heads < 1) return 0;
+  return static_cast<size_t>(plan->max_items) * (num_heads / plan->kv_heads) * 2 * sizeof(float);
+}
+
+extern "C" int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, int32_t page_size, int32_t tile_len,
+                                         int32_t ctas_per_sm, int32_t* stages, int32_t* smem_bytes,
+                                         int32_t* threads) {
+  if (tile_len <= 0 || page_size <= 0) return fail(HPC_ERR_ARG, "bad tile/page size");
+  LaunchShape ls;
+  const int C = tile_len < page_size ? tile_len : page_size;
+  int rc = launch_shape(head_dim, kv_dtype == HPC_E4M3, C, ctas_per_sm, &ls);
+  if (rc) return rc;
+  if (stages) *stages = ls.stages;
+  if (smem_bytes) *smem_bytes = ls.smem;
+  if (threads) *threads = kThreads;
+  return HPC_OK;
+}
+
+extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                                    const float* k_scale, const float* v_scale, int32_t num_pages,
+                                    int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
+                                    const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
+                                    const hpc_plan* plan, float sm_scale, float* partial_o, float* partial_ml,
+                                    void* out, hpc_dtype out_dtype, uint32_t* status, void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !plan || !partial_o || !partial_ml || !out ||
+      !status)
+    return fail(HPC_ERR_ARG, "null pointer argument");
+  if (kv_dtype != HPC_BF16 && kv_dtype != HPC_E4M3) return fail(HPC_ERR_DTYPE, "kv_dtype must be BF16 or E4M3");
+  if (out_dtype != HPC_FP32 && out_dtype != HPC_BF16) return fail(HPC_ERR_DTYPE, "out_dtype must be FP32 or BF16");
+  const bool fp8 = kv_dtype == HPC_E4M3;
+  if (fp8 && (!k_scale || !v_scale)) return fail(HPC_ERR_ARG, "E4M3 cache needs k_scale and v_scale");
+  if (num_pages < 1 || max_pages_per_req < 1 || num_heads < 1 || kv_heads < 1)
+    return fail(HPC_ERR_ARG, "sizes must be >= 1");
+  if (num_heads % kv_heads) return fail(HPC_ERR_SHAPE, "num_heads %% kv_heads != 0");
+  const int group = num_heads / kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return fail(HPC_ERR_SHAPE, "group size must be 1, 2, 4 or 8");
+  if (!(head_dim == 128 || (head_dim == 64 && !fp8)))
+    return fail(HPC_ERR_SHAPE, "head_dim must be 128 (or 64 with a bf16 cache)");
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
+    return fail(HPC_ERR_SHAPE, "page_size must be 16, 32, 64 or 128");
+  if (plan->kv_heads != kv_heads || plan->num_ctas < 1) return fail(HPC_ERR_ARG, "plan does not match kv_heads");
+  const int tl = plan->tile_len;
+  if (tl % 16 || !(tl % page_size == 0 || page_size % tl == 0))
+    return fail(HPC_ERR_SHAPE, "tile_len %d must be a multiple of 16 and of page_size %d, or divide it", tl, page_size);
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(partial_o) || !aligned16(out))
+    return fail(HPC_ERR_ALIGN, "q, caches, partial_o and out must be 16-byte aligned");
+
+  const int C = tl < page_size ? tl : page_size;
+  const int sms = device_sm_count();
+  int ctas_per_sm = sms > 0 ? (plan->num_ctas + sms - 1) / sms : 1;
+  if (plan->is_static || ctas_per_sm < 1) ctas_per_sm = 1;
+  if (ctas_per_sm > 4) ctas_per_sm = 4;
+  LaunchShape ls;
+  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, &ls);
+  if (rc) return rc;
+
+  CUtensorMap mk, mv;
+  if ((rc = make_pool_map(&mk, k_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
+  if ((rc = make_pool_map(&mv, v_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
+
+  AttnParams prm;
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.items = plan->items;
+  prm.cta_indptr = plan->cta_indptr;
+  prm.k_scale = k_scale;
+  prm.v_scale = v_scale;
+  prm.partial_o = partial_o;
+  prm.partial_ml = partial_ml;
+  prm.out = out;
+  prm.status = status;
+  prm.max_pages = max_pages_per_req;
+  prm.num_pages = num_pages;
+  prm.page_size = page_size;
+  prm.tile_len = tl;
+  prm.chunk_tokens = C;
+  prm.num_heads = num_heads;
+  prm.group = group;
+  prm.stages = ls.stages;
+  prm.out_bf16 = out_dtype == HPC_BF16;
+  prm.plane_bytes = ls.plane_bytes;
+  prm.stage_bytes = ls.stage_bytes;
+  prm.score_scale = sm_scale * kLog2e;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fp8) return launch<128, true>(mk, mv, prm, plan->num_ctas, ls.smem, st);
+  if (head_dim == 128) return launch<128, false>(mk, mv, prm, plan->num_ctas, ls.smem, st);
+  return launch<64, false>(mk, mv, prm, plan->num_ctas, ls.smem, st);
+}

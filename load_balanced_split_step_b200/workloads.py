@@ -261,6 +261,22 @@ def make_case(spec: DecodeSpec, requests=None) -> DecodeCase:
                       extra={"requests": sel})
 
 
+def extract_requests(case: DecodeCase, requests) -> DecodeCase:
+    """A case holding only ``requests`` of an existing case (copied pages, compact pool)."""
+    rows = [int(r) for r in requests]
+    bt = case.block_table[rows]
+    used = bt[bt >= 0].long()
+    remap = torch.full((case.num_pages,), -1, dtype=torch.int32)
+    remap[used] = torch.arange(len(used), dtype=torch.int32)
+    bt2 = torch.where(bt >= 0, remap[bt.clamp(min=0).long()], bt)
+    sel = lambda t: None if t is None else t[rows].clone()
+    return DecodeCase(replace(case.spec, seq_lens=tuple(case.spec.seq_lens[r] for r in rows),
+                              name=case.spec.name + "[sample]"),
+                      case.seq_lens[rows].clone(), bt2.contiguous(), case.pages_per_req[rows],
+                      case.k_pages[used].clone(), case.v_pages[used].clone(), sel(case.q), sel(case.qkv),
+                      case.k_scale, case.v_scale, case.q_norm_w, case.k_norm_w, extra={"requests": rows})
+
+
 def random_partials(seed: int, n_items: int, group: int, head_dim: int):
     """Random partial softmax states (m, l, o) for merge tests: m ~ N(0, 4),
     l ~ U[0.5, 50), o ~ N(0, 1) * l.  Returns float32 tensors o [n, grp, D], ml [n, grp, 2]."""

@@ -63,10 +63,14 @@ def _finish(items_rows, item_cta, B, Hkv, G, n_units, chunk) -> Plan:
     for k, (r, kvh, tb, te, direct) in enumerate(items_rows):
         items[k] = (r, kvh, FLAG_DIRECT if direct else 0, tb, te)
     item_cta = np.asarray(item_cta, dtype=np.int64)
+    # items were appended in unit order, so owners and segments are non-decreasing and
+    # "number of items with owner < g" is a sorted-array count
+    assert np.all(np.diff(item_cta) >= 0)
     # cta_indptr[g] = index of the first item owned by a CTA >= g
-    cta_indptr = np.array([int(np.sum(item_cta < g)) for g in range(G + 1)], dtype=np.int32)
+    cta_indptr = np.searchsorted(item_cta, np.arange(G + 1), side="left").astype(np.int32)
     seg = items["req"].astype(np.int64) * Hkv + items["kv_head"].astype(np.int64)
-    merge_indptr = np.array([int(np.sum(seg < s)) for s in range(B * Hkv + 1)], dtype=np.int32)
+    assert np.all(np.diff(seg) >= 0)
+    merge_indptr = np.searchsorted(seg, np.arange(B * Hkv + 1), side="left").astype(np.int32)
     counts = np.diff(merge_indptr)
     merge_list = np.array([s for s in range(B * Hkv) if counts[s] != 1], dtype=np.int32)
     return Plan(items, item_cta, cta_indptr, merge_indptr, merge_list, n_units, chunk, G)
