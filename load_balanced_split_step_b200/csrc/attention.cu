@@ -19,6 +19,11 @@
 //    shapes fit the group without padding. The S^T accumulator becomes the P^T operand
 //    through two movmatrix transposes. The 128-byte swizzle keeps ldmatrix free of bank
 //    conflicts.
+//  * With a bf16 cache, P goes into the PV product as a bf16 high part plus a bf16
+//    residual: two products accumulated in fp32. "Tencent HPC llega a SGLang …" (remio.ai),
+//    section "Dynamic Attention y Fused MoE atacan distintos cuellos de botella", describes
+//    this split for an FP32 operand of the Router GEMM. Here it carries P at ~16 significant
+//    bits for a few percent of tensor-pipe time.
 //  * E4M3 cache: codes are widened to f16 in registers (cvt.f16x2.e4m3x2, exact). V needs
 //    the k = token orientation: it is loaded untransposed and transposed with movmatrix
 //    after widening. k_scale folds into the score scale, v_scale into the output.
@@ -289,10 +294,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             o[i][2] *= al0;
             o[i][3] *= al1;
           }
-          // P^T fragments: rows = tokens, cols = heads -> transpose to (k = token, n = head)
+          // P^T fragments: rows = tokens, cols = heads -> transpose to (k = token, n = head).
+          // bf16 keeps 8 significant bits, too few for P on short, peaked rows, so a bf16
+          // cache splits P into a bf16 high part and a bf16 residual and multiplies both
+          // (two products summed in fp32, ~16 significant bits). f16 P (E4M3 cache) keeps 11
+          // bits and goes as one product.
           const uint32_t pa = FP8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
           const uint32_t pb = FP8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
           const uint32_t b0 = movmatrix_trans(pa), b1 = movmatrix_trans(pb);
+          uint32_t r0 = 0, r1 = 0;
+          if (!FP8) {
+            const uint32_t ra = pack_bf16x2(p0 - __uint_as_float(pa << 16), p1 - __uint_as_float(pa & 0xffff0000u));
+            const uint32_t rb2 = pack_bf16x2(p2 - __uint_as_float(pb << 16), p3 - __uint_as_float(pb & 0xffff0000u));
+            r0 = movmatrix_trans(ra);
+            r1 = movmatrix_trans(rb2);
+          }
 
           // tokens held in the A-operand halves: (2c, 2c+1) and (8+2c, 9+2c)
           uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
@@ -310,7 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t addr = vbase + (chunk >> 3) * p.plane_bytes + swz128(row, chunk & 7);
               uint32_t a0, a1, a2, a3;
               ldsm_x4_trans(addr, a0, a1, a2, a3);
-              mma_bf16_16816(o[mi], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0, b1);
+              a0 &= mlo;
+              a1 &= mlo;
+              a2 &= mhi;
+              a3 &= mhi;
+              mma_bf16_16816(o[mi], a0, a1, a2, a3, b0, b1);
+              mma_bf16_16816(o[mi], a0, a1, a2, a3, r0, r1);
             }
           } else {
             const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
