@@ -215,6 +215,36 @@ HPC_API int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const fl
                         int32_t batch, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
                         uint32_t* status, void* stream);
 
+/* ---- decode step without caller scratch ------------------------------------------------ */
+
+/* Scratch held by the library for hpc_decode_step_noalloc: one static device array of this
+ * many bytes. Every GPU that loads the library holds it until the process exits. */
+#define HPC_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* The pages have no counterpart to this entry point. It is for callers that cannot call
+ * cudaMalloc: code that runs inside a CUDA graph capture, serving loops that reserve all
+ * device memory up front and must not stall (cudaMalloc can synchronise the device and can
+ * fail under memory pressure), and plugins hosted by a framework whose allocator owns the
+ * device memory.
+ * It runs hpc_decode_plan, hpc_decode_attention and hpc_merge_states for one decode step.
+ * The plan workspace and the partial states live in the library's static array of
+ * HPC_NOALLOC_SCRATCH_BYTES; the caller passes only inputs (as in hpc_decode_attention,
+ * plus batch, tile_len and num_ctas) and outputs (out, status). It allocates nothing.
+ *  - Needed scratch = plan workspace + max_items*group*(head_dim+2)*4 bytes (each part
+ *    rounded up to 256), with max_items = num_ctas + batch*kv_heads. A shape that needs
+ *    more than HPC_NOALLOC_SCRATCH_BYTES returns HPC_ERR_CAPACITY and launches nothing.
+ *  - All calls share the one array and leave its contents behind. Nothing in it has to
+ *    start at zero. Calls that overlap on the GPU race: issue them on one stream, or
+ *    order them.
+ *  - The first call on a device (with that device current) looks up the array's device
+ *    address and caches it. Make that first call before any stream capture begins. */
+HPC_API int hpc_decode_step_noalloc(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                                    const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                                    int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                                    int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch,
+                                    int32_t tile_len, int32_t num_ctas, float sm_scale, void* out,
+                                    hpc_dtype out_dtype, uint32_t* status, void* stream);
+
 /* ---- misc ---------------------------------------------------------------------------- */
 
 /* Launch shape the attention kernel would use: pipeline stages, dynamic shared memory

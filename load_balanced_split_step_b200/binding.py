@@ -26,7 +26,7 @@ ITEM_DTYPE = np.dtype([("req", "<i4"), ("kv_head", "<i2"), ("flags", "<i2"),
 EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_decode_plan",
            "hpc_decode_plan_static", "hpc_plan_cpu", "hpc_partial_o_bytes", "hpc_partial_ml_bytes",
            "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue", "hpc_attention_launch_info",
-           "hpc_status_string", "hpc_last_error", "hpc_abi_version")
+           "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc")
 
 
 class HpcError(RuntimeError):
@@ -68,6 +68,8 @@ def _load():
                                                i32, vp, i32, i32, i32, i32, vp, vp]),
         "hpc_attention_launch_info": (ctypes.c_int, [i32, ctypes.c_int, i32, i32, i32, ctypes.POINTER(i32),
                                                      ctypes.POINTER(i32), ctypes.POINTER(i32)]),
+        "hpc_decode_step_noalloc": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp,
+                                                   i32, vp, i32, i32, i32, fp, vp, ctypes.c_int, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -315,6 +317,37 @@ def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads,
                              v_scale=v_scale, out=out, out_dtype=out_dtype, status=status)
     merge(p, po, pml, out, num_heads, status)
     return out, p, status
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_step_noalloc(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *,
+                        kv_dtype="bf16", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None,
+                        out_dtype=torch.float32, status=None):
+    """One decode step through ``hpc_decode_step_noalloc``: the library keeps the plan and
+    partial states in its own static device array, for callers that cannot allocate device
+    memory. Returns (out, status). Calls that overlap on the GPU share that array; keep
+    them on one stream."""
+    _need(q, "q", torch.bfloat16)
+    dev = q.device
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    code = _kv_code(kv_dtype, k_pages)
+    B, Hq, D = q.shape
+    num_pages, Hkv, P, _ = k_pages.shape
+    if num_ctas is None:
+        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
+    status = new_status(dev) if status is None else status
+    scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    _check(_lib.hpc_decode_step_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(out),
+        HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status), _stream(dev)),
+        "hpc_decode_step_noalloc")
+    return out, status
 
 
 def launch_info(head_dim, kv_dtype, page_size, tile_len, ctas_per_sm=1):
