@@ -368,7 +368,12 @@ def run_ours(args, rank, world, local):
     K, W_ = args.steps, max(3, args.warmup)
 
     with ClockSampler(local) as clk:
-        total_ms, kern_ms = time_steps(step, lens, K, W_, world)
+        # the step as a user runs it: kernels back to back, chained by programmatic dependent launch
+        total_ms, _ = time_steps(step, lens, K, W_, world, kernel_events=False)
+        # the same steps again with CUDA events around each attention launch (on the launching
+        # stream) for the kernel's own duration; events between kernels break the launch overlap,
+        # so this loop is not the step time
+        _, kern_ms = time_steps(step, lens, K, 0, world, kernel_events=True)
     st = int(step.status.item())
     if st:
         raise RuntimeError(f"device status {st:#x} during the timed region")

@@ -12,8 +12,9 @@
 //    a ring of shared-memory stages with 4-D TMA tensor loads (SWIZZLE_128B). Each stage
 //    completes on an mbarrier with the transferred byte count. Whole pages travel as a
 //    few bulk copies, with an evict-first L2 policy: each byte is read once.
-//  * Warps 0..7 are consumers. They take 16-token blocks of the stream round-robin. Each
-//    keeps its own online-softmax state for the GQA group of the item's kv head.
+//  * Warps 0..7 are consumers, in groups that take whole stages round-robin. Inside a stage,
+//    each warp takes two consecutive 16-token blocks, which gives two independent MMA chains.
+//    Each warp keeps its own online-softmax state for the GQA group of the item's kv head.
 //  * QK^T runs as S^T = K * Q^T on mma.m16n8k16: M = 16 tokens, N = 8 query heads, K = head
 //    dim. PV runs as O^T = V^T * P^T: M = 16 head-dim rows, N = 8 heads, K = 16 tokens. Both
 //    shapes fit the group without padding. The S^T accumulator becomes the P^T operand
@@ -90,6 +91,193 @@ __device__ __forceinline__ int64_t item_end(const hpc_work_item& w, int32_t L, i
   return e;
 }
 
+// Online-softmax update of one warp's state with NB consecutive 16-token blocks of a stage.
+// K and V rows rb.. rb + 16*NB of the stage sit at kbase / vbase, in 128-byte swizzled
+// planes. Tokens tb.. of the request; tokens >= tok1 are masked. The NB blocks give
+// independent MMA chains, so the warp hides latency without more warps.
+template <int D, bool FP8, int NB>
+__device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, uint32_t plane_bytes, int rb,
+                                               int64_t tb, int64_t tok1, const uint32_t (&qf)[D / 16][2],
+                                               float score_scale, float& m0, float& m1, float& l0, float& l1,
+                                               float (&o)[D / 16][4], int lane) {
+  constexpr int KSTEPS = D / 16;
+  const int g = lane >> 2, c = lane & 3;
+
+  // ---- S^T = K * Q^T, one 16x8 tile per block
+  float s[NB][4];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) s[b][0] = s[b][1] = s[b][2] = s[b][3] = 0.f;
+  {
+    const int row0 = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
+    if (!FP8) {
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int chunk = 2 * ks + (lane >> 4);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const int row = row0 + 16 * b;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kbase + (chunk >> 3) * plane_bytes + swz128(row, chunk & 7), a0, a1, a2, a3);
+          mma_bf16_16816(s[b], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+        const int chunk = 2 * kp + (lane >> 4);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          uint32_t x0, x1, x2, x3;  // rows 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
+          ldsm_x4(kbase + swz128(row0 + 16 * b, chunk), x0, x1, x2, x3);
+          uint32_t f0l, f0h, f1l, f1h, f2l, f2h, f3l, f3h;
+          e4m3x4_to_f16x4(x0, f0l, f0h);
+          e4m3x4_to_f16x4(x1, f1l, f1h);
+          e4m3x4_to_f16x4(x2, f2l, f2h);
+          e4m3x4_to_f16x4(x3, f3l, f3h);
+          mma_f16_16816(s[b], f0l, f1l, f0h, f1h, qf[2 * kp][0], qf[2 * kp][1]);
+          mma_f16_16816(s[b], f2l, f3l, f2h, f3h, qf[2 * kp + 1][0], qf[2 * kp + 1][1]);
+        }
+      }
+    }
+  }
+
+  // ---- online softmax (base 2) over these NB blocks, per head
+  const bool tail = tb + 16 * NB > tok1;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[b][i] *= score_scale;
+    if (tail) {
+      if (tb + 16 * b + g >= tok1) s[b][0] = s[b][1] = -INFINITY;
+      if (tb + 16 * b + g + 8 >= tok1) s[b][2] = s[b][3] = -INFINITY;
+    }
+  }
+  float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
+#pragma unroll
+  for (int b = 1; b < NB; ++b) {
+    mx0 = fmaxf(mx0, fmaxf(s[b][0], s[b][2]));
+    mx1 = fmaxf(mx1, fmaxf(s[b][1], s[b][3]));
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: every call has a live token
+  const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+  float pr[NB][4];
+  float add0 = 0.f, add1 = 0.f;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    pr[b][0] = exp2f(s[b][0] - mn0);
+    pr[b][1] = exp2f(s[b][1] - mn1);
+    pr[b][2] = exp2f(s[b][2] - mn0);
+    pr[b][3] = exp2f(s[b][3] - mn1);
+    add0 += pr[b][0] + pr[b][2];
+    add1 += pr[b][1] + pr[b][3];
+  }
+  l0 = l0 * al0 + add0;
+  l1 = l1 * al1 + add1;
+  m0 = mn0;
+  m1 = mn1;
+  // a factor of exactly 1 leaves O unchanged, so the rescale is skipped when no row max moved
+  if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+    for (int i = 0; i < KSTEPS; ++i) {
+      o[i][0] *= al0;
+      o[i][1] *= al1;
+      o[i][2] *= al0;
+      o[i][3] *= al1;
+    }
+  }
+
+  // ---- P^T operands: rows = tokens, cols = heads, transposed to (k = token, n = head).
+  // bf16 keeps 8 significant bits, too few for P on short, peaked rows, so a bf16 cache
+  // sends P as a bf16 high part plus a bf16 residual (two products summed in fp32). f16 P
+  // (E4M3 cache) keeps 11 bits and goes as one product.
+  uint32_t ph0[NB], ph1[NB], pl0[NB], pl1[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const uint32_t pa = FP8 ? pack_f16x2(pr[b][0], pr[b][1]) : pack_bf16x2(pr[b][0], pr[b][1]);
+    const uint32_t pb = FP8 ? pack_f16x2(pr[b][2], pr[b][3]) : pack_bf16x2(pr[b][2], pr[b][3]);
+    ph0[b] = movmatrix_trans(pa);
+    ph1[b] = movmatrix_trans(pb);
+    if (!FP8) {
+      pl0[b] = movmatrix_trans(pack_bf16x2(pr[b][0] - __uint_as_float(pa << 16),
+                                           pr[b][1] - __uint_as_float(pa & 0xffff0000u)));
+      pl1[b] = movmatrix_trans(pack_bf16x2(pr[b][2] - __uint_as_float(pb << 16),
+                                           pr[b][3] - __uint_as_float(pb & 0xffff0000u)));
+    }
+  }
+  // V rows past the end may hold anything (even NaN): zero them so 0 * v stays 0.
+  // The A-operand halves hold tokens (2c, 2c+1) and (8+2c, 9+2c) of each block.
+  uint32_t mlo[NB], mhi[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    mlo[b] = mhi[b] = 0xffffffffu;
+    if (tail) {
+      const int64_t t0 = tb + 16 * b;
+      mlo[b] = (t0 + 2 * c < tok1 ? 0x0000ffffu : 0u) | (t0 + 2 * c + 1 < tok1 ? 0xffff0000u : 0u);
+      mhi[b] = (t0 + 2 * c + 8 < tok1 ? 0x0000ffffu : 0u) | (t0 + 2 * c + 9 < tok1 ? 0xffff0000u : 0u);
+    }
+  }
+
+  // ---- O^T += V^T * P^T
+  if (!FP8) {
+    const int row0 = rb + (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+    for (int mi = 0; mi < KSTEPS; ++mi) {
+      const int chunk = 2 * mi + ((lane >> 3) & 1);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int row = row0 + 16 * b;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(vbase + (chunk >> 3) * plane_bytes + swz128(row, chunk & 7), a0, a1, a2, a3);
+        if (tail) {
+          a0 &= mlo[b];
+          a1 &= mlo[b];
+          a2 &= mhi[b];
+          a3 &= mhi[b];
+        }
+        mma_bf16_16816(o[mi], a0, a1, a2, a3, ph0[b], ph1[b]);
+        mma_bf16_16816(o[mi], a0, a1, a2, a3, pl0[b], pl1[b]);
+      }
+    }
+  } else {
+    const int row0 = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+      const int chunk = 2 * kp + (lane >> 4);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        uint32_t x0, x1, x2, x3;  // tokens 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
+        ldsm_x4(vbase + swz128(row0 + 16 * b, chunk), x0, x1, x2, x3);
+        uint32_t f0l, f0h, f1l, f1h, f2l, f2h, f3l, f3h;
+        e4m3x4_to_f16x4(x0, f0l, f0h);
+        e4m3x4_to_f16x4(x1, f1l, f1h);
+        e4m3x4_to_f16x4(x2, f2l, f2h);
+        e4m3x4_to_f16x4(x3, f3l, f3h);
+        uint32_t a0 = movmatrix_trans(f0l), a1 = movmatrix_trans(f0h);
+        uint32_t a2 = movmatrix_trans(f1l), a3 = movmatrix_trans(f1h);
+        uint32_t c0 = movmatrix_trans(f2l), c1 = movmatrix_trans(f2h);
+        uint32_t c2 = movmatrix_trans(f3l), c3 = movmatrix_trans(f3h);
+        if (tail) {
+          a0 &= mlo[b];
+          a1 &= mlo[b];
+          a2 &= mhi[b];
+          a3 &= mhi[b];
+          c0 &= mlo[b];
+          c1 &= mlo[b];
+          c2 &= mhi[b];
+          c3 &= mhi[b];
+        }
+        mma_f16_16816(o[2 * kp], a0, a1, a2, a3, ph0[b], ph1[b]);
+        mma_f16_16816(o[2 * kp + 1], c0, c1, c2, c3, ph0[b], ph1[b]);
+      }
+    }
+  }
+}
+
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -102,20 +290,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* red_o = reinterpret_cast<float*>(smem + static_cast<size_t>(stages) * p.stage_bytes);
   float* red_m = red_o + kConsumerWarps * 8 * S::kRedStride;
   float* red_l = red_m + kConsumerWarps * 8;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * 8);  // full[stages], empty[stages]
+  // Barriers: full[stages][groups], then empty[stages]. Stage n (counted over this CTA's items)
+  // lives in slot n % stages and is read by warp group n % groups. Its fill completes on
+  // full[n % stages][n % groups]. Each group therefore waits on every phase of its own full
+  // barriers in order, and a parity wait can never match a phase two behind.
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * 8);
+  const int bpc = p.chunk_tokens / 16;          // 16-token blocks per stage
+  const int nb = bpc >= 2 ? 2 : 1;              // blocks per warp per stage
+  const int wps = bpc / nb;                     // warps per stage
+  const int groups = kConsumerWarps / wps;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ring_u32 = smem_u32(ring);
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + stages);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + stages * groups);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kConsumerWarps);
-    }
+    for (int s = 0; s < stages * groups; ++s) mbar_init(full0 + 8 * s, 1);
+    for (int s = 0; s < stages; ++s) mbar_init(empty0 + 8 * s, wps);
     fence_barrier_init();
   }
+  if (threadIdx.x == kConsumerWarps * 32) {
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
   __syncthreads();
+  // Everything above overlaps the planner's tail under programmatic dependent launch; the
+  // plan, q and the output buffers are touched only after the previous kernel has finished.
+  pdl_wait();
+  pdl_launch_dependents();
 
   const int it_begin = p.cta_indptr[blockIdx.x], it_end = p.cta_indptr[blockIdx.x + 1];
   const int C = p.chunk_tokens;
@@ -123,12 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer
-    if (lane != 0) return;
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
+    // The whole warp fetches the page ids of the next 32 chunks in one coalesced load; lane 0
+    // takes them by shuffle and issues the TMA copies. A dependent page-id load per stage
+    // would cap the issue rate at one stage per global-load latency.
     const uint64_t policy = l2_policy_evict_first();
     int stage = 0;
     uint32_t phase = 0;
+    int gidx = 0;
+    uint64_t fill_par = 0;  // bit (slot * groups + group): parity of the next fill of that barrier
+    int last_bar[kMaxStages], last_par[kMaxStages];
     int64_t issued = 0;
     bool ok = true;
     uint32_t bad = 0;
@@ -138,52 +343,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tok0 = static_cast<int64_t>(w.tile_begin) * tl;
       const int64_t tok1 = item_end(w, L, tl, p.max_pages * P);
       const int32_t* bt = p.block_table + w.req * p.max_pages;
-      for (int64_t t = tok0; t < tok1; t += C) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
-          ok = false;
-          bad |= HPC_DEV_TIMEOUT;
-          break;
-        }
-        const int32_t page = bt[t / P];
-        const int32_t off = static_cast<int32_t>(t % P);
-        if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
-        const uint32_t full = full0 + 8 * stage;
-        const uint32_t dst = ring_u32 + stage * p.stage_bytes;
-        mbar_arrive_expect_tx(full, p.stage_bytes);
+      const int64_t nchunks = tok1 > tok0 ? (tok1 - tok0 + C - 1) / C : 0;
+      for (int64_t cb = 0; cb < nchunks && ok; cb += 32) {
+        int32_t my_page = 0;
+        if (cb + lane < nchunks) my_page = bt[(tok0 + (cb + lane) * C) / P];
+        const int nk = static_cast<int>(nchunks - cb < 32 ? nchunks - cb : 32);
+        for (int k = 0; k < nk; ++k) {
+          const int32_t page = __shfl_sync(0xffffffffu, my_page, k);
+          if (lane == 0) {
+            if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
+              ok = false;
+              bad |= HPC_DEV_TIMEOUT;
+            } else {
+              const int32_t off = static_cast<int32_t>((tok0 + (cb + k) * C) % P);
+              if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
+              const int bi = stage * groups + gidx;
+              const uint32_t full = full0 + 8 * bi;
+              last_bar[stage] = bi;
+              last_par[stage] = static_cast<int>((fill_par >> bi) & 1);
+              fill_par ^= uint64_t(1) << bi;
+              const uint32_t dst = ring_u32 + stage * p.stage_bytes;
+              mbar_arrive_expect_tx(full, p.stage_bytes);
 #pragma unroll
-        for (int pl = 0; pl < S::kPlanes; ++pl)
-          tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, w.kv_head, page, policy);
+              for (int pl = 0; pl < S::kPlanes; ++pl)
+                tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, w.kv_head, page,
+                            policy);
 #pragma unroll
-        for (int pl = 0; pl < S::kPlanes; ++pl)
-          tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off, w.kv_head,
-                      page, policy);
-        ++issued;
-        if (++stage == stages) {
-          stage = 0;
-          phase ^= 1;
+              for (int pl = 0; pl < S::kPlanes; ++pl)
+                tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off,
+                            w.kv_head, page, policy);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          ++issued;
+          if (++stage == stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (++gidx == groups) gidx = 0;
         }
       }
     }
-    // Drain: the last fill of every slot must have landed before the CTA may exit.
-    const int64_t n = issued < stages ? issued : stages;
-    for (int64_t k = 1; k <= n; ++k) {
-      int s = stage - static_cast<int>(k);
-      uint32_t ph = phase;
-      if (s < 0) {
-        s += stages;
-        ph ^= 1;
-      }
-      if (!mbar_wait(full0 + 8 * s, ph)) bad |= HPC_DEV_TIMEOUT;
+    // Drain: the last fill of every slot must have landed before the CTA may exit (the
+    // consumers stop waiting after a timeout).
+    if (lane == 0) {
+      const int n = issued < stages ? static_cast<int>(issued) : stages;
+      for (int s = 0; s < n; ++s)
+        if (!mbar_wait(full0 + 8 * last_bar[s], static_cast<uint32_t>(last_par[s]))) bad |= HPC_DEV_TIMEOUT;
+      if (bad) atomicOr(p.status, bad);
     }
-    if (bad) atomicOr(p.status, bad);
     return;
   }
 
   // -------------------------------------------------------------------- consumers
+  // Stage n (counted across this CTA's items) is read by the warps of group n % groups:
+  // wps warps, each taking nb consecutive 16-token blocks. Only those warps wait on it and
+  // release it (empty-barrier count = wps).
   const int g = lane >> 2, c = lane & 3;  // MMA fragment row / column pair
   constexpr int KSTEPS = D / 16;
-  int stage = 0;
-  uint32_t phase = 0;
+  const int my_group = warp / wps, my_first = (warp % wps) * nb;
+  const uint32_t my_full0 = full0 + 8 * my_group;  // + 8 * groups * slot
+  int stage = 0, gidx = 0;
+  uint32_t wait_par = 0;  // bit s: parity of this group's next wait on slot s
   bool ok = true;
 
   for (int it = it_begin; it < it_end; ++it) {
@@ -220,151 +442,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < KSTEPS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-    int64_t blk = 0;  // 16-token block counter inside the item
-    const int blocks_per_chunk = C / 16;
     for (int64_t t = tok0; t < tok1; t += C) {
-      if (ok && !mbar_wait(full0 + 8 * stage, phase)) {
-        ok = false;
-        if (lane == 0) atomicOr(p.status, HPC_DEV_TIMEOUT);
-      }
-      if (ok) {
-        const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
-        const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
-        for (int j = 0; j < blocks_per_chunk; ++j) {
-          if (((blk + j) % kConsumerWarps) != warp) continue;
-          const int64_t tb = t + 16 * j;  // first token of this block
-          if (tb >= tok1) break;
-          const int rb = 16 * j;  // first row of this block inside the stage
-
-          // ---- S^T = K * Q^T (16 tokens x 8 heads)
-          float s[4] = {0.f, 0.f, 0.f, 0.f};
-          if (!FP8) {
-            const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int ks = 0; ks < KSTEPS; ++ks) {
-              const int chunk = 2 * ks + (lane >> 4);
-              const uint32_t addr = kbase + (chunk >> 3) * p.plane_bytes + swz128(row, chunk & 7);
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4(addr, a0, a1, a2, a3);
-              mma_bf16_16816(s, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-            }
-          } else {
-            const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int kp = 0; kp < KSTEPS / 2; ++kp) {
-              const int chunk = 2 * kp + (lane >> 4);
-              uint32_t x0, x1, x2, x3;  // rows 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
-              ldsm_x4(kbase + swz128(row, chunk), x0, x1, x2, x3);
-              mma_f16_16816(s, e4m3x2_to_f16x2(x0 & 0xffff), e4m3x2_to_f16x2(x1 & 0xffff),
-                            e4m3x2_to_f16x2(x0 >> 16), e4m3x2_to_f16x2(x1 >> 16), qf[2 * kp][0], qf[2 * kp][1]);
-              mma_f16_16816(s, e4m3x2_to_f16x2(x2 & 0xffff), e4m3x2_to_f16x2(x3 & 0xffff),
-                            e4m3x2_to_f16x2(x2 >> 16), e4m3x2_to_f16x2(x3 >> 16), qf[2 * kp + 1][0],
-                            qf[2 * kp + 1][1]);
-            }
-          }
-
-          // ---- online softmax (base 2) over this block, per head
-          const bool tail = tb + 16 > tok1;
-          s[0] *= score_scale;
-          s[1] *= score_scale;
-          s[2] *= score_scale;
-          s[3] *= score_scale;
-          if (tail) {
-            if (tb + g >= tok1) s[0] = s[1] = -INFINITY;
-            if (tb + g + 8 >= tok1) s[2] = s[3] = -INFINITY;
-          }
-          float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
-#pragma unroll
-          for (int off = 4; off < 32; off <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-          }
-          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-          const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-          const float p0 = exp2f(s[0] - mn0), p1 = exp2f(s[1] - mn1);
-          const float p2 = exp2f(s[2] - mn0), p3 = exp2f(s[3] - mn1);
-          m0 = mn0;
-          m1 = mn1;
-          l0 = l0 * al0 + (p0 + p2);
-          l1 = l1 * al1 + (p1 + p3);
-#pragma unroll
-          for (int i = 0; i < KSTEPS; ++i) {
-            o[i][0] *= al0;
-            o[i][1] *= al1;
-            o[i][2] *= al0;
-            o[i][3] *= al1;
-          }
-          // P^T fragments: rows = tokens, cols = heads -> transpose to (k = token, n = head).
-          // bf16 keeps 8 significant bits, too few for P on short, peaked rows, so a bf16
-          // cache splits P into a bf16 high part and a bf16 residual and multiplies both
-          // (two products summed in fp32, ~16 significant bits). f16 P (E4M3 cache) keeps 11
-          // bits and goes as one product.
-          const uint32_t pa = FP8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-          const uint32_t pb = FP8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
-          const uint32_t b0 = movmatrix_trans(pa), b1 = movmatrix_trans(pb);
-          uint32_t r0 = 0, r1 = 0;
-          if (!FP8) {
-            const uint32_t ra = pack_bf16x2(p0 - __uint_as_float(pa << 16), p1 - __uint_as_float(pa & 0xffff0000u));
-            const uint32_t rb2 = pack_bf16x2(p2 - __uint_as_float(pb << 16), p3 - __uint_as_float(pb & 0xffff0000u));
-            r0 = movmatrix_trans(ra);
-            r1 = movmatrix_trans(rb2);
-          }
-
-          // tokens held in the A-operand halves: (2c, 2c+1) and (8+2c, 9+2c)
-          uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-          if (tail) {
-            mlo = (tb + 2 * c < tok1 ? 0x0000ffffu : 0u) | (tb + 2 * c + 1 < tok1 ? 0xffff0000u : 0u);
-            mhi = (tb + 2 * c + 8 < tok1 ? 0x0000ffffu : 0u) | (tb + 2 * c + 9 < tok1 ? 0xffff0000u : 0u);
-          }
-
-          // ---- O^T += V^T * P^T
-          if (!FP8) {
-            const int row = rb + (lane & 7) + (lane >> 4) * 8;
-#pragma unroll
-            for (int mi = 0; mi < KSTEPS; ++mi) {
-              const int chunk = 2 * mi + ((lane >> 3) & 1);
-              const uint32_t addr = vbase + (chunk >> 3) * p.plane_bytes + swz128(row, chunk & 7);
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4_trans(addr, a0, a1, a2, a3);
-              a0 &= mlo;
-              a1 &= mlo;
-              a2 &= mhi;
-              a3 &= mhi;
-              mma_bf16_16816(o[mi], a0, a1, a2, a3, b0, b1);
-              mma_bf16_16816(o[mi], a0, a1, a2, a3, r0, r1);
-            }
-          } else {
-            const int row = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int kp = 0; kp < KSTEPS / 2; ++kp) {
-              const int chunk = 2 * kp + (lane >> 4);
-              uint32_t x0, x1, x2, x3;  // tokens 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
-              ldsm_x4(vbase + swz128(row, chunk), x0, x1, x2, x3);
-              {
-                const uint32_t lo0 = movmatrix_trans(e4m3x2_to_f16x2(x0 & 0xffff));
-                const uint32_t hi0 = movmatrix_trans(e4m3x2_to_f16x2(x0 >> 16));
-                const uint32_t lo1 = movmatrix_trans(e4m3x2_to_f16x2(x1 & 0xffff));
-                const uint32_t hi1 = movmatrix_trans(e4m3x2_to_f16x2(x1 >> 16));
-                mma_f16_16816(o[2 * kp], lo0 & mlo, hi0 & mlo, lo1 & mhi, hi1 & mhi, b0, b1);
-              }
-              {
-                const uint32_t lo0 = movmatrix_trans(e4m3x2_to_f16x2(x2 & 0xffff));
-                const uint32_t hi0 = movmatrix_trans(e4m3x2_to_f16x2(x2 >> 16));
-                const uint32_t lo1 = movmatrix_trans(e4m3x2_to_f16x2(x3 & 0xffff));
-                const uint32_t hi1 = movmatrix_trans(e4m3x2_to_f16x2(x3 >> 16));
-                mma_f16_16816(o[2 * kp + 1], lo0 & mlo, hi0 & mlo, lo1 & mhi, hi1 & mhi, b0, b1);
-              }
-            }
-          }
+      if (gidx == my_group) {
+        if (ok && !mbar_wait(my_full0 + 8 * groups * stage, (wait_par >> stage) & 1u)) {
+          ok = false;
+          if (lane == 0) atomicOr(p.status, HPC_DEV_TIMEOUT);
         }
+        wait_par ^= 1u << stage;
+        const int64_t tb = t + 16 * my_first;
+        if (ok && tb < tok1) {
+          const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
+          const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
+          if (nb == 2)
+            consume_blocks<D, FP8, 2>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
+                                      l0, l1, o, lane);
+          else
+            consume_blocks<D, FP8, 1>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
+                                      l0, l1, o, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * stage);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
-      blk += blocks_per_chunk;
-      if (++stage == stages) {
-        stage = 0;
-        phase ^= 1;
-      }
+      if (++stage == stages) stage = 0;
+      if (++gidx == groups) gidx = 0;
     }
 
     // ---- merge the 8 warps' states for this item
@@ -473,7 +573,7 @@ int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
   const int stage_bytes = 2 * planes * plane_bytes;
   const int red = kConsumerWarps * 8 * (D + 4) * 4 + 2 * kConsumerWarps * 8 * 4;
   const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm);
-  const int fixed = red + 2 * kMaxStages * 8 + 1024;  // reduce buffers, barriers, alignment slack
+  const int fixed = red + (kMaxStages * kConsumerWarps + kMaxStages) * 8 + 1024;  // reduce, barriers, align slack
   int stages = (budget - fixed) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return fail(HPC_ERR_SHAPE, "page chunk of %d tokens does not fit two pipeline stages", C);
@@ -496,7 +596,8 @@ int launch(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, 
       return check_launch("cudaFuncSetAttribute(decode_attention_kernel)");
     configured[dev] = smem;
   }
-  kern<<<grid, kThreads, smem, stream>>>(mk, mv, prm);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kThreads), static_cast<size_t>(smem), stream, mk, mv, prm);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "decode_attention_kernel: %s", cudaGetErrorString(e));
   return check_launch("decode_attention_kernel");
 }
 

@@ -28,9 +28,35 @@ struct PlanLayout {
 };
 PlanLayout plan_layout(int32_t batch, int32_t kv_heads, int32_t num_ctas, int32_t max_items);
 
+// Launch with programmatic dependent launch (PDL) allowed: the kernel may start while the
+// previous kernel on the stream is still running. It must call pdl_wait() before touching
+// memory that earlier work on the stream reads or writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // ---------------------------------------------------------------------------------------
 // device side
 // ---------------------------------------------------------------------------------------
+
+// Wait until the previous kernel on the stream has completed and its writes are visible
+// (a no-op for a kernel launched without PDL).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel on the stream launch now; it still waits in pdl_wait() for this one.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: bound on any pipeline wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -156,6 +182,13 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   uint32_t d;
   asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(d) : "r"(two_codes));
   return d;
+}
+
+// Four E4M3 codes (bytes 0..3 of x) to f16 pairs: lo = bytes (0, 1), hi = bytes (2, 3). Exact.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
 }
 
 // One float to its E4M3 code: round to nearest even, finite overflow saturates to +-448.

@@ -35,7 +35,7 @@ constexpr int kPlanThreads = 1024;
 __host__ __device__ inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 __host__ __device__ inline int32_t tiles_of(int32_t L, int32_t tl) {
-  return L > 0 ? static_cast<int32_t>(ceil_div64(L, tl)) : 0;
+  return L > 0 ? static_cast<int32_t>(static_cast<uint32_t>(L - 1) / static_cast<uint32_t>(tl) + 1) : 0;
 }
 
 __host__ __device__ inline bool len_ok(int32_t L, int32_t max_seq_len) {
@@ -46,6 +46,12 @@ __host__ __device__ inline bool len_ok(int32_t L, int32_t max_seq_len) {
 __host__ __device__ inline int32_t pieces_of(int64_t U, int32_t nt, int64_t chunk) {
   if (nt == 0) return 0;
   return static_cast<int32_t>((U + nt - 1) / chunk - U / chunk + 1);
+}
+
+// a / b for non-negative operands; 32-bit hardware path when the whole plan fits in 31 bits
+// (the flag is uniform across the block).
+__device__ __forceinline__ int64_t udiv(int64_t a, int64_t b, bool small) {
+  return small ? static_cast<int64_t>(static_cast<uint32_t>(a) / static_cast<uint32_t>(b)) : a / b;
 }
 
 // Block-wide exclusive scan of one int64 per thread (kPlanThreads threads).
@@ -89,6 +95,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t s_total;
   const int tid = threadIdx.x;
+  pdl_wait();  // seq_lens may come from the previous kernel; the plan buffers may still be read by it
+  pdl_launch_dependents();
 
   // pass 1: total units
   int64_t local = 0;
@@ -113,6 +121,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
   __syncthreads();
   const int64_t T = s_total * Hkv;
   const int64_t chunk = T > 0 ? ceil_div64(T, G) : 0;
+  const bool small = T < (int64_t(1) << 31);
 
   // pass 2: items, in blocks of kPlanThreads requests with running carries
   int64_t carry_nt = 0, carry_items = 0, carry_merge = 0;
@@ -128,38 +137,47 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     const int64_t nt_before = carry_nt + block_exclusive_scan(nt, &tot_nt, warp_sums);
     const int64_t U_r = nt_before * Hkv;
     int64_t n_pieces = 0, n_merge = 0;
-    if (r < B) {
+    if (r < B && nt > 0) {
       for (int kvh = 0; kvh < Hkv; ++kvh) {
-        const int32_t pc = pieces_of(U_r + static_cast<int64_t>(kvh) * nt, nt, chunk);
+        const int64_t U = U_r + static_cast<int64_t>(kvh) * nt;
+        const int64_t pc = udiv(U + nt - 1, chunk, small) - udiv(U, chunk, small) + 1;
         n_pieces += pc;
         n_merge += (pc != 1);
       }
+    } else if (r < B) {
+      n_merge = Hkv;  // an empty request: every kv head is zero-filled by the merge step
     }
     int64_t idx = carry_items + block_exclusive_scan(n_pieces, &tot_items, warp_sums);
     int64_t midx = carry_merge + block_exclusive_scan(n_merge, &tot_merge, warp_sums);
     if (r < B) {
       for (int kvh = 0; kvh < Hkv; ++kvh) {
         const int64_t s = static_cast<int64_t>(r) * Hkv + kvh;
-        const int64_t U = U_r + static_cast<int64_t>(kvh) * nt;
-        const int32_t pc = pieces_of(U, nt, chunk);
         out.merge_indptr[s] = static_cast<int32_t>(idx);
+        if (nt == 0) {
+          out.merge_list[midx++] = static_cast<int32_t>(s);
+          continue;
+        }
+        const int64_t U = U_r + static_cast<int64_t>(kvh) * nt;
+        const int64_t q0 = udiv(U, chunk, small);
+        const int64_t pc = udiv(U + nt - 1, chunk, small) - q0 + 1;
         if (pc != 1) out.merge_list[midx++] = static_cast<int32_t>(s);
-        for (int32_t j = 0; j < pc; ++j) {
-          const int64_t start = j == 0 ? U : (U / chunk + j) * chunk;
-          const int64_t end = std::min((U / chunk + j + 1) * chunk, U + nt);
-          if (idx < max_items) {
-            hpc_work_item w;
-            w.req = r;
-            w.kv_head = static_cast<int16_t>(kvh);
-            w.flags = pc == 1 ? HPC_ITEM_DIRECT : 0;
-            w.tile_begin = static_cast<int32_t>(start - U);
-            w.tile_end = static_cast<int32_t>(end - U);
-            out.items[idx] = w;
-            if (start % chunk == 0) out.cta_indptr[start / chunk] = static_cast<int32_t>(idx);
-          } else {
+        // piece j starts at U (j = 0) or at the CTA boundary (q0 + j) * chunk, and ends at the
+        // next boundary or at the end of the segment; piece j belongs to CTA q0 + j
+        for (int64_t j = 0; j < pc; ++j, ++idx) {
+          const int64_t start = j == 0 ? U : (q0 + j) * chunk;
+          const int64_t end = min((q0 + j + 1) * chunk, U + nt);
+          if (idx >= max_items) {
             overflow = true;
+            continue;
           }
-          ++idx;
+          hpc_work_item w;
+          w.req = r;
+          w.kv_head = static_cast<int16_t>(kvh);
+          w.flags = pc == 1 ? HPC_ITEM_DIRECT : 0;
+          w.tile_begin = static_cast<int32_t>(start - U);
+          w.tile_end = static_cast<int32_t>(end - U);
+          out.items[idx] = w;
+          if (j > 0 || start == q0 * chunk) out.cta_indptr[q0 + j] = static_cast<int32_t>(idx);
         }
       }
     }
@@ -168,7 +186,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
     carry_merge += tot_merge;
   }
   if (overflow) atomicOr(status, HPC_DEV_CAPACITY);
-  const int64_t n_items = std::min<int64_t>(carry_items, max_items);
+  const int64_t n_items = min(carry_items, static_cast<int64_t>(max_items));
   const int64_t n_active = chunk > 0 ? ceil_div64(T, chunk) : 0;
   for (int64_t g = n_active + tid; g <= G; g += kPlanThreads) out.cta_indptr[g] = static_cast<int32_t>(n_items);
   if (tid == 0) {
@@ -185,6 +203,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
                        int32_t max_seq_len, PlanPtrs out, uint32_t* status) {
   __shared__ int64_t warp_sums[32];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   int64_t carry_items = 0, carry_merge = 0, carry_nt = 0;
   uint32_t bad = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
@@ -321,9 +341,10 @@ extern "C" int hpc_decode_plan(const int32_t* seq_lens, int32_t batch, int32_t n
   const PlanLayout L = plan_layout(batch, kv_heads, num_ctas, static_cast<int32_t>(max_items));
   if (workspace_bytes < L.total) return fail(HPC_ERR_CAPACITY, "plan workspace %zu < %zu bytes", workspace_bytes, L.total);
   bind_plan(workspace, L, batch, kv_heads, tile_len, num_ctas, static_cast<int32_t>(max_items), 0, plan);
-  dynamic_plan_kernel<<<1, kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      seq_lens, batch, kv_heads, tile_len, num_ctas, max_seq_len, static_cast<int32_t>(max_items), ptrs_of(plan),
-      status);
+  const cudaError_t e = launch_pdl(dynamic_plan_kernel, dim3(1), dim3(kPlanThreads), 0, static_cast<cudaStream_t>(stream),
+                                   seq_lens, batch, kv_heads, tile_len, num_ctas, max_seq_len,
+                                   static_cast<int32_t>(max_items), ptrs_of(plan), status);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "dynamic_plan_kernel: %s", cudaGetErrorString(e));
   return check_launch("dynamic_plan_kernel");
 }
 
@@ -339,8 +360,9 @@ extern "C" int hpc_decode_plan_static(const int32_t* seq_lens, int32_t batch, in
   const PlanLayout L = plan_layout(batch, kv_heads, static_cast<int32_t>(G), static_cast<int32_t>(G));
   if (workspace_bytes < L.total) return fail(HPC_ERR_CAPACITY, "plan workspace %zu < %zu bytes", workspace_bytes, L.total);
   bind_plan(workspace, L, batch, kv_heads, tile_len, static_cast<int32_t>(G), static_cast<int32_t>(G), 1, plan);
-  static_plan_kernel<<<1, kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      seq_lens, batch, kv_heads, tile_len, splits, max_seq_len, ptrs_of(plan), status);
+  const cudaError_t e = launch_pdl(static_plan_kernel, dim3(1), dim3(kPlanThreads), 0, static_cast<cudaStream_t>(stream),
+                                   seq_lens, batch, kv_heads, tile_len, splits, max_seq_len, ptrs_of(plan), status);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "static_plan_kernel: %s", cudaGetErrorString(e));
   return check_launch("static_plan_kernel");
 }
 

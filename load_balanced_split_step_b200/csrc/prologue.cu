@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kProWarps * 32)
   __shared__ float s_cos[D / 2], s_sin[D / 2];
   const int r = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
   const int32_t L = seq_lens[r];
   const bool len_ok = L >= 1 && static_cast<int64_t>(L) <= max_pages * P;
   const int64_t pos = len_ok ? L - 1 : 0;
@@ -117,15 +119,11 @@ extern "C" int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* x = static_cast<const __nv_bfloat16*>(qkv);
   auto* qo = static_cast<__nv_bfloat16*>(q_out);
-  if (head_dim == 128)
-    prologue_kernel<128><<<batch, kProWarps * 32, 0, st>>>(x, q_norm_w, k_norm_w, eps, rope_theta, qo, k_pages,
-                                                             v_pages, fp8, k_scale, v_scale, num_pages, page_size,
-                                                             block_table, max_pages_per_req, seq_lens, num_heads,
-                                                             kv_heads, status);
-  else
-    prologue_kernel<64><<<batch, kProWarps * 32, 0, st>>>(x, q_norm_w, k_norm_w, eps, rope_theta, qo, k_pages,
-                                                            v_pages, fp8, k_scale, v_scale, num_pages, page_size,
-                                                            block_table, max_pages_per_req, seq_lens, num_heads,
-                                                            kv_heads, status);
+  auto kern = head_dim == 128 ? prologue_kernel<128> : prologue_kernel<64>;
+  const cudaError_t e = launch_pdl(kern, dim3(batch), dim3(kProWarps * 32), 0, st, x, q_norm_w, k_norm_w, eps,
+                                   static_cast<double>(rope_theta), qo, k_pages, v_pages, static_cast<int>(fp8),
+                                   k_scale, v_scale, num_pages, page_size, block_table,
+                                   static_cast<int64_t>(max_pages_per_req), seq_lens, num_heads, kv_heads, status);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "prologue_kernel: %s", cudaGetErrorString(e));
   return check_launch("prologue_kernel");
 }
