@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tile-len", type=int, default=0)
     ap.add_argument("--ctas-per-sm", type=int, default=1)
+    ap.add_argument("--path", default="fused", choices=["fused", "split"],
+                    help="fused: one launch per step (in-kernel plan + ticket merge); split: plan, attention and "
+                         "merge kernels")
     ap.add_argument("--no-extras", action="store_true", help="skip static split-k, e2e and CPU baseline legs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     return ap.parse_args(argv)
@@ -158,9 +161,10 @@ class ClockSampler:
 class Step:
     """One decode step through the binding, with buffers allocated once."""
 
-    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None):
+    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None, fused=False):
         self.B, self.spec, self.dc = B, spec, dc
         self.tl = tile_len
+        self.fused = fused and not static_splits
         dev = dc["seq_lens"].device
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.max_seq = dc["block_table"].shape[1] * spec.page_size
@@ -174,6 +178,8 @@ class Step:
             self.static_splits = None
         self.num_ctas = num_ctas
         self.po, self.pml = B.partial_buffers(self.plan, spec.num_heads, spec.head_dim, dev)
+        if self.fused:
+            self.ws = B.step_workspace(spec.batch, spec.num_heads, spec.kv_heads, spec.head_dim, num_ctas, dev)
         self.out = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.float32, device=dev)
         self.q = dc["q"]
         if spec.prologue:
@@ -187,6 +193,16 @@ class Step:
                        seq, s.num_heads, s.kv_heads, kv_dtype=s.kv_dtype, k_scale=dc["k_scale"],
                        v_scale=dc["v_scale"], eps=s.rms_eps, rope_theta=s.rope_theta, q_out=self.q,
                        status=self.status)
+        if self.fused:
+            if ev is not None:
+                ev[0].record()
+            B.decode_step_fused(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, s.num_heads,
+                                s.kv_heads, self.tl, kv_dtype=s.kv_dtype, k_scale=dc["k_scale"],
+                                v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
+                                workspace=self.ws)
+            if ev is not None:
+                ev[1].record()
+            return self.out
         if self.static_splits:
             B.plan_static(seq, s.num_heads, s.kv_heads, self.tl, self.static_splits, self.max_seq, self.status,
                           workspace=self.plan.workspace)
@@ -205,7 +221,8 @@ class Step:
 
     @property
     def launches(self):
-        return 4 if self.spec.prologue else 3
+        n = 1 if self.fused else 3
+        return n + (1 if self.spec.prologue else 0)
 
 
 def step_lengths(dc, spec):
@@ -247,7 +264,7 @@ def static_leg(B, spec, dc, tl, steps, sms):
             "sweep_us": {str(k): round(v, 2) for k, v in res.items()}}
 
 
-def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world):
+def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True):
     """Same metric through the public call with per-step H2D of the step inputs (q or qkv,
     seq_lens, block_table) from pinned host memory and D2H of the output. The KV cache is
     device-resident decode state and is not copied."""
@@ -257,6 +274,7 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world):
     src[qname] = getattr(case, qname).pin_memory()
     dst = {k: torch.empty_like(v, device=dev) for k, v in src.items()}
     out_host = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.float32).pin_memory()
+    ws = B.step_workspace(spec.batch, spec.num_heads, spec.kv_heads, spec.head_dim, num_ctas, dev) if fused else None
     h2d = sum(v.numel() * v.element_size() for v in src.values())
     d2h = out_host.numel() * out_host.element_size()
     ddc = dict(dc)
@@ -271,9 +289,15 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world):
                            ddc["block_table"], ddc["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype,
                            k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], eps=spec.rms_eps,
                            rope_theta=spec.rope_theta)
-        out, _, _ = B.decode_step(q, ddc["k_pages"], ddc["v_pages"], ddc["block_table"], ddc["seq_lens"],
-                                  spec.num_heads, spec.kv_heads, tl, kv_dtype=spec.kv_dtype, k_scale=ddc["k_scale"],
-                                  v_scale=ddc["v_scale"], num_ctas=num_ctas)
+        if fused:
+            out, _, _ = B.decode_step_fused(q, ddc["k_pages"], ddc["v_pages"], ddc["block_table"], ddc["seq_lens"],
+                                            spec.num_heads, spec.kv_heads, tl, kv_dtype=spec.kv_dtype,
+                                            k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], num_ctas=num_ctas,
+                                            workspace=ws)
+        else:
+            out, _, _ = B.decode_step(q, ddc["k_pages"], ddc["v_pages"], ddc["block_table"], ddc["seq_lens"],
+                                      spec.num_heads, spec.kv_heads, tl, kv_dtype=spec.kv_dtype,
+                                      k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], num_ctas=num_ctas)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -363,7 +387,7 @@ def run_ours(args, rank, world, local):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     tl = args.tile_len or spec.tile_len
     G = sms * args.ctas_per_sm
-    step = Step(B, spec, dc, G, tl)
+    step = Step(B, spec, dc, G, tl, fused=args.path == "fused")
     lens = step_lengths(dc, spec)
     K, W_ = args.steps, max(3, args.warmup)
 
@@ -411,7 +435,7 @@ def run_ours(args, rank, world, local):
         del g
         extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms)
         extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step), 3)
-    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world)
+    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path == "fused")
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_steps = max(50, K // 4)
     e2e_val = world * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
@@ -428,12 +452,15 @@ def run_ours(args, rank, world, local):
         "data": "synthetic (seeded N(0,1), bf16-rounded; random page permutation)",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "tile_len": tl, "num_ctas": G,
                    "plan": "dynamic (re-planned on the device every step)",
+                   "path": ("single launch: in-kernel plan, attention, ticket merge" if args.path == "fused"
+                            else "plan, attention and merge kernels chained by PDL"),
                    "l2": f"inputs larger than L2 ({bytes_step / 1e9:.2f} GB per step), no flush",
                    "parallelism": f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8000": round(achieved / 8000.0, 4),
-                     "kernel": "decode_attention_kernel", "kernel_us": round(1000 * kern_ms, 2),
+                     "kernel": "decode_attention_kernel" + ("<fused>" if args.path == "fused" else ""),
+                     "kernel_us": round(1000 * kern_ms, 2),
                      "traffic": load_traffic(args.workload)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

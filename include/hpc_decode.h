@@ -183,6 +183,38 @@ HPC_API int hpc_decode_attention(const void* q, const void* k_pages, const void*
                          float sm_scale, float* partial_o, float* partial_ml, void* out,
                          hpc_dtype out_dtype, uint32_t* status, void* stream);
 
+/* ---- single-launch step ---------------------------------------------------------------- */
+
+/* Bytes of workspace hpc_decode_step needs: batch*kv_heads int32 merge tickets, then
+ * 2*num_ctas partial states (group*(head_dim+2) floats each), each part rounded up to 256. */
+HPC_API size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads, int32_t kv_heads,
+                                               int32_t head_dim, int32_t num_ctas);
+
+/* One decode step in a single launch: the planner, the attention and the merge together.
+ * This is the fewer-launches direction of the pages' own roadmap: "Tencent HPC llega a
+ * SGLang …" (remio.ai), section "Tres señales …", lists megakernels; "vLLM × HPC-Ops"
+ * describes PDL-chained stages.
+ *  - Planning: each of the num_ctas persistent CTAs reads seq_lens and derives its own items
+ *    with the same closed form as hpc_decode_plan (same tiles, same CTA assignment).
+ *  - Merge: a split (request, kv head) is merged by the CTA that finishes its last piece. It
+ *    finds out via an atomic ticket; there is no wait.
+ *  - Requests with no tiles (L = 0, or an invalid length with HPC_DEV_BAD_SEQLEN) get a
+ *    zero output.
+ *  - Arguments as hpc_decode_attention, plus batch, tile_len and num_ctas. max_seq_len is
+ *    max_pages_per_req * page_size.
+ *  - workspace: device, 256-byte aligned, >= hpc_decode_step_workspace_bytes(). Its ticket
+ *    part must be zero before the first call (e.g. cudaMemset the whole workspace once).
+ *    Each call leaves it zero again. After a call that reported HPC_DEV_TIMEOUT, zero it
+ *    again. Calls that overlap on the GPU must not share a workspace.
+ *  - batch <= 4223 for head_dim 128 and <= 2175 for head_dim 64 (the per-request prefix is
+ *    held in shared memory). Beyond that, HPC_ERR_SHAPE: use hpc_decode_plan. */
+HPC_API int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                            const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                            int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                            int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
+                            int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
+                            hpc_dtype out_dtype, uint32_t* status, void* stream);
+
 /* ---- merge --------------------------------------------------------------------------- */
 
 /* Log-sum-exp merge of the partial states of every (request, kv head) that the plan split

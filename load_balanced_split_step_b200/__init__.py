@@ -7,7 +7,8 @@ below) loads the library and raises if it is missing: there is no CPU fallback.
 
 ``workloads`` holds the seeded synthetic inputs and needs no library.
 """
-_API = ("plan", "plan_static", "plan_host", "attention", "merge", "prologue", "decode_step",
+_API = ("plan", "plan_static", "plan_host", "attention", "merge", "prologue", "decode_step", "decode_step_fused",
+        "decode_step_noalloc",
         "Plan", "HpcError", "library_path", "status_string", "DEV_STATUS")
 
 

@@ -26,8 +26,9 @@
 //    this split for an FP32 operand of the Router GEMM. Here it carries P at ~16 significant
 //    bits for a few percent of tensor-pipe time.
 //  * E4M3 cache: codes are widened to f16 in registers (cvt.f16x2.e4m3x2, exact). V needs
-//    the k = token orientation: it is loaded untransposed and transposed with movmatrix
-//    after widening. k_scale folds into the score scale, v_scale into the output.
+//    the k = token orientation: ldmatrix.trans moves byte pairs, and one byte permute per
+//    register regroups them into token pairs before widening. k_scale folds into the score
+//    scale, v_scale into the output.
 //  * At the end of an item, the 8 consumer warps merge their states through shared memory.
 //  * Every wait is bounded (2 s). On expiry the kernel sets HPC_DEV_TIMEOUT, stops waiting,
 //    drains its outstanding copies (bounded too) and returns.
@@ -64,7 +65,28 @@ struct AttnParams {
   int32_t stages, out_bf16;
   uint32_t plane_bytes, stage_bytes;
   float score_scale;  // sm_scale * log2(e)
+  // single-launch step only: the plan is derived in the kernel from seq_lens
+  int32_t batch, kv_heads, max_seq_len;
+  int32_t* tickets;  // [batch * kv_heads], zero between steps
 };
+
+// One work item as the producer and the consumers see it.
+struct ItemInfo {
+  int32_t req, kvh;
+  int64_t tok0, tok1;  // tokens to stream
+  bool direct;         // covers its whole (request, kv head): writes the output itself
+  int64_t slot;        // partial-state slot of a split item
+  int64_t U;           // single-launch step: first unit of the (request, kv head) segment
+  int32_t nt;          // and its tile count
+};
+
+__device__ __forceinline__ int32_t tiles_of(int32_t L, int32_t tl) {
+  return L > 0 ? static_cast<int32_t>(static_cast<uint32_t>(L - 1) / static_cast<uint32_t>(tl) + 1) : 0;
+}
+
+__device__ __forceinline__ bool len_ok(int32_t L, int32_t max_seq_len) {
+  return L >= 0 && (max_seq_len <= 0 || L <= max_seq_len);
+}
 
 template <int D, bool FP8>
 struct Shape {
@@ -74,11 +96,11 @@ struct Shape {
 };
 
 // Output row index of accumulator register `half` (0: c0/c1, 1: c2/c3) for lane row g
-// inside a 16-row block. bf16 V comes from ldmatrix.trans in natural order. E4M3 V comes
-// from movmatrix in pairs: rows g -> 4*(g/2) + g%2, and the second half two further on.
+// inside a 16-row block. bf16 V comes from ldmatrix.trans in natural order (rows g, g+8).
+// E4M3 V comes from ldmatrix.trans on byte pairs, so rows g and g+8 hold d = 2g and 2g+1.
 template <bool FP8>
 __device__ __forceinline__ int out_row(int g, int half) {
-  if (FP8) return 4 * (g >> 1) + (g & 1) + 2 * half;
+  if (FP8) return 2 * g + half;
   return g + 8 * half;
 }
 
@@ -90,6 +112,73 @@ __device__ __forceinline__ int64_t item_end(const hpc_work_item& w, int32_t L, i
   if (e > capacity) e = capacity;
   return e;
 }
+
+// Items of one CTA, read from a device plan (hpc_decode_plan / hpc_decode_plan_static).
+struct PlanCursor {
+  int it, it_end;
+  __device__ bool next(const AttnParams& p, ItemInfo& x) {
+    if (it >= it_end) return false;
+    const hpc_work_item w = p.items[it];
+    x.req = w.req;
+    x.kvh = w.kv_head;
+    x.tok0 = static_cast<int64_t>(w.tile_begin) * p.tile_len;
+    x.tok1 = item_end(w, p.seq_lens[w.req], p.tile_len, p.max_pages * p.page_size);
+    x.direct = (w.flags & HPC_ITEM_DIRECT) != 0;
+    x.slot = it;
+    x.U = 0;
+    x.nt = 0;
+    ++it;
+    return true;
+  }
+};
+
+// Items of one CTA, derived in the kernel by the planner's closed form: the CTA owns units
+// [u, u_end) of the request -> kv head -> tile enumeration and cuts them at (request, kv head)
+// boundaries. A split (request, kv head) is always this CTA's first or last item, so two
+// partial slots per CTA suffice: 2g for a piece that starts at the CTA's first unit, 2g + 1
+// otherwise.
+struct WalkCursor {
+  int64_t u, u_end, u_first, U_r;
+  int32_t r, kvh, nt, tb, g;
+  __device__ bool next(const AttnParams& p, ItemInfo& x) {
+    if (u >= u_end) return false;
+    const int32_t te = static_cast<int32_t>(min(static_cast<int64_t>(nt), tb + (u_end - u)));
+    const int32_t L = p.seq_lens[r];
+    x.req = r;
+    x.kvh = kvh;
+    x.tok0 = static_cast<int64_t>(tb) * p.tile_len;
+    int64_t e = static_cast<int64_t>(te) * p.tile_len;
+    if (e > L) e = L;
+    x.tok1 = e;
+    x.direct = tb == 0 && te == nt;
+    x.slot = 2 * static_cast<int64_t>(g) + (u == u_first ? 0 : 1);
+    x.U = U_r + static_cast<int64_t>(kvh) * nt;
+    x.nt = nt;
+    u += te - tb;
+    tb = 0;
+    if (u < u_end) {  // step to the next (request, kv head) with tiles
+      if (++kvh == p.kv_heads) {
+        kvh = 0;
+        U_r += static_cast<int64_t>(p.kv_heads) * nt;
+        do {
+          ++r;
+          const int32_t Ln = p.seq_lens[r];
+          nt = len_ok(Ln, p.max_seq_len) ? tiles_of(Ln, p.tile_len) : 0;
+        } while (nt == 0);
+      }
+    }
+    return true;
+  }
+};
+
+template <bool FUSED>
+struct CursorOf {
+  using type = PlanCursor;
+};
+template <>
+struct CursorOf<true> {
+  using type = WalkCursor;
+};
 
 // Online-softmax update of one warp's state with NB consecutive 16-token blocks of a stage.
 // K and V rows rb.. rb + 16*NB of the stage sit at kbase / vbase, in 128-byte swizzled
@@ -244,6 +333,9 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
       }
     }
   } else {
+    // ldmatrix.trans on byte pairs: lane (g, c) receives bytes (d 2g, 2g+1) of tokens 2c and
+    // 2c+1. One byte permute regroups them into the token pairs (2c, 2c+1) at d = 2g and at
+    // d = 2g+1, which widen to the f16 A-operand halves of output rows 2g and 2g+1.
     const int row0 = rb + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
     for (int kp = 0; kp < KSTEPS / 2; ++kp) {
@@ -251,16 +343,12 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         uint32_t x0, x1, x2, x3;  // tokens 0-7 / 8-15 of chunk 2kp, then of chunk 2kp+1
-        ldsm_x4(vbase + swz128(row0 + 16 * b, chunk), x0, x1, x2, x3);
-        uint32_t f0l, f0h, f1l, f1h, f2l, f2h, f3l, f3h;
-        e4m3x4_to_f16x4(x0, f0l, f0h);
-        e4m3x4_to_f16x4(x1, f1l, f1h);
-        e4m3x4_to_f16x4(x2, f2l, f2h);
-        e4m3x4_to_f16x4(x3, f3l, f3h);
-        uint32_t a0 = movmatrix_trans(f0l), a1 = movmatrix_trans(f0h);
-        uint32_t a2 = movmatrix_trans(f1l), a3 = movmatrix_trans(f1h);
-        uint32_t c0 = movmatrix_trans(f2l), c1 = movmatrix_trans(f2h);
-        uint32_t c2 = movmatrix_trans(f3l), c3 = movmatrix_trans(f3h);
+        ldsm_x4_trans(vbase + swz128(row0 + 16 * b, chunk), x0, x1, x2, x3);
+        uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+        e4m3x4_to_f16x4(__byte_perm(x0, 0, 0x3120), a0, a1);
+        e4m3x4_to_f16x4(__byte_perm(x1, 0, 0x3120), a2, a3);
+        e4m3x4_to_f16x4(__byte_perm(x2, 0, 0x3120), c0, c1);
+        e4m3x4_to_f16x4(__byte_perm(x3, 0, 0x3120), c2, c3);
         if (tail) {
           a0 &= mlo[b];
           a1 &= mlo[b];
@@ -278,12 +366,195 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
   }
 }
 
-template <int D, bool FP8>
+// Single-launch step: each CTA finds where its unit range starts. It forms the exclusive
+// prefix sum of per-request tile counts in shared memory (the reduce buffer, unused until
+// the first item ends) and binary-searches it. Requests with no valid tiles get a zero
+// output from CTA r % num_ctas. Returns the walk cursor (all threads get the same one).
+template <int D>
+__device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_scan, int64_t* s_walk,
+                               WalkCursor& cur, int64_t& chunk) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int B = p.batch, Hkv = p.kv_heads, G = gridDim.x, g = blockIdx.x;
+  // per-thread contiguous run of requests, then a block scan of the run totals
+  const int per = (B + nthr - 1) / nthr;
+  const int r0 = min(B, tid * per), r1 = min(B, r0 + per);
+  int64_t run = 0;
+  uint32_t bad = 0;
+  for (int r = r0; r < r1; ++r) {
+    const int32_t L = p.seq_lens[r];
+    const bool ok = len_ok(L, p.max_seq_len);
+    if (!ok) bad |= HPC_DEV_BAD_SEQLEN;
+    run += ok ? tiles_of(L, p.tile_len) : 0;
+  }
+  if (bad && (r0 % G) == g) atomicOr(p.status, bad);
+  const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
+  int64_t x = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_scan[warp] = x;
+  __syncthreads();
+  if (tid == 0) {
+    int64_t acc = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int64_t t = s_scan[w];
+      s_scan[w] = acc;
+      acc += t;
+    }
+    s_scan[nwarps] = acc;
+  }
+  __syncthreads();
+  int64_t pre = s_scan[warp] + x - run;
+  for (int r = r0; r < r1; ++r) {
+    s_pre[r] = pre;
+    const int32_t L = p.seq_lens[r];
+    pre += len_ok(L, p.max_seq_len) ? tiles_of(L, p.tile_len) : 0;
+  }
+  if (tid == 0) s_pre[B] = s_scan[nwarps];
+  __syncthreads();
+  if (tid == 0) {
+    const int64_t T = s_pre[B] * Hkv;
+    const int64_t ch = T > 0 ? (T + G - 1) / G : 0;
+    const int64_t u0 = static_cast<int64_t>(g) * ch;
+    const int64_t u1 = min(u0 + ch, T);
+    int64_t r = 0, kvh = 0, tb = 0, nt = 0, U_r = 0;
+    if (u0 < T) {
+      // largest r with Hkv * s_pre[r] <= u0: the request that holds unit u0
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] * Hkv <= u0) lo = mid;
+        else hi = mid - 1;
+      }
+      r = lo;
+      nt = s_pre[r + 1] - s_pre[r];
+      U_r = s_pre[r] * Hkv;
+      kvh = (u0 - U_r) / nt;
+      tb = u0 - U_r - kvh * nt;
+    }
+    s_walk[0] = u0;
+    s_walk[1] = u1;
+    s_walk[2] = U_r;
+    s_walk[3] = r;
+    s_walk[4] = kvh;
+    s_walk[5] = nt;
+    s_walk[6] = tb;
+    s_walk[7] = ch;
+  }
+  __syncthreads();
+  cur.u = s_walk[0];
+  cur.u_first = s_walk[0];
+  cur.u_end = s_walk[1];
+  cur.U_r = s_walk[2];
+  cur.r = static_cast<int32_t>(s_walk[3]);
+  cur.kvh = static_cast<int32_t>(s_walk[4]);
+  cur.nt = static_cast<int32_t>(s_walk[5]);
+  cur.tb = static_cast<int32_t>(s_walk[6]);
+  cur.g = g;
+  chunk = s_walk[7];
+}
+
+// Zero output rows of requests that own no tiles (L = 0 or an invalid length).
+template <int D>
+__device__ void zero_empty_requests(const AttnParams& p, int tid, int nthr) {
+  for (int r = blockIdx.x; r < p.batch; r += gridDim.x) {
+    const int32_t L = p.seq_lens[r];
+    if (len_ok(L, p.max_seq_len) && L > 0) continue;
+    const int64_t base = static_cast<int64_t>(r) * p.num_heads * D;
+    for (int i = tid; i < p.num_heads * D; i += nthr) {
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[base + i] = __float2bfloat16_rn(0.f);
+      else reinterpret_cast<float*>(p.out)[base + i] = 0.f;
+    }
+  }
+}
+
+// Log-sum-exp merge of a split (request, kv head) by the CTA that finished its last piece.
+// Piece slots follow the walk cursor's rule: the piece in CTA gg is slot 2gg, except the first
+// piece when it starts inside CTA g1's range (slot 2 g1 + 1). All (piece, head) states are
+// loaded at once into shared memory (the reduce buffer, free at this point) and turned into
+// weights exp(m_i - M) / L. The output is then a weighted sum over independent loads. The
+// other CTAs' partial states are read through L2 (ld.global.cg) after the ticket's fence.
+template <int D>
+__device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t chunk, int tid, int nthr,
+                              float* s_buf, int buf_floats) {
+  const int64_t g1 = x.U / chunk, g2 = (x.U + x.nt - 1) / chunk;
+  const int64_t first_slot = (x.U > g1 * chunk) ? 2 * g1 + 1 : 2 * g1;
+  const int grp = p.group;
+  const int n = static_cast<int>(g2 - g1 + 1);
+  auto slot_of = [&](int i) -> int64_t { return i == 0 ? first_slot : 2 * (g1 + i); };
+  const int64_t orow = (static_cast<int64_t>(x.req) * p.num_heads + x.kvh * grp) * D;
+  float* s_m = s_buf;
+  float* s_w = s_buf + n * grp;
+  float* s_M = s_w + n * grp;
+  float* s_iL = s_M + 8;
+  if (2 * n * grp + 16 <= buf_floats) {
+    for (int k = tid; k < n * grp; k += nthr) {
+      const int i = k / grp, h = k - i * grp;
+      const float* ml = p.partial_ml + 2 * (slot_of(i) * grp + h);
+      s_m[k] = __ldcg(ml);
+      s_w[k] = __ldcg(ml + 1);
+    }
+    named_barrier_sync(1, nthr);
+    if (tid < grp) {
+      float M = -INFINITY;
+      for (int i = 0; i < n; ++i) M = fmaxf(M, s_m[i * grp + tid]);
+      float L = 0.f;
+      for (int i = 0; i < n; ++i) L += expf(s_m[i * grp + tid] - M) * s_w[i * grp + tid];
+      s_M[tid] = M;
+      s_iL[tid] = L > 0.f ? 1.f / L : 0.f;
+    }
+    named_barrier_sync(1, nthr);
+    for (int k = tid; k < n * grp; k += nthr) {
+      const int h = k % grp;
+      s_w[k] = expf(s_m[k] - s_M[h]) * s_iL[h];
+    }
+    named_barrier_sync(1, nthr);
+    for (int idx = tid; idx < grp * D; idx += nthr) {
+      const int h = idx / D;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      int i = 0;
+      for (; i + 4 <= n; i += 4) {
+        a0 += s_w[(i + 0) * grp + h] * __ldcg(p.partial_o + slot_of(i + 0) * grp * D + idx);
+        a1 += s_w[(i + 1) * grp + h] * __ldcg(p.partial_o + slot_of(i + 1) * grp * D + idx);
+        a2 += s_w[(i + 2) * grp + h] * __ldcg(p.partial_o + slot_of(i + 2) * grp * D + idx);
+        a3 += s_w[(i + 3) * grp + h] * __ldcg(p.partial_o + slot_of(i + 3) * grp * D + idx);
+      }
+      for (; i < n; ++i) a0 += s_w[i * grp + h] * __ldcg(p.partial_o + slot_of(i) * grp * D + idx);
+      const float val = (a0 + a1) + (a2 + a3);
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow + idx] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(p.out)[orow + idx] = val;
+    }
+    return;
+  }
+  // more pieces than the buffer holds: two passes over the partial states per output
+  for (int idx = tid; idx < grp * D; idx += nthr) {
+    const int h = idx / D;
+    float M = -INFINITY;
+    for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(p.partial_ml + 2 * (slot_of(i) * grp + h)));
+    float Ls = 0.f, acc = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const int64_t pi = slot_of(i) * grp + h;
+      const float e = expf(__ldcg(p.partial_ml + 2 * pi) - M);
+      Ls += e * __ldcg(p.partial_ml + 2 * pi + 1);
+      acc += e * __ldcg(p.partial_o + pi * D + (idx - h * D));
+    }
+    const float val = Ls > 0.f ? acc / Ls : 0.f;
+    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow + idx] = __float2bfloat16_rn(val);
+    else reinterpret_cast<float*>(p.out)[orow + idx] = val;
+  }
+}
+
+template <int D, bool FP8, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                             const AttnParams p) {
   using S = Shape<D, FP8>;
+  using Cursor = typename CursorOf<FUSED>::type;
   extern __shared__ uint8_t smem_raw[];
+  __shared__ int64_t s_scan[16], s_walk[8];
+  __shared__ int s_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stages = p.stages;
   uint8_t* ring = smem;
@@ -314,14 +585,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_v);
   }
   __syncthreads();
-  // Everything above overlaps the planner's tail under programmatic dependent launch; the
-  // plan, q and the output buffers are touched only after the previous kernel has finished.
+  // Everything above overlaps the previous kernel's tail under programmatic dependent launch;
+  // the plan, seq_lens, q and the output buffers are touched only after it has finished.
   pdl_wait();
   pdl_launch_dependents();
 
-  const int it_begin = p.cta_indptr[blockIdx.x], it_end = p.cta_indptr[blockIdx.x + 1];
+  Cursor cursor;
+  int64_t chunk = 0;
+  if constexpr (FUSED) {
+    plan_in_kernel<D>(p, reinterpret_cast<int64_t*>(red_o), s_scan, s_walk, cursor, chunk);
+  } else {
+    cursor.it = p.cta_indptr[blockIdx.x];
+    cursor.it_end = p.cta_indptr[blockIdx.x + 1];
+  }
   const int C = p.chunk_tokens;
-  const int tl = p.tile_len, P = p.page_size;
+  const int P = p.page_size;
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer
@@ -337,16 +615,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t issued = 0;
     bool ok = true;
     uint32_t bad = 0;
-    for (int it = it_begin; it < it_end && ok; ++it) {
-      const hpc_work_item w = p.items[it];
-      const int32_t L = p.seq_lens[w.req];
-      const int64_t tok0 = static_cast<int64_t>(w.tile_begin) * tl;
-      const int64_t tok1 = item_end(w, L, tl, p.max_pages * P);
-      const int32_t* bt = p.block_table + w.req * p.max_pages;
-      const int64_t nchunks = tok1 > tok0 ? (tok1 - tok0 + C - 1) / C : 0;
+    ItemInfo x;
+    while (ok && cursor.next(p, x)) {
+      const int32_t* bt = p.block_table + x.req * p.max_pages;
+      const int64_t nchunks = x.tok1 > x.tok0 ? (x.tok1 - x.tok0 + C - 1) / C : 0;
       for (int64_t cb = 0; cb < nchunks && ok; cb += 32) {
         int32_t my_page = 0;
-        if (cb + lane < nchunks) my_page = bt[(tok0 + (cb + lane) * C) / P];
+        if (cb + lane < nchunks) my_page = bt[(x.tok0 + (cb + lane) * C) / P];
         const int nk = static_cast<int>(nchunks - cb < 32 ? nchunks - cb : 32);
         for (int k = 0; k < nk; ++k) {
           const int32_t page = __shfl_sync(0xffffffffu, my_page, k);
@@ -355,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               bad |= HPC_DEV_TIMEOUT;
             } else {
-              const int32_t off = static_cast<int32_t>((tok0 + (cb + k) * C) % P);
+              const int32_t off = static_cast<int32_t>((x.tok0 + (cb + k) * C) % P);
               if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
               const int bi = stage * groups + gidx;
               const uint32_t full = full0 + 8 * bi;
@@ -366,12 +641,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(full, p.stage_bytes);
 #pragma unroll
               for (int pl = 0; pl < S::kPlanes; ++pl)
-                tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, w.kv_head, page,
-                            policy);
+                tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, x.kvh, page, policy);
 #pragma unroll
               for (int pl = 0; pl < S::kPlanes; ++pl)
-                tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off,
-                            w.kv_head, page, policy);
+                tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off, x.kvh,
+                            page, policy);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -397,31 +671,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // -------------------------------------------------------------------- consumers
-  // Stage n (counted across this CTA's items) is read by the warps of group n % groups:
-  // wps warps, each taking nb consecutive 16-token blocks. Only those warps wait on it and
-  // release it (empty-barrier count = wps).
+  // Stage n is read by the warps of group n % groups: wps warps, each taking nb consecutive
+  // 16-token blocks. Only those warps wait on it and release it (empty-barrier count = wps).
   const int g = lane >> 2, c = lane & 3;  // MMA fragment row / column pair
   constexpr int KSTEPS = D / 16;
   const int my_group = warp / wps, my_first = (warp % wps) * nb;
   const uint32_t my_full0 = full0 + 8 * my_group;  // + 8 * groups * slot
+  const int ctid = threadIdx.x, cthreads = kConsumerWarps * 32;
   int stage = 0, gidx = 0;
   uint32_t wait_par = 0;  // bit s: parity of this group's next wait on slot s
   bool ok = true;
+  if constexpr (FUSED) zero_empty_requests<D>(p, ctid, cthreads);
 
-  for (int it = it_begin; it < it_end; ++it) {
-    const hpc_work_item w = p.items[it];
-    const int32_t L = p.seq_lens[w.req];
-    const int64_t tok0 = static_cast<int64_t>(w.tile_begin) * tl;
-    const int64_t tok1 = item_end(w, L, tl, p.max_pages * P);
-    const int kvh = w.kv_head;
+  ItemInfo x;
+  while (cursor.next(p, x)) {
+    const int kvh = x.kvh;
     const int head0 = kvh * p.group;
+    const int64_t tok0 = x.tok0, tok1 = x.tok1;
 
     // Q^T fragments (B operand): lane (g, c) holds query head head0 + g.
     uint32_t qf[KSTEPS][2];
     {
       const bool live = g < p.group;
       const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          p.q + (static_cast<int64_t>(w.req) * p.num_heads + head0 + (live ? g : 0)) * D);
+          p.q + (static_cast<int64_t>(x.req) * p.num_heads + head0 + (live ? g : 0)) * D);
 #pragma unroll
       for (int ks = 0; ks < KSTEPS; ++ks) {
         if (!FP8) {
@@ -491,10 +764,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         r1[d1] = o[i][3];
       }
     }
-    named_barrier_sync(1, kConsumerWarps * 32);
-    const bool direct = (w.flags & HPC_ITEM_DIRECT) != 0;
+    named_barrier_sync(1, cthreads);
     const float vs = FP8 ? p.v_scale[kvh] : 1.f;
-    for (int idx = threadIdx.x; idx < p.group * D; idx += kConsumerWarps * 32) {
+    for (int idx = ctid; idx < p.group * D; idx += cthreads) {
       const int h = idx / D, d = idx - h * D;
       float M = -INFINITY;
 #pragma unroll
@@ -509,13 +781,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       acc *= vs;
-      if (direct) {
+      if (x.direct) {
         const float val = Ls > 0.f ? acc / Ls : 0.f;
-        const int64_t oi = (static_cast<int64_t>(w.req) * p.num_heads + head0 + h) * D + d;
+        const int64_t oi = (static_cast<int64_t>(x.req) * p.num_heads + head0 + h) * D + d;
         if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
         else reinterpret_cast<float*>(p.out)[oi] = val;
       } else {
-        const int64_t pi = static_cast<int64_t>(it) * p.group + h;
+        const int64_t pi = x.slot * p.group + h;
         p.partial_o[pi * D + d] = acc;
         if (d == 0) {
           p.partial_ml[2 * pi] = M * kLn2;  // natural-log units
@@ -523,7 +795,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    named_barrier_sync(1, kConsumerWarps * 32);  // reduce buffers are reused by the next item
+    if constexpr (FUSED) {
+      if (!x.direct) {
+        // the CTA that completes the last piece of this (request, kv head) merges it
+        __threadfence();
+        named_barrier_sync(1, cthreads);
+        if (ctid == 0) {
+          const int64_t pieces = (x.U + x.nt - 1) / chunk - x.U / chunk + 1;
+          int32_t* ticket = p.tickets + static_cast<int64_t>(x.req) * p.kv_heads + kvh;
+          const int old = atomicAdd(ticket, 1);
+          const int last = old == pieces - 1;
+          if (last) {
+            __threadfence();
+            *ticket = 0;  // ready for the next step
+          }
+          s_flag = last;
+        }
+        named_barrier_sync(1, cthreads);
+        if (s_flag) merge_segment<D>(p, x, chunk, ctid, cthreads, red_o, kConsumerWarps * 8 * S::kRedStride);
+      }
+    }
+    named_barrier_sync(1, cthreads);  // reduce buffers are reused by the next item
   }
 }
 
@@ -572,7 +864,7 @@ int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
   const int plane_bytes = C * 128;
   const int stage_bytes = 2 * planes * plane_bytes;
   const int red = kConsumerWarps * 8 * (D + 4) * 4 + 2 * kConsumerWarps * 8 * 4;
-  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm);
+  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - 256;  // 256: static shared memory
   const int fixed = red + (kMaxStages * kConsumerWarps + kMaxStages) * 8 + 1024;  // reduce, barriers, align slack
   int stages = (budget - fixed) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
@@ -584,10 +876,10 @@ int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
   return HPC_OK;
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool FUSED>
 int launch(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid, int smem,
            cudaStream_t stream) {
-  auto kern = decode_attention_kernel<D, FP8>;
+  auto kern = decode_attention_kernel<D, FP8, FUSED>;
   static int configured[64] = {0};  // per device: largest dynamic smem already allowed
   int dev = 0;
   cudaGetDevice(&dev);
@@ -630,20 +922,23 @@ extern "C" int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, i
   return HPC_OK;
 }
 
-extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
-                                    const float* k_scale, const float* v_scale, int32_t num_pages,
-                                    int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
-                                    const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
-                                    const hpc_plan* plan, float sm_scale, float* partial_o, float* partial_ml,
-                                    void* out, hpc_dtype out_dtype, uint32_t* status, void* stream) {
-  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !plan || !partial_o || !partial_ml || !out ||
-      !status)
+namespace hpc {
+namespace {
+
+// Checks shared by the attention entry points; fills the tensor maps, launch shape and the
+// common kernel parameters.
+int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype, const float* k_scale,
+            const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads, int32_t kv_heads,
+            int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
+            int32_t tile_len, int32_t grid, bool persistent, float sm_scale, void* out, hpc_dtype out_dtype,
+            uint32_t* status, CUtensorMap* mk, CUtensorMap* mv, LaunchShape* ls, AttnParams* prm) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !status)
     return fail(HPC_ERR_ARG, "null pointer argument");
   if (kv_dtype != HPC_BF16 && kv_dtype != HPC_E4M3) return fail(HPC_ERR_DTYPE, "kv_dtype must be BF16 or E4M3");
   if (out_dtype != HPC_FP32 && out_dtype != HPC_BF16) return fail(HPC_ERR_DTYPE, "out_dtype must be FP32 or BF16");
   const bool fp8 = kv_dtype == HPC_E4M3;
   if (fp8 && (!k_scale || !v_scale)) return fail(HPC_ERR_ARG, "E4M3 cache needs k_scale and v_scale");
-  if (num_pages < 1 || max_pages_per_req < 1 || num_heads < 1 || kv_heads < 1)
+  if (num_pages < 1 || max_pages_per_req < 1 || num_heads < 1 || kv_heads < 1 || grid < 1)
     return fail(HPC_ERR_ARG, "sizes must be >= 1");
   if (num_heads % kv_heads) return fail(HPC_ERR_SHAPE, "num_heads %% kv_heads != 0");
   const int group = num_heads / kv_heads;
@@ -652,53 +947,133 @@ extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const vo
     return fail(HPC_ERR_SHAPE, "head_dim must be 128 (or 64 with a bf16 cache)");
   if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
     return fail(HPC_ERR_SHAPE, "page_size must be 16, 32, 64 or 128");
-  if (plan->kv_heads != kv_heads || plan->num_ctas < 1) return fail(HPC_ERR_ARG, "plan does not match kv_heads");
-  const int tl = plan->tile_len;
-  if (tl % 16 || !(tl % page_size == 0 || page_size % tl == 0))
+  const int tl = tile_len;
+  if (tl < 16 || tl % 16 || !(tl % page_size == 0 || page_size % tl == 0))
     return fail(HPC_ERR_SHAPE, "tile_len %d must be a multiple of 16 and of page_size %d, or divide it", tl, page_size);
-  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(partial_o) || !aligned16(out))
-    return fail(HPC_ERR_ALIGN, "q, caches, partial_o and out must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out))
+    return fail(HPC_ERR_ALIGN, "q, caches and out must be 16-byte aligned");
 
   const int C = tl < page_size ? tl : page_size;
   const int sms = device_sm_count();
-  int ctas_per_sm = sms > 0 ? (plan->num_ctas + sms - 1) / sms : 1;
-  if (plan->is_static || ctas_per_sm < 1) ctas_per_sm = 1;
+  int ctas_per_sm = (persistent && sms > 0) ? (grid + sms - 1) / sms : 1;
+  if (ctas_per_sm < 1) ctas_per_sm = 1;
   if (ctas_per_sm > 4) ctas_per_sm = 4;
-  LaunchShape ls;
-  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, &ls);
+  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, ls);
   if (rc) return rc;
+  if ((rc = make_pool_map(mk, k_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
+  if ((rc = make_pool_map(mv, v_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
 
+  *prm = AttnParams{};
+  prm->q = static_cast<const __nv_bfloat16*>(q);
+  prm->block_table = block_table;
+  prm->seq_lens = seq_lens;
+  prm->k_scale = k_scale;
+  prm->v_scale = v_scale;
+  prm->out = out;
+  prm->status = status;
+  prm->max_pages = max_pages_per_req;
+  prm->num_pages = num_pages;
+  prm->page_size = page_size;
+  prm->tile_len = tl;
+  prm->chunk_tokens = C;
+  prm->num_heads = num_heads;
+  prm->group = group;
+  prm->stages = ls->stages;
+  prm->out_bf16 = out_dtype == HPC_BF16;
+  prm->plane_bytes = ls->plane_bytes;
+  prm->stage_bytes = ls->stage_bytes;
+  prm->score_scale = sm_scale * kLog2e;
+  prm->kv_heads = kv_heads;
+  prm->max_seq_len = max_pages_per_req * page_size;
+  return HPC_OK;
+}
+
+template <bool FUSED>
+int dispatch(int head_dim, bool fp8, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
+             int smem, cudaStream_t st) {
+  if (fp8) return launch<128, true, FUSED>(mk, mv, prm, grid, smem, st);
+  if (head_dim == 128) return launch<128, false, FUSED>(mk, mv, prm, grid, smem, st);
+  return launch<64, false, FUSED>(mk, mv, prm, grid, smem, st);
+}
+
+struct StepLayout {
+  size_t tickets, partial_o, partial_ml, total;
+};
+
+StepLayout step_layout(int32_t batch, int32_t group, int32_t kv_heads, int32_t head_dim, int32_t num_ctas) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  StepLayout L;
+  L.tickets = 0;
+  L.partial_o = up(static_cast<size_t>(batch) * kv_heads * sizeof(int32_t));
+  L.partial_ml = L.partial_o + up(2 * static_cast<size_t>(num_ctas) * group * head_dim * sizeof(float));
+  L.total = L.partial_ml + up(2 * static_cast<size_t>(num_ctas) * group * 2 * sizeof(float));
+  return L;
+}
+
+}  // namespace
+}  // namespace hpc
+
+extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                                    const float* k_scale, const float* v_scale, int32_t num_pages,
+                                    int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
+                                    const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
+                                    const hpc_plan* plan, float sm_scale, float* partial_o, float* partial_ml,
+                                    void* out, hpc_dtype out_dtype, uint32_t* status, void* stream) {
+  if (!plan || !partial_o || !partial_ml) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (plan->kv_heads != kv_heads || plan->num_ctas < 1) return fail(HPC_ERR_ARG, "plan does not match kv_heads");
+  if (!aligned16(partial_o)) return fail(HPC_ERR_ALIGN, "partial_o must be 16-byte aligned");
   CUtensorMap mk, mv;
-  if ((rc = make_pool_map(&mk, k_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
-  if ((rc = make_pool_map(&mv, v_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
-
+  LaunchShape ls;
   AttnParams prm;
-  prm.q = static_cast<const __nv_bfloat16*>(q);
-  prm.block_table = block_table;
-  prm.seq_lens = seq_lens;
+  int rc = prepare(q, k_pages, v_pages, kv_dtype, k_scale, v_scale, num_pages, page_size, num_heads, kv_heads,
+                   head_dim, block_table, max_pages_per_req, seq_lens, plan->tile_len, plan->num_ctas,
+                   !plan->is_static, sm_scale, out, out_dtype, status, &mk, &mv, &ls, &prm);
+  if (rc) return rc;
   prm.items = plan->items;
   prm.cta_indptr = plan->cta_indptr;
-  prm.k_scale = k_scale;
-  prm.v_scale = v_scale;
   prm.partial_o = partial_o;
   prm.partial_ml = partial_ml;
-  prm.out = out;
-  prm.status = status;
-  prm.max_pages = max_pages_per_req;
-  prm.num_pages = num_pages;
-  prm.page_size = page_size;
-  prm.tile_len = tl;
-  prm.chunk_tokens = C;
-  prm.num_heads = num_heads;
-  prm.group = group;
-  prm.stages = ls.stages;
-  prm.out_bf16 = out_dtype == HPC_BF16;
-  prm.plane_bytes = ls.plane_bytes;
-  prm.stage_bytes = ls.stage_bytes;
-  prm.score_scale = sm_scale * kLog2e;
+  prm.batch = plan->batch;
+  return dispatch<false>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, plan->num_ctas, ls.smem,
+                         static_cast<cudaStream_t>(stream));
+}
 
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (fp8) return launch<128, true>(mk, mv, prm, plan->num_ctas, ls.smem, st);
-  if (head_dim == 128) return launch<128, false>(mk, mv, prm, plan->num_ctas, ls.smem, st);
-  return launch<64, false>(mk, mv, prm, plan->num_ctas, ls.smem, st);
+extern "C" size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads, int32_t kv_heads,
+                                                  int32_t head_dim, int32_t num_ctas) {
+  if (batch < 1 || num_heads < 1 || kv_heads < 1 || head_dim < 1 || num_ctas < 1 || num_heads % kv_heads) return 0;
+  return step_layout(batch, num_heads / kv_heads, kv_heads, head_dim, num_ctas).total;
+}
+
+extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                               const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                               int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                               int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
+                               int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
+                               hpc_dtype out_dtype, uint32_t* status, void* stream) {
+  if (!workspace) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (batch < 1) return fail(HPC_ERR_ARG, "batch must be >= 1");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return fail(HPC_ERR_ALIGN, "workspace must be 256-byte aligned");
+  if (kv_heads > 32767 || static_cast<int64_t>(batch) * kv_heads > (1ll << 30))
+    return fail(HPC_ERR_SHAPE, "batch * kv_heads too large");
+  CUtensorMap mk, mv;
+  LaunchShape ls;
+  AttnParams prm;
+  int rc = prepare(q, k_pages, v_pages, kv_dtype, k_scale, v_scale, num_pages, page_size, num_heads, kv_heads,
+                   head_dim, block_table, max_pages_per_req, seq_lens, tile_len, num_ctas, true, sm_scale, out,
+                   out_dtype, status, &mk, &mv, &ls, &prm);
+  if (rc) return rc;
+  // the per-request tile prefix lives in the reduce buffer while the CTA plans
+  const size_t red_bytes = static_cast<size_t>(kConsumerWarps) * 8 * (head_dim + 4) * sizeof(float);
+  if ((static_cast<size_t>(batch) + 1) * sizeof(int64_t) > red_bytes)
+    return fail(HPC_ERR_SHAPE, "batch %d is above the single-launch limit %zu; plan with hpc_decode_plan", batch,
+                red_bytes / sizeof(int64_t) - 1);
+  const StepLayout L = step_layout(batch, num_heads / kv_heads, kv_heads, head_dim, num_ctas);
+  if (workspace_bytes < L.total) return fail(HPC_ERR_CAPACITY, "step workspace %zu < %zu bytes", workspace_bytes, L.total);
+  char* ws = static_cast<char*>(workspace);
+  prm.tickets = reinterpret_cast<int32_t*>(ws + L.tickets);
+  prm.partial_o = reinterpret_cast<float*>(ws + L.partial_o);
+  prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
+  prm.batch = batch;
+  return dispatch<true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
+                        static_cast<cudaStream_t>(stream));
 }
