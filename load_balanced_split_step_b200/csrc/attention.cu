@@ -43,7 +43,7 @@ namespace {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 16;
 constexpr int kSmemLimit = 232448;  // 227 KB per block on sm_100
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -610,8 +610,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     int gidx = 0;
-    uint64_t fill_par = 0;  // bit (slot * groups + group): parity of the next fill of that barrier
+    uint32_t fill_par[kMaxStages];  // bit k of word s: parity of the next fill of full[s][k]
     int last_bar[kMaxStages], last_par[kMaxStages];
+    for (int s = 0; s < kMaxStages; ++s) fill_par[s] = 0;
     int64_t issued = 0;
     bool ok = true;
     uint32_t bad = 0;
@@ -635,8 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int bi = stage * groups + gidx;
               const uint32_t full = full0 + 8 * bi;
               last_bar[stage] = bi;
-              last_par[stage] = static_cast<int>((fill_par >> bi) & 1);
-              fill_par ^= uint64_t(1) << bi;
+              last_par[stage] = static_cast<int>((fill_par[stage] >> gidx) & 1u);
+              fill_par[stage] ^= 1u << gidx;
               const uint32_t dst = ring_u32 + stage * p.stage_bytes;
               mbar_arrive_expect_tx(full, p.stage_bytes);
 #pragma unroll
@@ -863,17 +864,26 @@ int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
   const int planes = D * elt / 128;
   const int plane_bytes = C * 128;
   const int stage_bytes = 2 * planes * plane_bytes;
+  const int bpc = C / 16, nb = bpc >= 2 ? 2 : 1, groups = kConsumerWarps / (bpc / nb);
   const int red = kConsumerWarps * 8 * (D + 4) * 4 + 2 * kConsumerWarps * 8 * 4;
   const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - 256;  // 256: static shared memory
-  const int fixed = red + (kMaxStages * kConsumerWarps + kMaxStages) * 8 + 1024;  // reduce, barriers, align slack
-  int stages = (budget - fixed) / stage_bytes;
-  if (stages > kMaxStages) stages = kMaxStages;
-  if (stages < 2) return fail(HPC_ERR_SHAPE, "page chunk of %d tokens does not fit two pipeline stages", C);
+  int stages = kMaxStages;
+  // reduce buffers, full[stages][groups] + empty[stages] barriers, 1 KB alignment slack
+  auto need = [&](int st) { return st * stage_bytes + red + (st * groups + st) * 8 + 1024; };
+  while (stages > 2 && need(stages) > budget) --stages;
+  if (need(stages) > budget) return fail(HPC_ERR_SHAPE, "page chunk of %d tokens does not fit two pipeline stages", C);
   ls->stages = stages;
   ls->plane_bytes = plane_bytes;
   ls->stage_bytes = stage_bytes;
-  ls->smem = stages * stage_bytes + fixed;
+  ls->smem = need(stages);
   return HPC_OK;
+}
+
+// Tokens per pipeline stage: one TMA box per tensor plane. A box never crosses a page and is
+// at most 64 tokens, so a stage is at most 32 KB and the ring keeps several stages in flight.
+inline int chunk_tokens(int tile_len, int page_size) {
+  int C = tile_len < page_size ? tile_len : page_size;
+  return C > 64 ? 64 : C;
 }
 
 template <int D, bool FP8, bool FUSED>
@@ -913,7 +923,7 @@ extern "C" int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, i
                                          int32_t* threads) {
   if (tile_len <= 0 || page_size <= 0) return fail(HPC_ERR_ARG, "bad tile/page size");
   LaunchShape ls;
-  const int C = tile_len < page_size ? tile_len : page_size;
+  const int C = chunk_tokens(tile_len, page_size);
   int rc = launch_shape(head_dim, kv_dtype == HPC_E4M3, C, ctas_per_sm, &ls);
   if (rc) return rc;
   if (stages) *stages = ls.stages;
@@ -953,7 +963,7 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out))
     return fail(HPC_ERR_ALIGN, "q, caches and out must be 16-byte aligned");
 
-  const int C = tl < page_size ? tl : page_size;
+  const int C = chunk_tokens(tl, page_size);
   const int sms = device_sm_count();
   int ctas_per_sm = (persistent && sms > 0) ? (grid + sms - 1) / sms : 1;
   if (ctas_per_sm < 1) ctas_per_sm = 1;
