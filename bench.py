@@ -365,14 +365,33 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("attention.cu", "hpc_common.cuh"):
+        with open(os.path.join(ROOT, "load_balanced_split_step_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(workload):
-    """DRAM bytes per attention launch from the committed ncu summary, if it is current."""
-    p = os.path.join(ROOT, "profiles", f"attention_{workload}_traffic.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d.get("traffic_bytes_per_launch")
-    return None
+    """DRAM bytes per attention launch from the committed ncu summary, or None when the
+    kernel source has changed since those counters were taken."""
+    p = os.path.join(ROOT, "profiles", f"attention_{workload}_dram.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith(("#", "|", " ")):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def run_ours(args, rank, world, local):
