@@ -206,7 +206,7 @@ HPC_API size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads,
  *    part must be zero before the first call (e.g. cudaMemset the whole workspace once).
  *    Each call leaves it zero again. After a call that reported HPC_DEV_TIMEOUT, zero it
  *    again. Calls that overlap on the GPU must not share a workspace.
- *  - batch <= 4223 for head_dim 128 and <= 2175 for head_dim 64 (the per-request prefix is
+ *  - batch <= 4095 for head_dim 128 and <= 2047 for head_dim 64 (the per-request prefix is
  *    held in shared memory). Beyond that, HPC_ERR_SHAPE: use hpc_decode_plan. */
 HPC_API int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
                             const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,

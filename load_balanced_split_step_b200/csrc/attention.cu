@@ -92,7 +92,7 @@ template <int D, bool FP8>
 struct Shape {
   static constexpr int kElt = FP8 ? 1 : 2;
   static constexpr int kPlanes = D * kElt / 128;  // 128-byte swizzle planes per token row
-  static constexpr int kRedStride = D + 4;        // floats per (warp, head) row of the reduce buffer
+  static constexpr int kRedStride = D;  // floats per (warp, head) row; columns XOR 4h against bank conflicts
 };
 
 // Output row index of accumulator register `half` (0: c0/c1, 1: c2/c3) for lane row g
@@ -555,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ int64_t s_scan[16], s_walk[8];
   __shared__ int s_flag;
+  __shared__ int32_t s_pages[32];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stages = p.stages;
   uint8_t* ring = smem;
@@ -603,69 +604,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer
-    // The whole warp fetches the page ids of the next 32 chunks in one coalesced load; lane 0
-    // takes them by shuffle and issues the TMA copies. A dependent page-id load per stage
-    // would cap the issue rate at one stage per global-load latency.
+    // The warp loads the page ids of the next 32 chunks in one coalesced load into shared
+    // memory; lane 0 then issues the TMA copies on its own. Per stage, lane 0 does only
+    // register work: the page offset is a mask (page sizes are powers of two), and the fill
+    // parities of the full[slot][group] barriers live in two 64-bit words.
     const uint64_t policy = l2_policy_evict_first();
-    int stage = 0;
+    const int p_shift = __ffs(P) - 1;
+    int stage = 0, gidx = 0;
     uint32_t phase = 0;
-    int gidx = 0;
-    uint32_t fill_par[kMaxStages];  // bit k of word s: parity of the next fill of full[s][k]
-    int last_bar[kMaxStages], last_par[kMaxStages];
-    for (int s = 0; s < kMaxStages; ++s) fill_par[s] = 0;
+    uint64_t par_lo = 0, par_hi = 0;  // bit slot * groups + group: parity of that barrier's next fill
     int64_t issued = 0;
     bool ok = true;
     uint32_t bad = 0;
     ItemInfo x;
     while (ok && cursor.next(p, x)) {
-      const int32_t* bt = p.block_table + x.req * p.max_pages;
+      const int32_t* bt = p.block_table + x.req * p.max_pages + (x.tok0 >> p_shift);
+      const int off0 = static_cast<int>(x.tok0 & (P - 1));
       const int64_t nchunks = x.tok1 > x.tok0 ? (x.tok1 - x.tok0 + C - 1) / C : 0;
       for (int64_t cb = 0; cb < nchunks && ok; cb += 32) {
-        int32_t my_page = 0;
-        if (cb + lane < nchunks) my_page = bt[(x.tok0 + (cb + lane) * C) / P];
         const int nk = static_cast<int>(nchunks - cb < 32 ? nchunks - cb : 32);
-        for (int k = 0; k < nk; ++k) {
-          const int32_t page = __shfl_sync(0xffffffffu, my_page, k);
-          if (lane == 0) {
+        __syncwarp();  // lane 0 has finished with the previous batch of page ids
+        if (lane < nk) s_pages[lane] = bt[(off0 + (cb + lane) * C) >> p_shift];
+        __syncwarp();
+        if (lane == 0) {
+          for (int k = 0; k < nk; ++k) {
             if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
               ok = false;
               bad |= HPC_DEV_TIMEOUT;
-            } else {
-              const int32_t off = static_cast<int32_t>((x.tok0 + (cb + k) * C) % P);
-              if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
-              const int bi = stage * groups + gidx;
-              const uint32_t full = full0 + 8 * bi;
-              last_bar[stage] = bi;
-              last_par[stage] = static_cast<int>((fill_par[stage] >> gidx) & 1u);
-              fill_par[stage] ^= 1u << gidx;
-              const uint32_t dst = ring_u32 + stage * p.stage_bytes;
-              mbar_arrive_expect_tx(full, p.stage_bytes);
-#pragma unroll
-              for (int pl = 0; pl < S::kPlanes; ++pl)
-                tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, x.kvh, page, policy);
-#pragma unroll
-              for (int pl = 0; pl < S::kPlanes; ++pl)
-                tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off, x.kvh,
-                            page, policy);
+              break;
             }
+            const int32_t page = s_pages[k];
+            const int off = static_cast<int>((off0 + (cb + k) * C) & (P - 1));
+            if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
+            const int bi = stage * groups + gidx;
+            const uint32_t full = full0 + 8 * bi;
+            if (bi < 64) par_lo ^= uint64_t(1) << bi;
+            else par_hi ^= uint64_t(1) << (bi - 64);
+            const uint32_t dst = ring_u32 + stage * p.stage_bytes;
+            mbar_arrive_expect_tx(full, p.stage_bytes);
+#pragma unroll
+            for (int pl = 0; pl < S::kPlanes; ++pl)
+              tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, x.kvh, page, policy);
+#pragma unroll
+            for (int pl = 0; pl < S::kPlanes; ++pl)
+              tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off, x.kvh,
+                          page, policy);
+            ++issued;
+            if (++stage == stages) {
+              stage = 0;
+              phase ^= 1;
+            }
+            if (++gidx == groups) gidx = 0;
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          ++issued;
-          if (++stage == stages) {
-            stage = 0;
-            phase ^= 1;
-          }
-          if (++gidx == groups) gidx = 0;
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
     }
     // Drain: the last fill of every slot must have landed before the CTA may exit (the
-    // consumers stop waiting after a timeout).
+    // consumers stop waiting after a timeout). Slot s was last filled by stage
+    // n = last - ((last - s) mod stages), for group n % groups, with the parity before its flip.
     if (lane == 0) {
-      const int n = issued < stages ? static_cast<int>(issued) : stages;
-      for (int s = 0; s < n; ++s)
-        if (!mbar_wait(full0 + 8 * last_bar[s], static_cast<uint32_t>(last_par[s]))) bad |= HPC_DEV_TIMEOUT;
+      const int64_t last = issued - 1;
+      for (int s = 0; s < stages && s <= last; ++s) {
+        const int64_t n = last - ((last - s) % stages);
+        const int bi = s * groups + static_cast<int>(n % groups);
+        const uint32_t par = static_cast<uint32_t>(((bi < 64 ? par_lo >> bi : par_hi >> (bi - 64)) & 1u) ^ 1u);
+        if (!mbar_wait(full0 + 8 * bi, par)) bad |= HPC_DEV_TIMEOUT;
+      }
       if (bad) atomicOr(p.status, bad);
     }
     return;
@@ -754,15 +759,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       red_l[warp * 8 + 2 * c + 1] = l1;
     }
     {
+      // rows of heads 2c and 2c+1; column d is stored at d ^ (4 * head)
       float* r0 = red_o + (warp * 8 + 2 * c) * S::kRedStride;
       float* r1 = r0 + S::kRedStride;
+      const int x0 = 8 * c, x1 = 8 * c + 4;
 #pragma unroll
       for (int i = 0; i < KSTEPS; ++i) {
         const int d0 = 16 * i + out_row<FP8>(g, 0), d1 = 16 * i + out_row<FP8>(g, 1);
-        r0[d0] = o[i][0];
-        r1[d0] = o[i][1];
-        r0[d1] = o[i][2];
-        r1[d1] = o[i][3];
+        r0[d0 ^ x0] = o[i][0];
+        r1[d0 ^ x1] = o[i][1];
+        r0[d1 ^ x0] = o[i][2];
+        r1[d1 ^ x1] = o[i][3];
       }
     }
     named_barrier_sync(1, cthreads);
@@ -778,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int wq = 0; wq < kConsumerWarps; ++wq) {
           const float e = exp2f(red_m[wq * 8 + h] - M);
           Ls += e * red_l[wq * 8 + h];
-          acc += e * red_o[(wq * 8 + h) * S::kRedStride + d];
+          acc += e * red_o[(wq * 8 + h) * S::kRedStride + (d ^ (4 * h))];
         }
       }
       acc *= vs;
@@ -865,8 +872,8 @@ int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
   const int plane_bytes = C * 128;
   const int stage_bytes = 2 * planes * plane_bytes;
   const int bpc = C / 16, nb = bpc >= 2 ? 2 : 1, groups = kConsumerWarps / (bpc / nb);
-  const int red = kConsumerWarps * 8 * (D + 4) * 4 + 2 * kConsumerWarps * 8 * 4;
-  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - 256;  // 256: static shared memory
+  const int red = kConsumerWarps * 8 * D * 4 + 2 * kConsumerWarps * 8 * 4;
+  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - 512;  // 512: static shared memory
   int stages = kMaxStages;
   // reduce buffers, full[stages][groups] + empty[stages] barriers, 1 KB alignment slack
   auto need = [&](int st) { return st * stage_bytes + red + (st * groups + st) * 8 + 1024; };
@@ -1073,7 +1080,7 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
                    out_dtype, status, &mk, &mv, &ls, &prm);
   if (rc) return rc;
   // the per-request tile prefix lives in the reduce buffer while the CTA plans
-  const size_t red_bytes = static_cast<size_t>(kConsumerWarps) * 8 * (head_dim + 4) * sizeof(float);
+  const size_t red_bytes = static_cast<size_t>(kConsumerWarps) * 8 * head_dim * sizeof(float);
   if ((static_cast<size_t>(batch) + 1) * sizeof(int64_t) > red_bytes)
     return fail(HPC_ERR_SHAPE, "batch %d is above the single-launch limit %zu; plan with hpc_decode_plan", batch,
                 red_bytes / sizeof(int64_t) - 1);
