@@ -265,50 +265,71 @@ def static_leg(B, spec, dc, tl, steps, sms):
 
 
 def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True):
-    """Same metric through the public call with per-step H2D of the step inputs (q or qkv,
+    """Same metric through the public call, with per-step H2D of the step inputs (q or qkv,
     seq_lens, block_table) from pinned host memory and D2H of the output. The KV cache is
-    device-resident decode state and is not copied."""
+    device-resident decode state and is not copied. The step runs as a serving loop would:
+    copy-in, compute and copy-out streams with two buffer sets. Step i+1's inputs arrive and
+    step i-1's output leaves while step i computes, ordered by events. Every step still
+    copies its own inputs in and its own result out."""
     dev = dc["seq_lens"].device
     src = {"seq_lens": case.seq_lens.pin_memory(), "block_table": case.block_table.pin_memory()}
     qname = "qkv" if spec.prologue else "q"
     src[qname] = getattr(case, qname).pin_memory()
-    dst = {k: torch.empty_like(v, device=dev) for k, v in src.items()}
-    out_host = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.float32).pin_memory()
+    shape = (spec.batch, spec.num_heads, spec.head_dim)
+    nbuf = 2
+    dsts = [{k: torch.empty_like(v, device=dev) for k, v in src.items()} for _ in range(nbuf)]
+    outs = [torch.empty(shape, dtype=torch.float32, device=dev) for _ in range(nbuf)]
+    hosts = [torch.empty(shape, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    qbufs = [torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
     ws = B.step_workspace(spec.batch, spec.num_heads, spec.kv_heads, spec.head_dim, num_ctas, dev) if fused else None
     h2d = sum(v.numel() * v.element_size() for v in src.values())
-    d2h = out_host.numel() * out_host.element_size()
-    ddc = dict(dc)
+    d2h = hosts[0].numel() * hosts[0].element_size()
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_cmp = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
 
-    def one():
-        for k in src:
-            dst[k].copy_(src[k], non_blocking=True)
-        ddc.update(dst)
-        q = ddc["q"]
-        if spec.prologue:
-            q = B.prologue(ddc["qkv"], ddc["q_norm_w"], ddc["k_norm_w"], ddc["k_pages"], ddc["v_pages"],
-                           ddc["block_table"], ddc["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype,
-                           k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], eps=spec.rms_eps,
-                           rope_theta=spec.rope_theta)
-        if fused:
-            out, _, _ = B.decode_step_fused(q, ddc["k_pages"], ddc["v_pages"], ddc["block_table"], ddc["seq_lens"],
-                                            spec.num_heads, spec.kv_heads, tl, kv_dtype=spec.kv_dtype,
-                                            k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], num_ctas=num_ctas,
-                                            workspace=ws)
-        else:
-            out, _, _ = B.decode_step(q, ddc["k_pages"], ddc["v_pages"], ddc["block_table"], ddc["seq_lens"],
-                                      spec.num_heads, spec.kv_heads, tl, kv_dtype=spec.kv_dtype,
-                                      k_scale=ddc["k_scale"], v_scale=ddc["v_scale"], num_ctas=num_ctas)
-        out_host.copy_(out, non_blocking=True)
+    def one(i):
+        b = i % nbuf
+        d = dict(dc)
+        d.update(dsts[b])
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[b])  # step i-2 has finished reading this input set
+            for k in src:
+                dsts[b][k].copy_(src[k], non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            s_cmp.wait_event(ev_out[b])  # step i-2's output has left this buffer
+            q = d["q"]
+            if spec.prologue:
+                q = B.prologue(d["qkv"], d["q_norm_w"], d["k_norm_w"], d["k_pages"], d["v_pages"], d["block_table"],
+                               d["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype,
+                               k_scale=d["k_scale"], v_scale=d["v_scale"], eps=spec.rms_eps,
+                               rope_theta=spec.rope_theta, q_out=qbufs[b])
+            if fused:
+                B.decode_step_fused(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
+                                    spec.kv_heads, tl, kv_dtype=spec.kv_dtype, k_scale=d["k_scale"],
+                                    v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws)
+            else:
+                B.decode_step(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
+                              spec.kv_heads, tl, kv_dtype=spec.kv_dtype, k_scale=d["k_scale"], v_scale=d["v_scale"],
+                              num_ctas=num_ctas, out=outs[b])
+            ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            hosts[b].copy_(outs[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(4):
+        one(i)
     torch.cuda.synchronize()
     barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        one()
-    t1.record()
+    t0.record(s_in)
+    for i in range(steps):
+        one(i)
+    t1.record(s_out)
     torch.cuda.synchronize()
     barrier(world)
     return t0.elapsed_time(t1), h2d, d2h
