@@ -54,6 +54,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tile-len", type=int, default=0)
     ap.add_argument("--ctas-per-sm", type=int, default=1)
+    ap.add_argument("--layout", default="HND", choices=["HND", "NHD"], help="KV cache page layout")
     ap.add_argument("--path", default="fused", choices=["fused", "split"],
                     help="fused: one launch per step (in-kernel plan + ticket merge); split: plan, attention and "
                          "merge kernels")
@@ -161,8 +162,9 @@ class ClockSampler:
 class Step:
     """One decode step through the binding, with buffers allocated once."""
 
-    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None, fused=False):
+    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None, fused=False, layout="HND"):
         self.B, self.spec, self.dc = B, spec, dc
+        self.layout = layout
         self.tl = tile_len
         self.fused = fused and not static_splits
         dev = dc["seq_lens"].device
@@ -190,14 +192,14 @@ class Step:
         seq = dc["seq_lens"] if seq_lens is None else seq_lens
         if s.prologue:
             B.prologue(dc["qkv"], dc["q_norm_w"], dc["k_norm_w"], dc["k_pages"], dc["v_pages"], dc["block_table"],
-                       seq, s.num_heads, s.kv_heads, kv_dtype=s.kv_dtype, k_scale=dc["k_scale"],
+                       seq, s.num_heads, s.kv_heads, kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                        v_scale=dc["v_scale"], eps=s.rms_eps, rope_theta=s.rope_theta, q_out=self.q,
                        status=self.status)
         if self.fused:
             if ev is not None:
                 ev[0].record()
             B.decode_step_fused(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, s.num_heads,
-                                s.kv_heads, self.tl, kv_dtype=s.kv_dtype, k_scale=dc["k_scale"],
+                                s.kv_heads, self.tl, kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                                 v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
                                 workspace=self.ws)
             if ev is not None:
@@ -212,7 +214,7 @@ class Step:
         if ev is not None:
             ev[0].record()
         B.attention(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, self.plan, kv_dtype=s.kv_dtype,
-                    k_scale=dc["k_scale"], v_scale=dc["v_scale"], out=self.out, partial_o=self.po,
+                    kv_layout=self.layout, k_scale=dc["k_scale"], v_scale=dc["v_scale"], out=self.out, partial_o=self.po,
                     partial_ml=self.pml, status=self.status)
         if ev is not None:
             ev[1].record()
@@ -250,12 +252,12 @@ def time_steps(step, lens, K, W_, world, kernel_events=True):
     return total_ms, kern_ms
 
 
-def static_leg(B, spec, dc, tl, steps, sms):
+def static_leg(B, spec, dc, tl, steps, sms, layout="HND"):
     S0 = max(1, -(-2 * sms // (spec.batch * spec.kv_heads)))
     res = {}
     lens = step_lengths(dc, spec)
     for S in sorted({S0, 1, 2, 4, 8, 16, 32}):
-        st = Step(B, spec, dc, None, tl, static_splits=S)
+        st = Step(B, spec, dc, None, tl, static_splits=S, layout=layout)
         ms, _ = time_steps(st, lens, steps, 3, 1, kernel_events=False)
         res[S] = 1000.0 * ms / steps
     best = min(res, key=res.get)
@@ -264,7 +266,7 @@ def static_leg(B, spec, dc, tl, steps, sms):
             "sweep_us": {str(k): round(v, 2) for k, v in res.items()}}
 
 
-def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True):
+def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND"):
     """Same metric through the public call, with per-step H2D of the step inputs (q or qkv,
     seq_lens, block_table) from pinned host memory and D2H of the output. The KV cache is
     device-resident decode state and is not copied. The step runs as a serving loop would:
@@ -304,16 +306,17 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True):
             q = d["q"]
             if spec.prologue:
                 q = B.prologue(d["qkv"], d["q_norm_w"], d["k_norm_w"], d["k_pages"], d["v_pages"], d["block_table"],
-                               d["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype,
+                               d["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype, kv_layout=layout,
                                k_scale=d["k_scale"], v_scale=d["v_scale"], eps=spec.rms_eps,
                                rope_theta=spec.rope_theta, q_out=qbufs[b])
             if fused:
                 B.decode_step_fused(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
-                                    spec.kv_heads, tl, kv_dtype=spec.kv_dtype, k_scale=d["k_scale"],
+                                    spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
                                     v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws)
             else:
                 B.decode_step(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
-                              spec.kv_heads, tl, kv_dtype=spec.kv_dtype, k_scale=d["k_scale"], v_scale=d["v_scale"],
+                              spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
+                              v_scale=d["v_scale"],
                               num_ctas=num_ctas, out=outs[b])
             ev_cmp[b].record(s_cmp)
         with torch.cuda.stream(s_out):
@@ -424,10 +427,13 @@ def run_ours(args, rank, world, local):
     dc = {k: (getattr(case, k).to(dev) if getattr(case, k) is not None else None)
           for k in ("q", "qkv", "k_pages", "v_pages", "block_table", "seq_lens", "k_scale", "v_scale", "q_norm_w",
                     "k_norm_w")}
+    if args.layout == "NHD":  # same tokens, vLLM page layout [pages][P][Hkv][D]
+        dc["k_pages"] = dc["k_pages"].permute(0, 2, 1, 3).contiguous()
+        dc["v_pages"] = dc["v_pages"].permute(0, 2, 1, 3).contiguous()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     tl = args.tile_len or spec.tile_len
     G = sms * args.ctas_per_sm
-    step = Step(B, spec, dc, G, tl, fused=args.path == "fused")
+    step = Step(B, spec, dc, G, tl, fused=args.path == "fused", layout=args.layout)
     lens = step_lengths(dc, spec)
     K, W_ = args.steps, max(3, args.warmup)
 
@@ -473,9 +479,10 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         extra["graph_us_per_step"] = round(1000.0 * a.elapsed_time(b) / K, 2)
         del g
-        extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms)
+        extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms, args.layout)
         extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step), 3)
-    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path == "fused")
+    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path == "fused",
+                               layout=args.layout)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_steps = max(50, K // 4)
     e2e_val = world * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
@@ -494,6 +501,7 @@ def run_ours(args, rank, world, local):
                    "plan": "dynamic (re-planned on the device every step)",
                    "path": ("single launch: in-kernel plan, attention, ticket merge" if args.path == "fused"
                             else "plan, attention and merge kernels chained by PDL"),
+                   "kv_layout": args.layout,
                    "l2": f"inputs larger than L2 ({bytes_step / 1e9:.2f} GB per step), no flush",
                    "parallelism": f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",

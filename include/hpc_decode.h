@@ -34,8 +34,9 @@
  *    ids, and wait timeouts. The kernels never trap. After a non-zero status the
  *    outputs of the affected requests are unspecified (but no out-of-bounds access
  *    happens). Clear *status before the step.
- *  - Cache layout (HND): k_pages / v_pages are [num_pages][kv_heads][page_size][head_dim],
- *    row-major, with elements bf16 or E4M3 codes. block_table is int32
+ *  - Cache layout: k_pages / v_pages are [num_pages][kv_heads][page_size][head_dim] (HPC_HND)
+ *    or [num_pages][page_size][kv_heads][head_dim] (HPC_NHD), row-major, with elements bf16 or
+ *    E4M3 codes. block_table is int32
  *    [batch][max_pages_per_req]. block_table[r][j] is the page that holds tokens
  *    [j*page_size, (j+1)*page_size) of request r. seq_lens is int32 [batch]: the number
  *    of valid tokens, including the one being decoded.
@@ -51,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 1
+#define HPC_DECODE_ABI_VERSION 2
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -71,6 +72,14 @@ typedef enum {
 } hpc_status;
 
 typedef enum { HPC_BF16 = 0, HPC_FP32 = 1, HPC_E4M3 = 2 } hpc_dtype;
+
+/* Page layout of the KV cache.
+ *   HPC_HND: [num_pages][kv_heads][page_size][head_dim]. One (page, kv head) block is contiguous.
+ *   HPC_NHD: [num_pages][page_size][kv_heads][head_dim]. The vLLM paged-cache layout: the
+ *            kv heads of one token are contiguous.
+ * Both stream through the same TMA boxes: a box holds up to 64 tokens x 128 bytes of one kv
+ * head, with the token stride given by the layout. */
+typedef enum { HPC_HND = 0, HPC_NHD = 1 } hpc_kv_layout;
 
 /* Bits the kernels OR into the caller's device status word. */
 #define HPC_DEV_BAD_SEQLEN 0x1u /* seq_len < 0 or > max tokens; the request gets no tiles and a zero output */
@@ -162,8 +171,8 @@ HPC_API size_t hpc_partial_ml_bytes(const hpc_plan* plan, int32_t num_heads);
  * grid = plan->num_ctas CTAs. Each CTA streams its items' KV pages through a shared-memory
  * ring filled by TMA, with tensor-core QK^T and PV on the GQA group.
  *   q:        device bf16 [batch][num_heads][head_dim].
- *   k_pages, v_pages: device cache, see the layout above. kv_dtype is HPC_BF16 or HPC_E4M3.
- *             Base addresses must be 16-byte aligned.
+ *   k_pages, v_pages: device cache, see the layouts above. kv_dtype is HPC_BF16 or HPC_E4M3,
+ *             kv_layout HPC_HND or HPC_NHD. Base addresses must be 16-byte aligned.
  *   k_scale, v_scale: device float [kv_heads], required for HPC_E4M3 (value = code * scale),
  *             ignored for HPC_BF16.
  *   page_size: 16, 32, 64 or 128.  head_dim: 64 or 128 for bf16, 128 for E4M3.
@@ -177,7 +186,7 @@ HPC_API size_t hpc_partial_ml_bytes(const hpc_plan* plan, int32_t num_heads);
  *   out:      device [batch][num_heads][head_dim], out_dtype HPC_FP32 or HPC_BF16. DIRECT
  *             items write it here; hpc_merge_states writes the rest. */
 HPC_API int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
-                         const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                         hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
                          int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                          int32_t max_pages_per_req, const int32_t* seq_lens, const hpc_plan* plan,
                          float sm_scale, float* partial_o, float* partial_ml, void* out,
@@ -209,7 +218,7 @@ HPC_API size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads,
  *  - batch <= 4095 for head_dim 128 and <= 2047 for head_dim 64 (the per-request prefix is
  *    held in shared memory). Beyond that, HPC_ERR_SHAPE: use hpc_decode_plan. */
 HPC_API int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
-                            const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                            hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
                             int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                             int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
                             int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
@@ -232,8 +241,8 @@ HPC_API int hpc_merge_states(const float* partial_o, const float* partial_ml, co
  *   q heads:  RMSNorm (q_norm_w, eps), then NeoX RoPE at pos (pairs (i, i+D/2),
  *             angle pos * theta^(-2i/D), computed in fp64), written as bf16 to q_out.
  *   k heads:  RMSNorm (k_norm_w), RoPE, then stored to page block_table[r][pos/page_size],
- *             slot pos % page_size, as bf16 or as E4M3 code of x / k_scale[g] (RNE,
- *             saturating to +-448).
+ *             slot pos % page_size (in kv_layout), as bf16 or as E4M3 code of x / k_scale[g]
+ *             (RNE, saturating to +-448).
  *   v heads:  stored as is (bf16) or as E4M3 of v / v_scale[g].
  *   qkv:      device bf16 [batch][num_heads + 2*kv_heads][head_dim] (q heads, then k, then v).
  *   q_norm_w, k_norm_w: device float [head_dim].
@@ -242,6 +251,7 @@ HPC_API int hpc_merge_states(const float* partial_o, const float* partial_ml, co
  * q_out row is zeroed. */
 HPC_API int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,
                         float rope_theta, void* q_out, void* k_pages, void* v_pages, hpc_dtype kv_dtype,
+                        hpc_kv_layout kv_layout,
                         const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
                         const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
                         int32_t batch, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
@@ -260,8 +270,9 @@ HPC_API int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const fl
  * device memory.
  * It runs hpc_decode_plan, hpc_decode_attention and hpc_merge_states for one decode step.
  * The plan workspace and the partial states live in the library's static array of
- * HPC_NOALLOC_SCRATCH_BYTES; the caller passes only inputs (as in hpc_decode_attention,
- * plus batch, tile_len and num_ctas) and outputs (out, status). It allocates nothing.
+ * HPC_NOALLOC_SCRATCH_BYTES; the caller passes only inputs (as in hpc_decode_attention, with
+ * an HPC_HND cache, plus batch, tile_len and num_ctas) and outputs (out, status). It
+ * allocates nothing.
  *  - Needed scratch = plan workspace + max_items*group*(head_dim+2)*4 bytes (each part
  *    rounded up to 256), with max_items = num_ctas + batch*kv_heads. A shape that needs
  *    more than HPC_NOALLOC_SCRATCH_BYTES returns HPC_ERR_CAPACITY and launches nothing.

@@ -19,6 +19,8 @@ from .build import LIB
 
 HPC_OK, HPC_ERR_ARG, HPC_ERR_SHAPE, HPC_ERR_DTYPE, HPC_ERR_ALIGN, HPC_ERR_CUDA, HPC_ERR_CAPACITY = range(7)
 HPC_BF16, HPC_FP32, HPC_E4M3 = 0, 1, 2
+HPC_HND, HPC_NHD = 0, 1
+_LAYOUTS = {"HND": HPC_HND, "NHD": HPC_NHD}
 DEV_STATUS = {"bad_seqlen": 0x1, "bad_page": 0x2, "capacity": 0x4, "timeout": 0x8}
 ITEM_DTYPE = np.dtype([("req", "<i4"), ("kv_head", "<i2"), ("flags", "<i2"),
                        ("tile_begin", "<i4"), ("tile_end", "<i4")])
@@ -62,18 +64,18 @@ def _load():
         "hpc_plan_cpu": (ctypes.c_int, [vp, i32, i32, i32, i32, i32, i32, vp, sz, P, vp]),
         "hpc_partial_o_bytes": (sz, [P, i32, i32]),
         "hpc_partial_ml_bytes": (sz, [P, i32]),
-        "hpc_decode_attention": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp, i32,
-                                                vp, P, fp, vp, vp, vp, ctypes.c_int, vp, vp]),
+        "hpc_decode_attention": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32,
+                                                vp, i32, vp, P, fp, vp, vp, vp, ctypes.c_int, vp, vp]),
         "hpc_merge_states": (ctypes.c_int, [vp, vp, P, i32, i32, vp, ctypes.c_int, vp, vp]),
-        "hpc_decode_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, vp,
-                                               i32, vp, i32, i32, i32, i32, vp, vp]),
+        "hpc_decode_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32,
+                                               i32, vp, i32, vp, i32, i32, i32, i32, vp, vp]),
         "hpc_attention_launch_info": (ctypes.c_int, [i32, ctypes.c_int, i32, i32, i32, ctypes.POINTER(i32),
                                                      ctypes.POINTER(i32), ctypes.POINTER(i32)]),
         "hpc_decode_step_noalloc": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp,
                                                    i32, vp, i32, i32, i32, fp, vp, ctypes.c_int, vp, vp]),
         "hpc_decode_step_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
-        "hpc_decode_step": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp, i32, vp,
-                                           i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp]),
+        "hpc_decode_step": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp,
+                                           i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -234,9 +236,22 @@ def _kv_code(kv_dtype: str, t: torch.Tensor) -> int:
     return _KV_DTYPES[kv_dtype]
 
 
-def attention(q, k_pages, v_pages, block_table, seq_lens, p: Plan, *, kv_dtype="bf16", k_scale=None,
-              v_scale=None, sm_scale=None, out=None, out_dtype=torch.float32, partial_o=None, partial_ml=None,
-              status=None):
+def _geometry(k_pages, kv_layout):
+    """(num_pages, kv_heads, page_size, head_dim, layout code) of a cache tensor."""
+    if kv_layout not in _LAYOUTS:
+        raise HpcError(f"kv_layout must be one of {list(_LAYOUTS)}")
+    if k_pages.dim() != 4:
+        raise HpcError("cache must be 4-D")
+    if kv_layout == "HND":
+        n, hkv, psz, d = k_pages.shape
+    else:
+        n, psz, hkv, d = k_pages.shape
+    return n, hkv, psz, d, _LAYOUTS[kv_layout]
+
+
+def attention(q, k_pages, v_pages, block_table, seq_lens, p: Plan, *, kv_dtype="bf16", kv_layout="HND",
+              k_scale=None, v_scale=None, sm_scale=None, out=None, out_dtype=torch.float32, partial_o=None,
+              partial_ml=None, status=None):
     """Persistent split-KV attention (``hpc_decode_attention``). Returns (out, partial_o, partial_ml)."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
@@ -247,7 +262,7 @@ def attention(q, k_pages, v_pages, block_table, seq_lens, p: Plan, *, kv_dtype="
     code = _kv_code(kv_dtype, k_pages)
     _kv_code(kv_dtype, v_pages)
     B, Hq, D = q.shape
-    num_pages, Hkv, P, D2 = k_pages.shape
+    num_pages, Hkv, P, D2, lay = _geometry(k_pages, kv_layout)
     if D2 != D or v_pages.shape != k_pages.shape:
         raise HpcError("cache shape does not match q")
     if out is None:
@@ -261,7 +276,7 @@ def attention(q, k_pages, v_pages, block_table, seq_lens, p: Plan, *, kv_dtype="
         _need(v_scale, "v_scale", torch.float32, dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
     _check(_lib.hpc_decode_attention(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
         _ptr(block_table), block_table.shape[1], _ptr(seq_lens), ctypes.byref(p.raw), scale, _ptr(partial_o),
         _ptr(partial_ml), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
         _stream(dev)), "hpc_decode_attention")
@@ -283,7 +298,8 @@ def merge(p: Plan, partial_o, partial_ml, out, num_heads: int, status=None):
 
 
 def prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, *,
-             kv_dtype="bf16", k_scale=None, v_scale=None, eps=1e-6, rope_theta=1e6, q_out=None, status=None):
+             kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, eps=1e-6, rope_theta=1e6, q_out=None,
+             status=None):
     """Fused RMSNorm + RoPE + KV-page write of the new token (``hpc_decode_prologue``). Returns q_out."""
     _need(qkv, "qkv", torch.bfloat16)
     dev = qkv.device
@@ -295,13 +311,13 @@ def prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, n
     B, H, D = qkv.shape
     if H != num_heads + 2 * kv_heads:
         raise HpcError("qkv must hold num_heads + 2*kv_heads heads")
-    num_pages, Hkv, P, _ = k_pages.shape
+    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
     if q_out is None:
         q_out = torch.empty((B, num_heads, D), dtype=torch.bfloat16, device=dev)
     status = new_status(dev) if status is None else status
     _check(_lib.hpc_decode_prologue(
         _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(q_out), _ptr(k_pages),
-        _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, _ptr(block_table), block_table.shape[1],
+        _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, _ptr(block_table), block_table.shape[1],
         _ptr(seq_lens), B, num_heads, kv_heads, D, _ptr(status), _stream(dev)), "hpc_decode_prologue")
     return q_out
 
@@ -315,8 +331,8 @@ def step_workspace(batch, num_heads, kv_heads, head_dim, num_ctas, device):
 
 
 def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *,
-                      kv_dtype="bf16", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None,
-                      out_dtype=torch.float32, status=None, workspace=None):
+                      kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None,
+                      out=None, out_dtype=torch.float32, status=None, workspace=None):
     """One decode step in a single launch (``hpc_decode_step``): in-kernel planning, attention
     and ticket merge. Returns (out, status, workspace); pass the workspace back on later calls."""
     _need(q, "q", torch.bfloat16)
@@ -325,7 +341,7 @@ def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_
     _need(seq_lens, "seq_lens", torch.int32, dev)
     code = _kv_code(kv_dtype, k_pages)
     B, Hq, D = q.shape
-    num_pages, Hkv, P, _ = k_pages.shape
+    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
     if num_ctas is None:
         num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
     if out is None:
@@ -335,7 +351,7 @@ def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_
         workspace = step_workspace(B, Hq, Hkv, D, num_ctas, dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
     _check(_lib.hpc_decode_step(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
         _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
         workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
         _stream(dev)), "hpc_decode_step")
@@ -343,18 +359,18 @@ def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_
 
 
 def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",
-                k_scale=None, v_scale=None, num_ctas=None, out=None, out_dtype=torch.float32, status=None,
-                static_splits=None):
+                kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, out=None, out_dtype=torch.float32,
+                status=None, static_splits=None):
     """plan -> attention -> merge (three launches) for one decode step; returns (out, plan, status)."""
     dev = q.device
     status = new_status(dev) if status is None else status
-    max_seq = block_table.shape[1] * k_pages.shape[2]
+    max_seq = block_table.shape[1] * _geometry(k_pages, kv_layout)[2]
     if static_splits:
         p = plan_static(seq_lens, num_heads, kv_heads, tile_len, static_splits, max_seq, status)
     else:
         p = plan(seq_lens, num_heads, kv_heads, tile_len, num_ctas, max_seq, status)
-    out, po, pml = attention(q, k_pages, v_pages, block_table, seq_lens, p, kv_dtype=kv_dtype, k_scale=k_scale,
-                             v_scale=v_scale, out=out, out_dtype=out_dtype, status=status)
+    out, po, pml = attention(q, k_pages, v_pages, block_table, seq_lens, p, kv_dtype=kv_dtype, kv_layout=kv_layout,
+                             k_scale=k_scale, v_scale=v_scale, out=out, out_dtype=out_dtype, status=status)
     merge(p, po, pml, out, num_heads, status)
     return out, p, status
 

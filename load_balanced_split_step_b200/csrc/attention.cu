@@ -65,6 +65,7 @@ struct AttnParams {
   int32_t stages, out_bf16;
   uint32_t plane_bytes, stage_bytes;
   float score_scale;  // sm_scale * log2(e)
+  int32_t nhd;        // cache layout: token stride Hkv*D (NHD) or D (HND); only the TMA coordinates differ
   // single-launch step only: the plan is derived in the kernel from seq_lens
   int32_t batch, kv_heads, max_seq_len;
   int32_t* tickets;  // [batch * kv_heads], zero between steps
@@ -641,14 +642,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (bi < 64) par_lo ^= uint64_t(1) << bi;
             else par_hi ^= uint64_t(1) << (bi - 64);
             const uint32_t dst = ring_u32 + stage * p.stage_bytes;
+            // tensor-map coordinates: (d, token, kv head, page) for HND, (d, kv head, token, page) for NHD
+            const int c1 = p.nhd ? x.kvh : off, c2 = p.nhd ? off : x.kvh;
             mbar_arrive_expect_tx(full, p.stage_bytes);
 #pragma unroll
             for (int pl = 0; pl < S::kPlanes; ++pl)
-              tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), off, x.kvh, page, policy);
+              tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), c1, c2, page, policy);
 #pragma unroll
             for (int pl = 0; pl < S::kPlanes; ++pl)
-              tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), off, x.kvh,
-                          page, policy);
+              tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), c1, c2, page,
+                          policy);
             ++issued;
             if (++stage == stages) {
               stage = 0;
@@ -842,22 +845,48 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Tensor map of a page pool [num_pages][Hkv][P][D]. Each box is 128 bytes of one token
-// row x `box_tokens` tokens of one (page, kv head), stored with the 128-byte swizzle.
-int make_pool_map(CUtensorMap* map, const void* base, bool fp8, int D, int P, int Hkv, int num_pages,
+// Tensor map of a page pool, HND [num_pages][Hkv][P][D] or NHD [num_pages][P][Hkv][D]. Each box
+// is 128 bytes of one token row x `box_tokens` tokens of one (page, kv head), stored with the
+// 128-byte swizzle. Dimensions are listed innermost first: (D, P, Hkv, pages) for HND and
+// (D, Hkv, P, pages) for NHD, so the same box lands in shared memory in the same layout.
+int make_pool_map(CUtensorMap* map, const void* base, bool fp8, bool nhd, int D, int P, int Hkv, int num_pages,
                   int box_tokens) {
   auto fn = encode_fn();
   if (!fn) return fail(HPC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const int elt = fp8 ? 1 : 2;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(Hkv),
-                        static_cast<cuuint64_t>(num_pages)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * elt, static_cast<cuuint64_t>(P) * D * elt,
-                           static_cast<cuuint64_t>(Hkv) * P * D * elt};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elt), static_cast<cuuint32_t>(box_tokens), 1, 1};
+  const cuuint64_t row = static_cast<cuuint64_t>(D) * elt;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  dims[0] = static_cast<cuuint64_t>(D);
+  dims[3] = static_cast<cuuint64_t>(num_pages);
+  box[0] = static_cast<cuuint32_t>(128 / elt);
+  box[3] = 1;
+  if (nhd) {
+    dims[1] = static_cast<cuuint64_t>(Hkv);
+    dims[2] = static_cast<cuuint64_t>(P);
+    strides[0] = row;
+    strides[1] = row * Hkv;
+    strides[2] = row * Hkv * P;
+    box[1] = 1;
+    box[2] = static_cast<cuuint32_t>(box_tokens);
+  } else {
+    dims[1] = static_cast<cuuint64_t>(P);
+    dims[2] = static_cast<cuuint64_t>(Hkv);
+    strides[0] = row;
+    strides[1] = row * P;
+    strides[2] = row * P * Hkv;
+    box[1] = static_cast<cuuint32_t>(box_tokens);
+    box[2] = 1;
+  }
   cuuint32_t estr[4] = {1, 1, 1, 1};
+  // L2 fetch granularity: 256 B when a box row is followed in memory by data the same stream
+  // reads (HND rows are contiguous, and a bf16 NHD row is 256 B read as two 128 B boxes).
+  // An E4M3 NHD row is 128 B followed by another kv head's row, so 128 B.
+  const CUtensorMapL2promotion promo =
+      (nhd && row <= 128) ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
   CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_SWIZZLE_128B, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(HPC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return HPC_OK;
 }
@@ -944,7 +973,8 @@ namespace {
 
 // Checks shared by the attention entry points; fills the tensor maps, launch shape and the
 // common kernel parameters.
-int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype, const float* k_scale,
+int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype, hpc_kv_layout kv_layout,
+            const float* k_scale,
             const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads, int32_t kv_heads,
             int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
             int32_t tile_len, int32_t grid, bool persistent, float sm_scale, void* out, hpc_dtype out_dtype,
@@ -953,7 +983,9 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
     return fail(HPC_ERR_ARG, "null pointer argument");
   if (kv_dtype != HPC_BF16 && kv_dtype != HPC_E4M3) return fail(HPC_ERR_DTYPE, "kv_dtype must be BF16 or E4M3");
   if (out_dtype != HPC_FP32 && out_dtype != HPC_BF16) return fail(HPC_ERR_DTYPE, "out_dtype must be FP32 or BF16");
+  if (kv_layout != HPC_HND && kv_layout != HPC_NHD) return fail(HPC_ERR_ARG, "kv_layout must be HND or NHD");
   const bool fp8 = kv_dtype == HPC_E4M3;
+  const bool nhd = kv_layout == HPC_NHD;
   if (fp8 && (!k_scale || !v_scale)) return fail(HPC_ERR_ARG, "E4M3 cache needs k_scale and v_scale");
   if (num_pages < 1 || max_pages_per_req < 1 || num_heads < 1 || kv_heads < 1 || grid < 1)
     return fail(HPC_ERR_ARG, "sizes must be >= 1");
@@ -977,8 +1009,8 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   if (ctas_per_sm > 4) ctas_per_sm = 4;
   int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, ls);
   if (rc) return rc;
-  if ((rc = make_pool_map(mk, k_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
-  if ((rc = make_pool_map(mv, v_pages, fp8, head_dim, page_size, kv_heads, num_pages, C))) return rc;
+  if ((rc = make_pool_map(mk, k_pages, fp8, nhd, head_dim, page_size, kv_heads, num_pages, C))) return rc;
+  if ((rc = make_pool_map(mv, v_pages, fp8, nhd, head_dim, page_size, kv_heads, num_pages, C))) return rc;
 
   *prm = AttnParams{};
   prm->q = static_cast<const __nv_bfloat16*>(q);
@@ -1002,6 +1034,7 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   prm->score_scale = sm_scale * kLog2e;
   prm->kv_heads = kv_heads;
   prm->max_seq_len = max_pages_per_req * page_size;
+  prm->nhd = nhd ? 1 : 0;
   return HPC_OK;
 }
 
@@ -1031,7 +1064,7 @@ StepLayout step_layout(int32_t batch, int32_t group, int32_t kv_heads, int32_t h
 }  // namespace hpc
 
 extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
-                                    const float* k_scale, const float* v_scale, int32_t num_pages,
+                                    hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages,
                                     int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
                                     const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
                                     const hpc_plan* plan, float sm_scale, float* partial_o, float* partial_ml,
@@ -1042,7 +1075,8 @@ extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const vo
   CUtensorMap mk, mv;
   LaunchShape ls;
   AttnParams prm;
-  int rc = prepare(q, k_pages, v_pages, kv_dtype, k_scale, v_scale, num_pages, page_size, num_heads, kv_heads,
+  int rc = prepare(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads,
                    head_dim, block_table, max_pages_per_req, seq_lens, plan->tile_len, plan->num_ctas,
                    !plan->is_static, sm_scale, out, out_dtype, status, &mk, &mv, &ls, &prm);
   if (rc) return rc;
@@ -1062,7 +1096,7 @@ extern "C" size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_hea
 }
 
 extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
-                               const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                               hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
                                int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                                int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
                                int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
@@ -1075,7 +1109,8 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
   CUtensorMap mk, mv;
   LaunchShape ls;
   AttnParams prm;
-  int rc = prepare(q, k_pages, v_pages, kv_dtype, k_scale, v_scale, num_pages, page_size, num_heads, kv_heads,
+  int rc = prepare(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads,
                    head_dim, block_table, max_pages_per_req, seq_lens, tile_len, num_ctas, true, sm_scale, out,
                    out_dtype, status, &mk, &mv, &ls, &prm);
   if (rc) return rc;

@@ -91,7 +91,7 @@ extern "C" int hpc_decode_step_noalloc(const void* q, const void* k_pages, const
   rc = hpc_decode_plan(seq_lens, batch, num_heads, kv_heads, tile_len, num_ctas, max_pages_per_req * page_size,
                        plan_ws, plan_bytes, &plan, status, stream);
   if (rc) return rc;
-  rc = hpc_decode_attention(q, k_pages, v_pages, kv_dtype, k_scale, v_scale, num_pages, page_size, num_heads,
+  rc = hpc_decode_attention(q, k_pages, v_pages, kv_dtype, HPC_HND, k_scale, v_scale, num_pages, page_size, num_heads,
                             kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, &plan, sm_scale, partial_o,
                             partial_ml, out, out_dtype, status, stream);
   if (rc) return rc;

@@ -2,7 +2,7 @@
 //
 // "vLLM × HPC-Ops: High-Performance Attention and MoE Backends from Tencent Hunyuan" (8sync
 // News summary) names a fused RoPE + QK-Norm + KV-write prologue in front of the attention
-// backend. One CTA handles one request. The NeoX rotation angles pos * theta^(-2i/D) are
+// backend. One CTA handles one request; the cache may be HND or NHD. The NeoX rotation angles pos * theta^(-2i/D) are
 // evaluated once per request in fp64, because pos reaches 1e5 and an fp32 angle would lose
 // ~1e-3 rad. They are shared through shared memory. Each warp takes one head at a time:
 // q and k heads are RMS-normalised and rotated, v heads copied. q goes out as bf16; k and
@@ -21,7 +21,8 @@ __global__ void __launch_bounds__(kProWarps * 32)
                     const float* __restrict__ k_norm_w, float eps, double theta, __nv_bfloat16* __restrict__ q_out,
                     void* __restrict__ k_pages, void* __restrict__ v_pages, int fp8, const float* __restrict__ k_scale,
                     const float* __restrict__ v_scale, int32_t num_pages, int32_t P, const int32_t* __restrict__ block_table,
-                    int64_t max_pages, const int32_t* __restrict__ seq_lens, int32_t Hq, int32_t Hkv, uint32_t* status) {
+                    int64_t max_pages, const int32_t* __restrict__ seq_lens, int32_t Hq, int32_t Hkv, int nhd,
+                    uint32_t* status) {
   constexpr int PER = D / 32;  // elements per lane: d = lane + 32 k
   constexpr int HALF = PER / 2;
   __shared__ float s_cos[D / 2], s_sin[D / 2];
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(kProWarps * 32)
     if (!page_ok) continue;
     const bool is_k = h < Hq + Hkv;
     const int g = is_k ? h - Hq : h - Hq - Hkv;
-    const int64_t base = ((static_cast<int64_t>(page) * Hkv + g) * P + slot) * D;
+    const int64_t base = nhd ? ((static_cast<int64_t>(page) * P + slot) * Hkv + g) * D
+                             : ((static_cast<int64_t>(page) * Hkv + g) * P + slot) * D;
     if (fp8) {
       const float sc = is_k ? k_scale[g] : v_scale[g];
       uint8_t* dst = static_cast<uint8_t*>(is_k ? k_pages : v_pages) + base;
@@ -102,13 +104,14 @@ using namespace hpc;
 
 extern "C" int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,
                                    float rope_theta, void* q_out, void* k_pages, void* v_pages, hpc_dtype kv_dtype,
-                                   const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                                   hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
                                    const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
                                    int32_t batch, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
                                    uint32_t* status, void* stream) {
   if (!qkv || !q_norm_w || !k_norm_w || !q_out || !k_pages || !v_pages || !block_table || !seq_lens || !status)
     return fail(HPC_ERR_ARG, "null pointer argument");
   if (kv_dtype != HPC_BF16 && kv_dtype != HPC_E4M3) return fail(HPC_ERR_DTYPE, "kv_dtype must be BF16 or E4M3");
+  if (kv_layout != HPC_HND && kv_layout != HPC_NHD) return fail(HPC_ERR_ARG, "kv_layout must be HND or NHD");
   const bool fp8 = kv_dtype == HPC_E4M3;
   if (fp8 && (!k_scale || !v_scale)) return fail(HPC_ERR_ARG, "E4M3 cache needs k_scale and v_scale");
   if (batch < 1 || num_heads < 1 || kv_heads < 1 || num_pages < 1 || page_size < 1 || max_pages_per_req < 1)
@@ -123,7 +126,8 @@ extern "C" int hpc_decode_prologue(const void* qkv, const float* q_norm_w, const
   const cudaError_t e = launch_pdl(kern, dim3(batch), dim3(kProWarps * 32), 0, st, x, q_norm_w, k_norm_w, eps,
                                    static_cast<double>(rope_theta), qo, k_pages, v_pages, static_cast<int>(fp8),
                                    k_scale, v_scale, num_pages, page_size, block_table,
-                                   static_cast<int64_t>(max_pages_per_req), seq_lens, num_heads, kv_heads, status);
+                                   static_cast<int64_t>(max_pages_per_req), seq_lens, num_heads, kv_heads,
+                                   static_cast<int>(kv_layout == HPC_NHD), status);
   if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "prologue_kernel: %s", cudaGetErrorString(e));
   return check_launch("prologue_kernel");
 }

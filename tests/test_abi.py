@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 1
+    assert B._lib.hpc_abi_version() == 2
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -52,7 +52,7 @@ def test_host_argument_errors_return_codes(B):
     P = B.CPlan()
     i32 = ctypes.c_int32
     # null pointers -> HPC_ERR_ARG before any CUDA call
-    rc = B._lib.hpc_decode_attention(None, None, None, 0, None, None, 1, 16, 8, 2, 64, None, 1, None,
+    rc = B._lib.hpc_decode_attention(None, None, None, 0, 0, None, None, 1, 16, 8, 2, 64, None, 1, None,
                                      ctypes.byref(P), 0.1, None, None, None, 1, None, None)
     assert rc == B.HPC_ERR_ARG
     assert "null" in B._lib.hpc_last_error().decode()
