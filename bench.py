@@ -55,9 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--tile-len", type=int, default=0)
     ap.add_argument("--ctas-per-sm", type=int, default=1)
     ap.add_argument("--layout", default="HND", choices=["HND", "NHD"], help="KV cache page layout")
-    ap.add_argument("--path", default="fused", choices=["fused", "split"],
-                    help="fused: one launch per step (in-kernel plan + ticket merge); split: plan, attention and "
-                         "merge kernels")
+    ap.add_argument("--path", default="fused", choices=["fused", "folded", "split"],
+                    help="fused: one launch per step (in-kernel plan + ticket merge), after the prologue kernel on "
+                         "the FP8 workload; folded: the same with the prologue folded into that launch; split: "
+                         "plan, attention and merge kernels")
     ap.add_argument("--no-extras", action="store_true", help="skip static split-k, e2e and CPU baseline legs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     return ap.parse_args(argv)
@@ -162,11 +163,13 @@ class ClockSampler:
 class Step:
     """One decode step through the binding, with buffers allocated once."""
 
-    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None, fused=False, layout="HND"):
+    def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None, fused=False, layout="HND",
+                 folded=False):
         self.B, self.spec, self.dc = B, spec, dc
         self.layout = layout
         self.tl = tile_len
-        self.fused = fused and not static_splits
+        self.fused = (fused or folded) and not static_splits
+        self.folded = folded and self.fused and spec.prologue
         dev = dc["seq_lens"].device
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.max_seq = dc["block_table"].shape[1] * spec.page_size
@@ -190,6 +193,17 @@ class Step:
     def __call__(self, seq_lens=None, ev=None):
         B, s, dc = self.B, self.spec, self.dc
         seq = dc["seq_lens"] if seq_lens is None else seq_lens
+        if self.folded:  # one launch: the prologue is folded into the step
+            if ev is not None:
+                ev[0].record()
+            B.decode_step_prologue(dc["qkv"], dc["q_norm_w"], dc["k_norm_w"], dc["k_pages"], dc["v_pages"],
+                                   dc["block_table"], seq, s.num_heads, s.kv_heads, self.tl, kv_dtype=s.kv_dtype,
+                                   kv_layout=self.layout, k_scale=dc["k_scale"], v_scale=dc["v_scale"],
+                                   eps=s.rms_eps, rope_theta=s.rope_theta, num_ctas=self.num_ctas, out=self.out,
+                                   status=self.status, workspace=self.ws)
+            if ev is not None:
+                ev[1].record()
+            return self.out
         if s.prologue:
             B.prologue(dc["qkv"], dc["q_norm_w"], dc["k_norm_w"], dc["k_pages"], dc["v_pages"], dc["block_table"],
                        seq, s.num_heads, s.kv_heads, kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
@@ -223,8 +237,8 @@ class Step:
 
     @property
     def launches(self):
-        n = 1 if self.fused else 3
-        return n + (1 if self.spec.prologue else 0)
+        pro = 1 if self.spec.prologue and not self.folded else 0
+        return (1 if self.fused else 3) + pro
 
 
 def step_lengths(dc, spec):
@@ -266,7 +280,7 @@ def static_leg(B, spec, dc, tl, steps, sms, layout="HND"):
             "sweep_us": {str(k): round(v, 2) for k, v in res.items()}}
 
 
-def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND"):
+def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND", folded=False):
     """Same metric through the public call, with per-step H2D of the step inputs (q or qkv,
     seq_lens, block_table) from pinned host memory and D2H of the output. The KV cache is
     device-resident decode state and is not copied. The step runs as a serving loop would:
@@ -304,12 +318,20 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
             s_cmp.wait_event(ev_in[b])
             s_cmp.wait_event(ev_out[b])  # step i-2's output has left this buffer
             q = d["q"]
-            if spec.prologue:
+            if folded and spec.prologue:
+                B.decode_step_prologue(d["qkv"], d["q_norm_w"], d["k_norm_w"], d["k_pages"], d["v_pages"],
+                                       d["block_table"], d["seq_lens"], spec.num_heads, spec.kv_heads, tl,
+                                       kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
+                                       v_scale=d["v_scale"], eps=spec.rms_eps, rope_theta=spec.rope_theta,
+                                       num_ctas=num_ctas, out=outs[b], workspace=ws)
+            elif spec.prologue:
                 q = B.prologue(d["qkv"], d["q_norm_w"], d["k_norm_w"], d["k_pages"], d["v_pages"], d["block_table"],
                                d["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype, kv_layout=layout,
                                k_scale=d["k_scale"], v_scale=d["v_scale"], eps=spec.rms_eps,
                                rope_theta=spec.rope_theta, q_out=qbufs[b])
-            if fused:
+            if folded and spec.prologue:
+                pass  # done above, in one launch
+            elif fused:
                 B.decode_step_fused(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
                                     spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
                                     v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws)
@@ -433,7 +455,7 @@ def run_ours(args, rank, world, local):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     tl = args.tile_len or spec.tile_len
     G = sms * args.ctas_per_sm
-    step = Step(B, spec, dc, G, tl, fused=args.path == "fused", layout=args.layout)
+    step = Step(B, spec, dc, G, tl, fused=args.path == "fused", folded=args.path == "folded", layout=args.layout)
     lens = step_lengths(dc, spec)
     K, W_ = args.steps, max(3, args.warmup)
 
@@ -481,8 +503,8 @@ def run_ours(args, rank, world, local):
         del g
         extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms, args.layout)
         extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step), 3)
-    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path == "fused",
-                               layout=args.layout)
+    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path != "split",
+                               layout=args.layout, folded=args.path == "folded")
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_steps = max(50, K // 4)
     e2e_val = world * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
@@ -499,15 +521,19 @@ def run_ours(args, rank, world, local):
         "data": "synthetic (seeded N(0,1), bf16-rounded; random page permutation)",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "tile_len": tl, "num_ctas": G,
                    "plan": "dynamic (re-planned on the device every step)",
-                   "path": ("single launch: in-kernel plan, attention, ticket merge" if args.path == "fused"
-                            else "plan, attention and merge kernels chained by PDL"),
+                   "path": ({"fused": "single launch: in-kernel plan, attention, ticket merge"
+                                      + (" (after the prologue kernel, PDL)" if spec.prologue else ""),
+                             "folded": "single launch: prologue, in-kernel plan, attention, ticket merge",
+                             "split": "plan, attention and merge kernels chained by PDL"
+                                      + (" after the prologue kernel" if spec.prologue else "")}[args.path]),
                    "kv_layout": args.layout,
                    "l2": f"inputs larger than L2 ({bytes_step / 1e9:.2f} GB per step), no flush",
                    "parallelism": f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8000": round(achieved / 8000.0, 4),
-                     "kernel": "decode_attention_kernel" + ("<fused>" if args.path == "fused" else ""),
+                     "kernel": "decode_attention_kernel" + {"fused": "<fused>", "folded": "<fused, prologue>",
+                                                            "split": ""}[args.path],
                      "kernel_us": round(1000 * kern_ms, 2),
                      "traffic": load_traffic(args.workload)},
         "cpu_baseline": cpu,

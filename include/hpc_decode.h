@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 2
+#define HPC_DECODE_ABI_VERSION 3
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -223,6 +223,33 @@ HPC_API int hpc_decode_step(const void* q, const void* k_pages, const void* v_pa
                             int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
                             int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
                             hpc_dtype out_dtype, uint32_t* status, void* stream);
+
+/* hpc_decode_step with the decode prologue folded in ("vLLM × HPC-Ops" summary: "RoPE +
+ * QK-Norm + KV-write" in front of attention). One launch does what hpc_decode_prologue followed
+ * by hpc_decode_step does, without the q_out round trip through memory:
+ *  - For each (request r, kv head) the CTA that owns its last tile writes request r's new token
+ *    (position pos = seq_lens[r] - 1) into the cache for that kv head, with the arithmetic of
+ *    hpc_decode_prologue: k through RMSNorm (k_norm_w, eps) and NeoX RoPE at pos, v as is, both
+ *    as bf16 or E4M3 codes of x / scale. That CTA then reads the token back through its TMA
+ *    stream; no other CTA reads it.
+ *  - The attention query of every item is formed in registers from qkv: RMSNorm (q_norm_w),
+ *    RoPE at pos (angles pos * theta^(-2i/D) evaluated in fp64), rounded to bf16.
+ *  - qkv: device bf16 [batch][num_heads + 2*kv_heads][head_dim], 16-byte aligned.
+ *    q_norm_w, k_norm_w: device float [head_dim]. eps >= 0, rope_theta > 0.
+ *  - k_pages / v_pages are written (one token slot per request and kv head) and read.
+ *  - seq_lens[r] must count the new token. seq_lens[r] = 0 sets HPC_DEV_BAD_SEQLEN (there is no
+ *    token to decode) and gives a zero output row; a page id out of range sets
+ *    HPC_DEV_BAD_PAGE and skips that write.
+ *  - Everything else (workspace, batch limit, tickets) as hpc_decode_step. The rotated q is not
+ *    written out. */
+HPC_API int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,
+                                     float rope_theta, void* k_pages, void* v_pages, hpc_dtype kv_dtype,
+                                     hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale,
+                                     int32_t num_pages, int32_t page_size, int32_t num_heads, int32_t kv_heads,
+                                     int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
+                                     const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
+                                     float sm_scale, void* workspace, size_t workspace_bytes, void* out,
+                                     hpc_dtype out_dtype, uint32_t* status, void* stream);
 
 /* ---- merge --------------------------------------------------------------------------- */
 

@@ -29,7 +29,7 @@ EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_d
            "hpc_decode_plan_static", "hpc_plan_cpu", "hpc_partial_o_bytes", "hpc_partial_ml_bytes",
            "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue", "hpc_attention_launch_info",
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
-           "hpc_decode_step", "hpc_decode_step_workspace_bytes")
+           "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue")
 
 
 class HpcError(RuntimeError):
@@ -76,6 +76,9 @@ def _load():
         "hpc_decode_step_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
         "hpc_decode_step": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp,
                                            i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp]),
+        "hpc_decode_step_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp,
+                                                    i32, i32, i32, i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz,
+                                                    vp, ctypes.c_int, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -355,6 +358,41 @@ def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_
         _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
         workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
         _stream(dev)), "hpc_decode_step")
+    return out, status, workspace
+
+
+def decode_step_prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads,
+                         tile_len, *, kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, eps=1e-6,
+                         rope_theta=1e6, num_ctas=None, sm_scale=None, out=None, out_dtype=torch.float32,
+                         status=None, workspace=None):
+    """One decode step in a single launch with the prologue folded in
+    (``hpc_decode_step_prologue``): the new token's K/V go into the cache and q is formed from
+    qkv inside the attention kernel. Returns (out, status, workspace)."""
+    _need(qkv, "qkv", torch.bfloat16)
+    dev = qkv.device
+    _need(q_norm_w, "q_norm_w", torch.float32, dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    code = _kv_code(kv_dtype, k_pages)
+    B, H, D = qkv.shape
+    if H != num_heads + 2 * kv_heads:
+        raise HpcError("qkv must hold num_heads + 2*kv_heads heads")
+    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
+    if num_ctas is None:
+        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    if out is None:
+        out = torch.empty((B, num_heads, D), dtype=out_dtype, device=dev)
+    status = new_status(dev) if status is None else status
+    if workspace is None:
+        workspace = step_workspace(B, num_heads, Hkv, D, num_ctas, dev)
+    scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    _check(_lib.hpc_decode_step_prologue(
+        _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(k_pages), _ptr(v_pages), code,
+        lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, num_heads, Hkv, D, _ptr(block_table), block_table.shape[1],
+        _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace), workspace.numel(), _ptr(out),
+        HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status), _stream(dev)),
+        "hpc_decode_step_prologue")
     return out, status, workspace
 
 

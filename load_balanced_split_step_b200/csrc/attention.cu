@@ -69,6 +69,15 @@ struct AttnParams {
   // single-launch step only: the plan is derived in the kernel from seq_lens
   int32_t batch, kv_heads, max_seq_len;
   int32_t* tickets;  // [batch * kv_heads], zero between steps
+  // single-launch step with the prologue folded in: q comes from qkv through RMSNorm and RoPE,
+  // and the new token's K/V are written into the cache
+  const __nv_bfloat16* qkv;  // [batch][num_heads + 2 kv_heads][D]
+  const float* q_norm_w;
+  const float* k_norm_w;
+  void* k_pages_w;  // the caches, for the new token's write
+  void* v_pages_w;
+  float eps;
+  double rope_theta;
 };
 
 // One work item as the producer and the consumers see it.
@@ -80,6 +89,15 @@ struct ItemInfo {
   int64_t U;           // single-launch step: first unit of the (request, kv head) segment
   int32_t nt;          // and its tile count
 };
+
+// 16-token blocks that one consumer warp takes from a stage of `bpc` blocks. Two blocks give
+// two independent MMA chains. An E4M3 stage carries half the bytes per token, so the fixed
+// per-call softmax work (row max across lanes, rescale factors) and the stage handshake weigh
+// twice as much per byte: there a warp takes up to four blocks, a whole 64-token stage.
+__host__ __device__ __forceinline__ int blocks_per_warp(int bpc, bool fp8) {
+  if (fp8 && bpc >= 4) return 4;
+  return bpc >= 2 ? 2 : 1;
+}
 
 __device__ __forceinline__ int32_t tiles_of(int32_t L, int32_t tl) {
   return L > 0 ? static_cast<int32_t>(static_cast<uint32_t>(L - 1) / static_cast<uint32_t>(tl) + 1) : 0;
@@ -547,16 +565,164 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
   }
 }
 
-template <int D, bool FP8, bool FUSED>
+// ---- prologue folded into the single-launch step
+// "vLLM × HPC-Ops" (8sync News summary) puts a RoPE + QK-Norm + KV-write prologue in front of
+// attention. Folded in, it costs no launch and no pass over q through HBM:
+//  * The CTA that owns the last tile of a (request, kv head) writes that request's new token
+//    (position L - 1) into the cache for this kv head: k through RMSNorm and RoPE, v as is,
+//    both as bf16 or E4M3 codes of x / scale. No other CTA reads that token. Its consumer
+//    warps do these writes when the kernel starts, fence them against the async proxy and
+//    arrive on an mbarrier; the producer waits on it before it requests the chunk that holds
+//    the token. (Done by the producer itself, the write's loads and fp64 angles would stall
+//    the TMA stream at every segment end.)
+//  * Each item's consumers form q from qkv in registers: RMSNorm, NeoX RoPE at L - 1, rounded
+//    to bf16 as the prologue kernel's q_out. The rotation table of an item (cos, sin of
+//    pos * theta^(-2i/D), evaluated in fp64) is built by 64 consumer threads during the item
+//    before, so it is ready when the item starts.
+// Arithmetic follows hpc_decode_prologue (same formulas; the new K/V bytes use its lane order).
+
+// Rotation table of position pos into cs / sn (D/2 floats each), by threads t < D/2.
+template <int D>
+__device__ __forceinline__ void rope_table(int64_t pos, const double* inv_freq, float* cs, float* sn, int t) {
+  if (t < D / 2) {
+    double a, b;
+    sincos(static_cast<double>(pos) * inv_freq[t], &a, &b);
+    sn[t] = static_cast<float>(a);
+    cs[t] = static_cast<float>(b);
+  }
+}
+
+// New token of request r, kv head kvh: one warp. Lane holds d = lane + 32 j, as in
+// hpc_decode_prologue, and the arithmetic is the same.
+template <int D, bool FP8>
+__device__ void write_new_token(const AttnParams& p, int r, int kvh, const double* inv_freq, int lane) {
+  constexpr int PER = D / 32, HALF = PER / 2;
+  const int64_t pos = static_cast<int64_t>(p.seq_lens[r]) - 1;  // >= 0: the request owns tiles
+  const int32_t page = p.block_table[r * p.max_pages + pos / p.page_size];
+  if (page < 0 || page >= p.num_pages) {
+    if (lane == 0) atomicOr(p.status, HPC_DEV_BAD_PAGE);
+    return;
+  }
+  const int slot = static_cast<int>(pos % p.page_size);
+  const int64_t heads = p.num_heads + 2 * p.kv_heads;
+  const __nv_bfloat16* kx = p.qkv + (static_cast<int64_t>(r) * heads + p.num_heads + kvh) * D;
+  const __nv_bfloat16* vx = kx + static_cast<int64_t>(p.kv_heads) * D;
+  float k[PER], v[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    k[j] = __bfloat162float(kx[lane + 32 * j]);
+    v[j] = __bfloat162float(vx[lane + 32 * j]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) ss += k[j] * k[j];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = 1.f / sqrtf(ss / D + p.eps);
+#pragma unroll
+  for (int j = 0; j < PER; ++j) k[j] = k[j] * inv * p.k_norm_w[lane + 32 * j];
+#pragma unroll
+  for (int j = 0; j < HALF; ++j) {
+    double a, b;
+    sincos(static_cast<double>(pos) * inv_freq[lane + 32 * j], &a, &b);
+    const float cs = static_cast<float>(b), sn = static_cast<float>(a);
+    const float x1 = k[j], x2 = k[j + HALF];
+    k[j] = x1 * cs - x2 * sn;
+    k[j + HALF] = x2 * cs + x1 * sn;
+  }
+  const int64_t base = p.nhd ? ((static_cast<int64_t>(page) * p.page_size + slot) * p.kv_heads + kvh) * D
+                             : ((static_cast<int64_t>(page) * p.kv_heads + kvh) * p.page_size + slot) * D;
+  if (FP8) {
+    const float ks = p.k_scale[kvh], vs = p.v_scale[kvh];
+    uint8_t* kd = static_cast<uint8_t*>(p.k_pages_w) + base;
+    uint8_t* vd = static_cast<uint8_t*>(p.v_pages_w) + base;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      kd[lane + 32 * j] = f32_to_e4m3(k[j] / ks);
+      vd[lane + 32 * j] = f32_to_e4m3(v[j] / vs);
+    }
+  } else {
+    __nv_bfloat16* kd = static_cast<__nv_bfloat16*>(p.k_pages_w) + base;
+    __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(p.v_pages_w) + base;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      kd[lane + 32 * j] = __float2bfloat16_rn(k[j]);
+      vd[lane + 32 * j] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
+
+// Element index d of q fragment element (ks, e), e = 0..3, for lane column c: the bf16 path
+// holds pairs (16ks + 2c, +1) and (16ks + 8 + 2c, +1); the E4M3 path (16ks + 4c, +1, +2, +3).
+// Element (ks + KSTEPS/2, e) is d + D/2: each lane holds both halves of its RoPE pairs.
+template <bool FP8>
+__device__ __forceinline__ int q_elem_d(int ks, int e, int c) {
+  if (FP8) return 16 * ks + 4 * c + e;
+  return 16 * ks + 2 * c + (e & 1) + 8 * (e >> 1);
+}
+
+// q fragments of an item from qkv: RMSNorm (q_norm_w, eps), RoPE from the item's table,
+// rounded to bf16 (then to f16 for an E4M3 cache). Lanes of rows g >= group get zeros.
+template <int D, bool FP8>
+__device__ __forceinline__ void q_from_qkv(const AttnParams& p, int req, int head, bool live, const float* qw,
+                                           const float* cs, const float* sn, int c, uint32_t (&qf)[D / 16][2]) {
+  constexpr int KSTEPS = D / 16;
+  const int64_t heads = p.num_heads + 2 * p.kv_heads;
+  const __nv_bfloat16* src = p.qkv + (static_cast<int64_t>(req) * heads + (live ? head : 0)) * D;
+  float x[KSTEPS][4];
+  float ss = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks) {
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const uint32_t w = live ? *reinterpret_cast<const uint32_t*>(src + q_elem_d<FP8>(ks, e, c)) : 0u;
+      x[ks][e] = __uint_as_float(w << 16);
+      x[ks][e + 1] = __uint_as_float(w & 0xffff0000u);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ss += x[ks][e] * x[ks][e];
+  }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);  // the four lanes of one row hold the whole head
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  const float inv = 1.f / sqrtf(ss / D + p.eps);
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[ks][e] = x[ks][e] * inv * qw[q_elem_d<FP8>(ks, e, c)];
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS / 2; ++ks)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = q_elem_d<FP8>(ks, e, c);
+      const float x1 = x[ks][e], x2 = x[ks + KSTEPS / 2][e];
+      x[ks][e] = x1 * cs[i] - x2 * sn[i];
+      x[ks + KSTEPS / 2][e] = x2 * cs[i] + x1 * sn[i];
+    }
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks) {
+    const uint32_t lo = live ? pack_bf16x2(x[ks][0], x[ks][1]) : 0u;
+    const uint32_t hi = live ? pack_bf16x2(x[ks][2], x[ks][3]) : 0u;
+    qf[ks][0] = FP8 ? bf16x2_to_f16x2(lo) : lo;
+    qf[ks][1] = FP8 ? bf16x2_to_f16x2(hi) : hi;
+  }
+}
+
+template <int D, bool FP8, bool FUSED, bool PRO>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                             const AttnParams p) {
+  static_assert(FUSED || !PRO, "the prologue is folded into the single-launch step only");
   using S = Shape<D, FP8>;
   using Cursor = typename CursorOf<FUSED>::type;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int64_t s_scan[16], s_walk[8];
   __shared__ int s_flag;
   __shared__ int32_t s_pages[32];
+  // folded prologue: q_norm_w, theta^(-2i/D), two rotation tables [cos | sin], new-token barrier
+  __shared__ float s_qw[PRO ? D : 1];
+  __shared__ double s_invf[PRO ? D / 2 : 1];
+  __shared__ float s_rope[PRO ? 2 * D : 1];
+  __shared__ uint64_t s_pro_bar;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stages = p.stages;
   uint8_t* ring = smem;
@@ -569,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barriers in order, and a parity wait can never match a phase two behind.
   uint64_t* bars = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * 8);
   const int bpc = p.chunk_tokens / 16;          // 16-token blocks per stage
-  const int nb = bpc >= 2 ? 2 : 1;              // blocks per warp per stage
+  const int nb = blocks_per_warp(bpc, FP8);     // 16-token blocks per warp per stage
   const int wps = bpc / nb;                     // warps per stage
   const int groups = kConsumerWarps / wps;
 
@@ -580,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages * groups; ++s) mbar_init(full0 + 8 * s, 1);
     for (int s = 0; s < stages; ++s) mbar_init(empty0 + 8 * s, wps);
+    if (PRO) mbar_init(smem_u32(&s_pro_bar), kConsumerWarps);
     fence_barrier_init();
   }
   if (threadIdx.x == kConsumerWarps * 32) {
@@ -617,47 +784,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t issued = 0;
     bool ok = true;
     uint32_t bad = 0;
+    bool pro_done = !PRO;  // the new tokens of this CTA's segments are in the cache
     ItemInfo x;
     while (ok && cursor.next(p, x)) {
+      const bool has_new = PRO && x.tok1 == p.seq_lens[x.req];  // the item holds token L - 1
       const int32_t* bt = p.block_table + x.req * p.max_pages + (x.tok0 >> p_shift);
       const int off0 = static_cast<int>(x.tok0 & (P - 1));
       const int64_t nchunks = x.tok1 > x.tok0 ? (x.tok1 - x.tok0 + C - 1) / C : 0;
+      // Lane 0 requests chunk cb + k: waits for its slot, then issues the K and V boxes.
+      auto issue = [&](int64_t cb, int k) -> bool {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
+          bad |= HPC_DEV_TIMEOUT;
+          return false;
+        }
+        const int32_t page = s_pages[k];
+        const int off = static_cast<int>((off0 + (cb + k) * C) & (P - 1));
+        if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
+        const int bi = stage * groups + gidx;
+        const uint32_t full = full0 + 8 * bi;
+        if (bi < 64) par_lo ^= uint64_t(1) << bi;
+        else par_hi ^= uint64_t(1) << (bi - 64);
+        const uint32_t dst = ring_u32 + stage * p.stage_bytes;
+        // tensor-map coordinates: (d, token, kv head, page) for HND, (d, kv head, token, page) for NHD
+        const int c1 = p.nhd ? x.kvh : off, c2 = p.nhd ? off : x.kvh;
+        mbar_arrive_expect_tx(full, p.stage_bytes);
+#pragma unroll
+        for (int pl = 0; pl < S::kPlanes; ++pl)
+          tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), c1, c2, page, policy);
+#pragma unroll
+        for (int pl = 0; pl < S::kPlanes; ++pl)
+          tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), c1, c2, page,
+                      policy);
+        ++issued;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++gidx == groups) gidx = 0;
+        return true;
+      };
       for (int64_t cb = 0; cb < nchunks && ok; cb += 32) {
         const int nk = static_cast<int>(nchunks - cb < 32 ? nchunks - cb : 32);
         __syncwarp();  // lane 0 has finished with the previous batch of page ids
         if (lane < nk) s_pages[lane] = bt[(off0 + (cb + lane) * C) >> p_shift];
         __syncwarp();
         if (lane == 0) {
-          for (int k = 0; k < nk; ++k) {
-            if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
-              ok = false;
-              bad |= HPC_DEV_TIMEOUT;
-              break;
+          for (int k = 0; k < nk && ok; ++k) {
+            // with the folded prologue, the chunk that holds the new token waits for its write
+            if (PRO && has_new && !pro_done && cb + k == nchunks - 1) {
+              if (!mbar_wait(smem_u32(&s_pro_bar), 0)) {
+                bad |= HPC_DEV_TIMEOUT;
+                ok = false;
+                break;
+              }
+              pro_done = true;
             }
-            const int32_t page = s_pages[k];
-            const int off = static_cast<int>((off0 + (cb + k) * C) & (P - 1));
-            if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
-            const int bi = stage * groups + gidx;
-            const uint32_t full = full0 + 8 * bi;
-            if (bi < 64) par_lo ^= uint64_t(1) << bi;
-            else par_hi ^= uint64_t(1) << (bi - 64);
-            const uint32_t dst = ring_u32 + stage * p.stage_bytes;
-            // tensor-map coordinates: (d, token, kv head, page) for HND, (d, kv head, token, page) for NHD
-            const int c1 = p.nhd ? x.kvh : off, c2 = p.nhd ? off : x.kvh;
-            mbar_arrive_expect_tx(full, p.stage_bytes);
-#pragma unroll
-            for (int pl = 0; pl < S::kPlanes; ++pl)
-              tma_load_4d(dst + pl * p.plane_bytes, &tm_k, full, pl * (128 / S::kElt), c1, c2, page, policy);
-#pragma unroll
-            for (int pl = 0; pl < S::kPlanes; ++pl)
-              tma_load_4d(dst + (S::kPlanes + pl) * p.plane_bytes, &tm_v, full, pl * (128 / S::kElt), c1, c2, page,
-                          policy);
-            ++issued;
-            if (++stage == stages) {
-              stage = 0;
-              phase ^= 1;
-            }
-            if (++gidx == groups) gidx = 0;
+            ok = issue(cb, k);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -691,6 +873,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t wait_par = 0;  // bit s: parity of this group's next wait on slot s
   bool ok = true;
   if constexpr (FUSED) zero_empty_requests<D>(p, ctid, cthreads);
+  int it_par = 0;  // parity of the item count: selects the rotation table
+  if constexpr (PRO) {
+    for (int i = ctid; i < D; i += cthreads) s_qw[i] = p.q_norm_w[i];
+    if (ctid < D / 2) s_invf[ctid] = pow(p.rope_theta, -2.0 * ctid / D);
+    if (ctid == 0)
+      for (int r = blockIdx.x; r < p.batch; r += gridDim.x)
+        if (p.seq_lens[r] == 0) atomicOr(p.status, HPC_DEV_BAD_SEQLEN);  // no token to decode
+    named_barrier_sync(1, cthreads);
+    {
+      // the new token of every segment that ends in this CTA, one warp per segment
+      Cursor c2 = cursor;
+      ItemInfo y;
+      int j = 0;
+      while (c2.next(p, y)) {
+        if (y.tok1 != p.seq_lens[y.req]) continue;
+        if (j++ % kConsumerWarps == warp) write_new_token<D, FP8>(p, y.req, y.kvh, s_invf, lane);
+      }
+      fence_proxy_async_global();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_pro_bar));
+      // the first item's rotation table
+      c2 = cursor;
+      if (c2.next(p, y)) rope_table<D>(static_cast<int64_t>(p.seq_lens[y.req]) - 1, s_invf, s_rope, s_rope + D / 2, ctid);
+    }
+    named_barrier_sync(1, cthreads);
+  }
 
   ItemInfo x;
   while (cursor.next(p, x)) {
@@ -700,7 +908,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Q^T fragments (B operand): lane (g, c) holds query head head0 + g.
     uint32_t qf[KSTEPS][2];
-    {
+    if constexpr (PRO) {
+      const float* tab = s_rope + it_par * D;
+      q_from_qkv<D, FP8>(p, x.req, head0 + g, g < p.group, s_qw, tab, tab + D / 2, c, qf);
+      // the next item's rotation table goes into the other buffer; the item-end barrier
+      // publishes it, and nobody reads that buffer until then
+      Cursor c2 = cursor;
+      ItemInfo y;
+      if (ctid < D / 2 && c2.next(p, y)) {
+        float* nt = s_rope + (it_par ^ 1) * D;
+        rope_table<D>(static_cast<int64_t>(p.seq_lens[y.req]) - 1, s_invf, nt, nt + D / 2, ctid);
+      }
+    } else {
       const bool live = g < p.group;
       const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
           p.q + (static_cast<int64_t>(x.req) * p.num_heads + head0 + (live ? g : 0)) * D);
@@ -735,7 +954,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && tb < tok1) {
           const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
           const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
-          if (nb == 2)
+          if (FP8 && nb == 4)
+            consume_blocks<D, FP8, 4>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
+                                      l0, l1, o, lane);
+          else if (nb == 2)
             consume_blocks<D, FP8, 2>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
                                       l0, l1, o, lane);
           else
@@ -827,6 +1049,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     named_barrier_sync(1, cthreads);  // reduce buffers are reused by the next item
+    it_par ^= 1;
   }
 }
 
@@ -895,14 +1118,18 @@ struct LaunchShape {
   int stages, smem, plane_bytes, stage_bytes;
 };
 
-int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls) {
+// Static shared memory of the kernel: the walk and page-id arrays, plus the folded prologue's
+// norm weights, frequencies and rotation tables.
+inline int static_smem_bytes(int D, bool pro) { return 512 + (pro ? D * 4 + D / 2 * 8 + 2 * D * 4 + 64 : 0); }
+
+int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls, bool pro = false) {
   const int elt = fp8 ? 1 : 2;
   const int planes = D * elt / 128;
   const int plane_bytes = C * 128;
   const int stage_bytes = 2 * planes * plane_bytes;
-  const int bpc = C / 16, nb = bpc >= 2 ? 2 : 1, groups = kConsumerWarps / (bpc / nb);
+  const int bpc = C / 16, nb = blocks_per_warp(bpc, fp8), groups = kConsumerWarps / (bpc / nb);
   const int red = kConsumerWarps * 8 * D * 4 + 2 * kConsumerWarps * 8 * 4;
-  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - 512;  // 512: static shared memory
+  const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - static_smem_bytes(D, pro);
   int stages = kMaxStages;
   // reduce buffers, full[stages][groups] + empty[stages] barriers, 1 KB alignment slack
   auto need = [&](int st) { return st * stage_bytes + red + (st * groups + st) * 8 + 1024; };
@@ -922,10 +1149,10 @@ inline int chunk_tokens(int tile_len, int page_size) {
   return C > 64 ? 64 : C;
 }
 
-template <int D, bool FP8, bool FUSED>
+template <int D, bool FP8, bool FUSED, bool PRO = false>
 int launch(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid, int smem,
            cudaStream_t stream) {
-  auto kern = decode_attention_kernel<D, FP8, FUSED>;
+  auto kern = decode_attention_kernel<D, FP8, FUSED, PRO>;
   static int configured[64] = {0};  // per device: largest dynamic smem already allowed
   int dev = 0;
   cudaGetDevice(&dev);
@@ -978,7 +1205,8 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
             const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads, int32_t kv_heads,
             int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
             int32_t tile_len, int32_t grid, bool persistent, float sm_scale, void* out, hpc_dtype out_dtype,
-            uint32_t* status, CUtensorMap* mk, CUtensorMap* mv, LaunchShape* ls, AttnParams* prm) {
+            uint32_t* status, CUtensorMap* mk, CUtensorMap* mv, LaunchShape* ls, AttnParams* prm,
+            bool pro = false) {
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !status)
     return fail(HPC_ERR_ARG, "null pointer argument");
   if (kv_dtype != HPC_BF16 && kv_dtype != HPC_E4M3) return fail(HPC_ERR_DTYPE, "kv_dtype must be BF16 or E4M3");
@@ -1007,7 +1235,7 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   int ctas_per_sm = (persistent && sms > 0) ? (grid + sms - 1) / sms : 1;
   if (ctas_per_sm < 1) ctas_per_sm = 1;
   if (ctas_per_sm > 4) ctas_per_sm = 4;
-  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, ls);
+  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, ls, pro);
   if (rc) return rc;
   if ((rc = make_pool_map(mk, k_pages, fp8, nhd, head_dim, page_size, kv_heads, num_pages, C))) return rc;
   if ((rc = make_pool_map(mv, v_pages, fp8, nhd, head_dim, page_size, kv_heads, num_pages, C))) return rc;
@@ -1038,12 +1266,12 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   return HPC_OK;
 }
 
-template <bool FUSED>
+template <bool FUSED, bool PRO = false>
 int dispatch(int head_dim, bool fp8, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
              int smem, cudaStream_t st) {
-  if (fp8) return launch<128, true, FUSED>(mk, mv, prm, grid, smem, st);
-  if (head_dim == 128) return launch<128, false, FUSED>(mk, mv, prm, grid, smem, st);
-  return launch<64, false, FUSED>(mk, mv, prm, grid, smem, st);
+  if (fp8) return launch<128, true, FUSED, PRO>(mk, mv, prm, grid, smem, st);
+  if (head_dim == 128) return launch<128, false, FUSED, PRO>(mk, mv, prm, grid, smem, st);
+  return launch<64, false, FUSED, PRO>(mk, mv, prm, grid, smem, st);
 }
 
 struct StepLayout {
@@ -1095,12 +1323,24 @@ extern "C" size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_hea
   return step_layout(batch, num_heads / kv_heads, kv_heads, head_dim, num_ctas).total;
 }
 
-extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
-                               hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
-                               int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
-                               int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
-                               int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
-                               hpc_dtype out_dtype, uint32_t* status, void* stream) {
+namespace hpc {
+namespace {
+
+struct PrologueArgs {
+  const void* qkv;
+  const float* q_norm_w;
+  const float* k_norm_w;
+  float eps, rope_theta;
+};
+
+// Single-launch step; with `pro`, q is formed from qkv in the kernel and the new token's K/V
+// are written into the cache first.
+int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype, hpc_kv_layout kv_layout,
+              const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads,
+              int32_t kv_heads, int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
+              const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas, float sm_scale,
+              void* workspace, size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
+              void* stream, const PrologueArgs* pro) {
   if (!workspace) return fail(HPC_ERR_ARG, "null pointer argument");
   if (batch < 1) return fail(HPC_ERR_ARG, "batch must be >= 1");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return fail(HPC_ERR_ALIGN, "workspace must be 256-byte aligned");
@@ -1112,7 +1352,7 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
   int rc = prepare(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads,
                    head_dim, block_table, max_pages_per_req, seq_lens, tile_len, num_ctas, true, sm_scale, out,
-                   out_dtype, status, &mk, &mv, &ls, &prm);
+                   out_dtype, status, &mk, &mv, &ls, &prm, pro != nullptr);
   if (rc) return rc;
   // the per-request tile prefix lives in the reduce buffer while the CTA plans
   const size_t red_bytes = static_cast<size_t>(kConsumerWarps) * 8 * head_dim * sizeof(float);
@@ -1126,6 +1366,46 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
   prm.partial_o = reinterpret_cast<float*>(ws + L.partial_o);
   prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
   prm.batch = batch;
-  return dispatch<true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
-                        static_cast<cudaStream_t>(stream));
+  if (!pro)
+    return dispatch<true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
+                          static_cast<cudaStream_t>(stream));
+  prm.qkv = static_cast<const __nv_bfloat16*>(pro->qkv);
+  prm.q_norm_w = pro->q_norm_w;
+  prm.k_norm_w = pro->k_norm_w;
+  prm.eps = pro->eps;
+  prm.rope_theta = static_cast<double>(pro->rope_theta);
+  prm.k_pages_w = const_cast<void*>(k_pages);
+  prm.v_pages_w = const_cast<void*>(v_pages);
+  return dispatch<true, true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
+                              static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace hpc
+
+extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                               hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                               int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                               int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
+                               int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
+                               hpc_dtype out_dtype, uint32_t* status, void* stream) {
+  return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
+                   workspace, workspace_bytes, out, out_dtype, status, stream, nullptr);
+}
+
+extern "C" int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,
+                                        float rope_theta, void* k_pages, void* v_pages, hpc_dtype kv_dtype,
+                                        hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale,
+                                        int32_t num_pages, int32_t page_size, int32_t num_heads, int32_t kv_heads,
+                                        int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
+                                        const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
+                                        float sm_scale, void* workspace, size_t workspace_bytes, void* out,
+                                        hpc_dtype out_dtype, uint32_t* status, void* stream) {
+  if (!qkv || !q_norm_w || !k_norm_w) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (!(rope_theta > 0.f) || !(eps >= 0.f)) return fail(HPC_ERR_ARG, "rope_theta must be > 0 and eps >= 0");
+  const PrologueArgs pro{qkv, q_norm_w, k_norm_w, eps, rope_theta};
+  return step_impl(qkv, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
+                   workspace, workspace_bytes, out, out_dtype, status, stream, &pro);
 }

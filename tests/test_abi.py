@@ -31,7 +31,7 @@ def declared_symbols():
 def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ("hpc_decode_plan", "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue",
-              "hpc_plan_cpu", "hpc_decode_plan_static"):
+              "hpc_plan_cpu", "hpc_decode_plan_static", "hpc_decode_step", "hpc_decode_step_prologue"):
         assert n in names
 
 
@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 2
+    assert B._lib.hpc_abi_version() == 3
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -58,6 +58,15 @@ def test_host_argument_errors_return_codes(B):
     assert "null" in B._lib.hpc_last_error().decode()
     rc = B._lib.hpc_merge_states(None, None, ctypes.byref(P), 8, 64, None, 1, None, None)
     assert rc == B.HPC_ERR_ARG
+    # the single-launch step with the folded prologue: null qkv / norm weights, bad theta
+    i32 = ctypes.c_int32
+    rc = B._lib.hpc_decode_step_prologue(None, None, None, 1e-6, 1e6, None, None, 0, 0, None, None, 1, 16, 8, 2, 64,
+                                         None, 1, None, 1, 32, 4, 0.1, None, 0, None, 1, None, None)
+    assert rc == B.HPC_ERR_ARG
+    w = ctypes.c_void_p(16)  # never dereferenced: the argument checks fail first
+    rc = B._lib.hpc_decode_step_prologue(w, w, w, 1e-6, -1.0, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1,
+                                         32, 4, 0.1, w, 0, w, 1, w, None)
+    assert rc == B.HPC_ERR_ARG and "rope_theta" in B._lib.hpc_last_error().decode()
     # bad tile_len on the host planner
     lens = torch.tensor([5, 7], dtype=torch.int32)
     with pytest.raises(B.HpcError, match="tile_len"):

@@ -52,6 +52,24 @@ def test_shapes_ragged(B, Hq, Hkv, D, P, tl):
         assert_bf16_tol(out, ref, what=f"{(Hq, Hkv, D, P, tl, G)}")
 
 
+@pytest.mark.parametrize("Hq,Hkv,P,tl", [
+    (8, 8, 16, 16), (16, 2, 16, 48), (16, 4, 32, 32), (32, 8, 32, 64), (8, 2, 64, 64), (64, 8, 64, 128),
+    (32, 8, 128, 128), (16, 4, 128, 256),
+])
+def test_e4m3_shapes_ragged(B, Hq, Hkv, P, tl):
+    """E4M3 cache over every stage size (16, 32 and 64 tokens: one, two and four 16-token
+    blocks per consumer warp) and every GQA group size."""
+    lens = (1, 15, 16, 17, 63, 64, 65, 129, 300, 1000, 2049)
+    spec, case = _case(lens, Hq, Hkv, 128, P, tl, seed=Hq + P + tl, kv="e4m3")
+    dc = to_device(case)
+    ref = oracle_out(case)
+    for G in (5, 148):
+        out, _, st = run_attention(B, spec, dc, num_ctas=G)
+        assert st == 0
+        mx, _ = errors(out, ref)
+        assert mx <= 5e-2, (Hq, Hkv, P, tl, G, mx)
+
+
 def test_bf16_output_within_one_ulp(B):
     spec, case = _case((17, 200, 513, 1024), 16, 2, 128, 64, 128, seed=3)
     dc = to_device(case)
