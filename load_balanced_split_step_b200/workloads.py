@@ -59,6 +59,7 @@ class DecodeSpec:
     kv_dtype: str = "bf16"  # "bf16" or "e4m3"
     steps: int = 1  # decode steps; step i uses seq_lens + i
     prologue: bool = False
+    q_len: int = 1  # new tokens per request (the last q_len of the L_r cached tokens)
     rope_theta: float = 1e6
     rms_eps: float = 1e-6
     seed: int = 0
@@ -109,10 +110,10 @@ def config_spec(name: str, seed: int = 0) -> DecodeSpec:
 
 
 def custom_spec(seq_lens, num_heads=8, kv_heads=2, head_dim=64, page_size=16, tile_len=32,
-                kv_dtype="bf16", steps=1, prologue=False, seed=0, name="custom") -> DecodeSpec:
+                kv_dtype="bf16", steps=1, prologue=False, seed=0, name="custom", q_len=1) -> DecodeSpec:
     return DecodeSpec(name, tuple(int(x) for x in seq_lens), num_heads, kv_heads, head_dim,
                       page_size, tile_len, kv_dtype=kv_dtype, steps=steps, prologue=prologue,
-                      seed=seed)
+                      seed=seed, q_len=q_len)
 
 
 @dataclass
@@ -244,7 +245,10 @@ def make_case(spec: DecodeSpec, requests=None) -> DecodeCase:
 
     q = qkv = None
     rq = np.random.Generator(np.random.PCG64(ch[2]))
-    qa = rq.standard_normal((B, Hq, D), dtype=np.float32)[sel]
+    if spec.q_len == 1:
+        qa = rq.standard_normal((B, Hq, D), dtype=np.float32)[sel]
+    else:  # [B, q_len, Hq, D]
+        qa = rq.standard_normal((B, spec.q_len, Hq, D), dtype=np.float32)[sel]
     rqkv = np.random.Generator(np.random.PCG64(ch[3]))
     qkva = rqkv.standard_normal((B, Hq + 2 * Hkv, D), dtype=np.float32)[sel]
     if spec.prologue:
@@ -294,8 +298,8 @@ def algorithmic_bytes(spec: DecodeSpec, step: int = 0, out_bytes: int = 4) -> in
     kv_elem = 1 if spec.kv_dtype == "e4m3" else 2
     tokens = spec.kv_tokens(step)
     b = tokens * spec.kv_heads * spec.head_dim * 2 * kv_elem
-    b += spec.batch * spec.num_heads * spec.head_dim * 2  # q (bf16)
-    b += spec.batch * spec.num_heads * spec.head_dim * out_bytes
+    b += spec.batch * spec.q_len * spec.num_heads * spec.head_dim * 2  # q (bf16)
+    b += spec.batch * spec.q_len * spec.num_heads * spec.head_dim * out_bytes
     if spec.prologue:
         b += spec.batch * (spec.num_heads + 2 * spec.kv_heads) * spec.head_dim * 2
         b += spec.batch * spec.num_heads * spec.head_dim * 2  # q' written (bf16)

@@ -111,3 +111,55 @@ def _torch_gather(pages: torch.Tensor, bt: np.ndarray, r: int, g: int, L: int) -
     j = torch.arange(L)
     phys = torch.from_numpy(bt[r])[j // P]
     return pages[phys, g, j % P, :]
+
+
+def decode_attention_multi(q, k_pages, v_pages, block_table, seq_lens, sm_scale=None,
+                           kv_dtype="bf16", k_scale=None, v_scale=None, requests=None):
+    """Several new tokens per request, attending causally (speculative verification, or a
+    chunked extend of the decode batch).
+
+    q: [B, T, Hq, D]. The T query tokens of request r are the last T of its L_r cached
+    tokens: query token t sits at position L_r - T + t and attends to positions
+    0 .. L_r - T + t, itself included. Returns float64 [B, T, Hq, D]:
+
+        out[r, t, h, :] = sum_{j <= L_r - T + t} softmax_j(sm_scale * q[r,t,h] . k_j) v_j
+
+    Readings where the pages are silent (they report the backend's effect on time to first
+    token, not its prefill kernel): all requests of a step share T; L_r = 0 gives zeros, and a
+    request with 0 < L_r < T has no valid query position and also gives zeros. The rest
+    follows decode_attention (GQA map, page layout, E4M3 decoding, scale).
+    """
+    qf = to_f64(q)
+    B, T, Hq, D = qf.shape
+    if kv_dtype == "e4m3":
+        kp = np.asarray(k_pages.cpu().numpy() if isinstance(k_pages, torch.Tensor) else k_pages, dtype=np.uint8)
+        vp = np.asarray(v_pages.cpu().numpy() if isinstance(v_pages, torch.Tensor) else v_pages, dtype=np.uint8)
+        ks, vs = to_f64(k_scale), to_f64(v_scale)
+    else:
+        kp, vp = k_pages, v_pages
+        ks = vs = None
+    Hkv = kp.shape[1]
+    grp = Hq // Hkv
+    bt = np.asarray(block_table.cpu().numpy() if isinstance(block_table, torch.Tensor) else block_table, dtype=np.int64)
+    lens = np.asarray(seq_lens.cpu().numpy() if isinstance(seq_lens, torch.Tensor) else seq_lens, dtype=np.int64)
+    scale = (1.0 / math.sqrt(D)) if sm_scale is None else float(sm_scale)
+    out = np.zeros((B, T, Hq, D), dtype=np.float64)
+    for r in (range(B) if requests is None else requests):
+        L = int(lens[r])
+        if L < T:
+            continue
+        for g in range(Hkv):
+            if kv_dtype == "e4m3":
+                K = _kv_values(kp, kv_dtype, ks, bt, r, g, L)
+                V = _kv_values(vp, kv_dtype, vs, bt, r, g, L)
+            else:
+                K = to_f64(_torch_gather(kp, bt, r, g, L))
+                V = to_f64(_torch_gather(vp, bt, r, g, L))
+            for t in range(T):
+                n = L - T + t + 1  # tokens that query t may see
+                for h in range(g * grp, (g + 1) * grp):
+                    s = scale * (K[:n] @ qf[r, t, h])
+                    p = np.exp(s - s.max())
+                    p = p / p.sum()
+                    out[r, t, h] = p @ V[:n]
+    return out
