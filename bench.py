@@ -59,6 +59,8 @@ def parse_args(argv=None):
                     help="fused: one launch per step (in-kernel plan + ticket merge), after the prologue kernel on "
                          "the FP8 workload; folded: the same with the prologue folded into that launch; split: "
                          "plan, attention and merge kernels")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="new tokens per request, attending causally (1 to 4; single-launch path)")
     ap.add_argument("--no-extras", action="store_true", help="skip static split-k, e2e and CPU baseline legs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     return ap.parse_args(argv)
@@ -184,8 +186,11 @@ class Step:
         self.num_ctas = num_ctas
         self.po, self.pml = B.partial_buffers(self.plan, spec.num_heads, spec.head_dim, dev)
         if self.fused:
-            self.ws = B.step_workspace(spec.batch, spec.num_heads, spec.kv_heads, spec.head_dim, num_ctas, dev)
-        self.out = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.float32, device=dev)
+            self.ws = B.multi_workspace(spec.batch, spec.q_len, spec.num_heads, spec.kv_heads, spec.head_dim,
+                                        num_ctas, dev)
+        qshape = (spec.batch, spec.num_heads, spec.head_dim) if spec.q_len == 1 else \
+            (spec.batch, spec.q_len, spec.num_heads, spec.head_dim)
+        self.out = torch.empty(qshape, dtype=torch.float32, device=dev)
         self.q = dc["q"]
         if spec.prologue:
             self.q = torch.empty((spec.batch, spec.num_heads, spec.head_dim), dtype=torch.bfloat16, device=dev)
@@ -209,6 +214,16 @@ class Step:
                        seq, s.num_heads, s.kv_heads, kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                        v_scale=dc["v_scale"], eps=s.rms_eps, rope_theta=s.rope_theta, q_out=self.q,
                        status=self.status)
+        if self.fused and s.q_len > 1:
+            if ev is not None:
+                ev[0].record()
+            B.decode_step_multi(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, s.kv_heads, self.tl,
+                                kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
+                                v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
+                                workspace=self.ws)
+            if ev is not None:
+                ev[1].record()
+            return self.out
         if self.fused:
             if ev is not None:
                 ev[0].record()
@@ -291,13 +306,15 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
     src = {"seq_lens": case.seq_lens.pin_memory(), "block_table": case.block_table.pin_memory()}
     qname = "qkv" if spec.prologue else "q"
     src[qname] = getattr(case, qname).pin_memory()
-    shape = (spec.batch, spec.num_heads, spec.head_dim)
+    shape = (spec.batch, spec.num_heads, spec.head_dim) if spec.q_len == 1 else \
+        (spec.batch, spec.q_len, spec.num_heads, spec.head_dim)
     nbuf = 2
     dsts = [{k: torch.empty_like(v, device=dev) for k, v in src.items()} for _ in range(nbuf)]
     outs = [torch.empty(shape, dtype=torch.float32, device=dev) for _ in range(nbuf)]
     hosts = [torch.empty(shape, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
     qbufs = [torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
-    ws = B.step_workspace(spec.batch, spec.num_heads, spec.kv_heads, spec.head_dim, num_ctas, dev) if fused else None
+    ws = B.multi_workspace(spec.batch, spec.q_len, spec.num_heads, spec.kv_heads, spec.head_dim, num_ctas, dev) \
+        if fused else None
     h2d = sum(v.numel() * v.element_size() for v in src.values())
     d2h = hosts[0].numel() * hosts[0].element_size()
     s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -331,6 +348,10 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
                                rope_theta=spec.rope_theta, q_out=qbufs[b])
             if folded and spec.prologue:
                 pass  # done above, in one launch
+            elif fused and spec.q_len > 1:
+                B.decode_step_multi(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.kv_heads, tl,
+                                    kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
+                                    v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws)
             elif fused:
                 B.decode_step_fused(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
                                     spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
@@ -389,17 +410,36 @@ def cpu_baseline(spec, case, target_s):
                                    sub.k_scale, sub.v_scale, spec.num_heads, spec.kv_heads)[0]
             OA.decode_attention(q, kp, vp, sub.block_table, sub.seq_lens, kv_dtype=spec.kv_dtype,
                                 k_scale=sub.k_scale, v_scale=sub.v_scale)
+        elif spec.q_len > 1:
+            OA.decode_attention_multi(case.q[r:r + 1], case.k_pages, case.v_pages, case.block_table[r:r + 1],
+                                      case.seq_lens[r:r + 1], kv_dtype=spec.kv_dtype, k_scale=case.k_scale,
+                                      v_scale=case.v_scale)
         else:
             OA.decode_attention(case.q[r:r + 1], case.k_pages, case.v_pages, case.block_table[r:r + 1],
                                 case.seq_lens[r:r + 1], kv_dtype=spec.kv_dtype, k_scale=case.k_scale,
                                 v_scale=case.v_scale)
-        done_bytes += per_req_kv[r] + spec.num_heads * spec.head_dim * 6
+        done_bytes += per_req_kv[r] + spec.q_len * spec.num_heads * spec.head_dim * 6
         n_req += 1
     el = time.perf_counter() - t0
     frac = done_bytes / bytes_step
     desc = (f"{n_req} whole requests of the workload taken round-robin "
             f"({frac:.2f} of one step's algorithmic bytes) in {el:.1f} s")
     return done_bytes / el / 1e9, desc, threads, el
+
+
+def qlen_text(args):
+    return "" if args.q_len == 1 else f"; {args.q_len} new tokens per request, causal among themselves"
+
+
+def workload_spec(args):
+    """The named workload, with q_len new tokens per request when --q-len > 1."""
+    from dataclasses import replace
+    spec = W.config_spec(args.workload)
+    if args.q_len != 1:
+        if spec.prologue:
+            raise SystemExit("--q-len > 1 is not combined with the prologue workload")
+        spec = replace(spec, q_len=args.q_len, name=f"{spec.name}, {args.q_len} new tokens per request")
+    return spec
 
 
 def load_peaks():
@@ -444,7 +484,7 @@ def run_ours(args, rank, world, local):
     from load_balanced_split_step_b200 import binding as B
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    spec = W.config_spec(args.workload)
+    spec = workload_spec(args)
     case = W.make_case(spec)
     dc = {k: (getattr(case, k).to(dev) if getattr(case, k) is not None else None)
           for k in ("q", "qkv", "k_pages", "v_pages", "block_table", "seq_lens", "k_scale", "v_scale", "q_norm_w",
@@ -501,8 +541,10 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         extra["graph_us_per_step"] = round(1000.0 * a.elapsed_time(b) / K, 2)
         del g
-        extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms, args.layout)
-        extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step), 3)
+        if spec.q_len == 1:  # the static plan drives the three-launch path, which takes one new token
+            extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms, args.layout)
+            extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step),
+                                                       3)
     e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path != "split",
                                layout=args.layout, folded=args.path == "folded")
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -519,7 +561,7 @@ def run_ours(args, rank, world, local):
         "ms_per_step": round(ms_step, 5), "us_per_step": round(1000 * ms_step, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if spec.kv_dtype == "bf16" else "e4m3/f16",
         "data": "synthetic (seeded N(0,1), bf16-rounded; random page permutation)",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "tile_len": tl, "num_ctas": G,
+        "config": {"workload": WORKLOAD_TEXT[args.workload] + qlen_text(args), "tile_len": tl, "num_ctas": G,
                    "plan": "dynamic (re-planned on the device every step)",
                    "path": ({"fused": "single launch: in-kernel plan, attention, ticket merge"
                                       + (" (after the prologue kernel, PDL)" if spec.prologue else ""),
@@ -550,7 +592,7 @@ def run_reference(args, rank, world):
     """The reference arm: the fp64 CPU oracle as it stands, timed on the host cores."""
     if rank != 0:
         return None
-    spec = W.config_spec(args.workload)
+    spec = workload_spec(args)
     case = W.make_case(spec)
     K, W_ = max(1, min(args.steps, 3)), 0
     target = args.cpu_seconds
@@ -565,7 +607,8 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": W_, "ms_per_step": round(1000 * bytes_step / (v * 1e9), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "tile_len": spec.tile_len, "plan": "none (exact)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload] + qlen_text(args), "tile_len": spec.tile_len,
+                   "plan": "none (exact)",
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": descs[0]},

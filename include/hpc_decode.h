@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 3
+#define HPC_DECODE_ABI_VERSION 4
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -250,6 +250,38 @@ HPC_API int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, con
                                      const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
                                      float sm_scale, void* workspace, size_t workspace_bytes, void* out,
                                      hpc_dtype out_dtype, uint32_t* status, void* stream);
+
+/* ---- several new tokens per request ----------------------------------------------------- */
+
+/* Bytes of workspace hpc_decode_step_multi needs: as hpc_decode_step_workspace_bytes, with
+ * q_len * num_heads / kv_heads rows in each partial state. 0 for a bad shape. */
+HPC_API size_t hpc_decode_step_multi_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_heads,
+                                                     int32_t kv_heads, int32_t head_dim, int32_t num_ctas);
+
+/* hpc_decode_step for q_len new tokens per request, attending causally: speculative-decode
+ * verification, or a chunked extend. The pages report the attention backend's effect on time
+ * to first token ("vLLM × HPC-Ops" summary; remio.ai, "Por qué Tencent HPC importa …") but
+ * do not describe a multi-token kernel; this entry point is the plainest extension of the
+ * split-KV decode step to it. The planner is unchanged: KV tiles of a request do not depend
+ * on how many queries read them.
+ *  - q:   device bf16 [batch][q_len][num_heads][head_dim]. The q_len query tokens of request r
+ *         are the last q_len of its seq_lens[r] cached tokens: query token t sits at position
+ *         seq_lens[r] - q_len + t and attends to positions 0 .. seq_lens[r] - q_len + t.
+ *  - out: device [batch][q_len][num_heads][head_dim], HPC_FP32 or HPC_BF16.
+ *  - q_len: 1 to 4. Each consumer warp computes one query token's rows over its blocks of a
+ *         stage; q_len 3 leaves one warp slot of four idle.
+ *  - seq_lens[r] = 0 gives a zero output; 0 < seq_lens[r] < q_len sets HPC_DEV_BAD_SEQLEN and
+ *         also gives zeros.
+ *  - workspace: >= hpc_decode_step_multi_workspace_bytes(), zeroed once, as for
+ *         hpc_decode_step. Everything else as hpc_decode_step. q_len = 1 is hpc_decode_step. */
+HPC_API int hpc_decode_step_multi(const void* q, int32_t q_len, const void* k_pages, const void* v_pages,
+                                  hpc_dtype kv_dtype, hpc_kv_layout kv_layout, const float* k_scale,
+                                  const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads,
+                                  int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                                  int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch,
+                                  int32_t tile_len, int32_t num_ctas, float sm_scale, void* workspace,
+                                  size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
+                                  void* stream);
 
 /* ---- merge --------------------------------------------------------------------------- */
 

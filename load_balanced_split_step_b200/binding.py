@@ -29,7 +29,8 @@ EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_d
            "hpc_decode_plan_static", "hpc_plan_cpu", "hpc_partial_o_bytes", "hpc_partial_ml_bytes",
            "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue", "hpc_attention_launch_info",
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
-           "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue")
+           "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue",
+           "hpc_decode_step_multi", "hpc_decode_step_multi_workspace_bytes")
 
 
 class HpcError(RuntimeError):
@@ -79,6 +80,10 @@ def _load():
         "hpc_decode_step_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp,
                                                     i32, i32, i32, i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz,
                                                     vp, ctypes.c_int, vp, vp]),
+        "hpc_decode_step_multi_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+        "hpc_decode_step_multi": (ctypes.c_int, [vp, i32, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32,
+                                                 i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp,
+                                                 vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -393,6 +398,43 @@ def decode_step_prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table,
         _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace), workspace.numel(), _ptr(out),
         HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status), _stream(dev)),
         "hpc_decode_step_prologue")
+    return out, status, workspace
+
+
+def multi_workspace(batch, q_len, num_heads, kv_heads, head_dim, num_ctas, device):
+    """Zeroed workspace for ``decode_step_multi``."""
+    n = _lib.hpc_decode_step_multi_workspace_bytes(batch, q_len, num_heads, kv_heads, head_dim, num_ctas)
+    if n == 0:
+        raise HpcError("bad shape for hpc_decode_step_multi_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile_len, *, kv_dtype="bf16",
+                      kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None,
+                      out_dtype=torch.float32, status=None, workspace=None):
+    """q_len new tokens per request in one launch (``hpc_decode_step_multi``): q is
+    [B, q_len, Hq, D]; query token t of request r sits at position L_r - q_len + t and
+    attends causally. Returns (out [B, q_len, Hq, D], status, workspace)."""
+    _need(q, "q", torch.bfloat16)
+    dev = q.device
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    code = _kv_code(kv_dtype, k_pages)
+    B, T, Hq, D = q.shape
+    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
+    if num_ctas is None:
+        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    if out is None:
+        out = torch.empty((B, T, Hq, D), dtype=out_dtype, device=dev)
+    status = new_status(dev) if status is None else status
+    if workspace is None:
+        workspace = multi_workspace(B, T, Hq, Hkv, D, num_ctas, dev)
+    scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    _check(_lib.hpc_decode_step_multi(
+        _ptr(q), T, _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
+        workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
+        _stream(dev)), "hpc_decode_step_multi")
     return out, status, workspace
 
 

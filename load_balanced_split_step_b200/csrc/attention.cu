@@ -65,6 +65,7 @@ struct AttnParams {
   int32_t stages, out_bf16;
   uint32_t plane_bytes, stage_bytes;
   float score_scale;  // sm_scale * log2(e)
+  int32_t q_len;      // new tokens per request (single-launch step); 1 elsewhere
   int32_t nhd;        // cache layout: token stride Hkv*D (NHD) or D (HND); only the TMA coordinates differ
   // single-launch step only: the plan is derived in the kernel from seq_lens
   int32_t batch, kv_heads, max_seq_len;
@@ -94,17 +95,24 @@ struct ItemInfo {
 // two independent MMA chains. An E4M3 stage carries half the bytes per token, so the fixed
 // per-call softmax work (row max across lanes, rescale factors) and the stage handshake weigh
 // twice as much per byte: there a warp takes up to four blocks, a whole 64-token stage.
-__host__ __device__ __forceinline__ int blocks_per_warp(int bpc, bool fp8) {
-  if (fp8 && bpc >= 4) return 4;
+__host__ __device__ __forceinline__ int blocks_per_warp(int bpc, bool fp8, int q_pad = 1) {
+  if (fp8 && bpc >= 4 && q_pad == 1) return 4;
   return bpc >= 2 ? 2 : 1;
 }
+
+// Several new tokens per request: q_len query tokens take q_pad = 1, 2 or 4 warp slots of each
+// stage (q_len 3 leaves one slot idle). Each warp computes one query token's rows over its
+// blocks, so a stage is read by (blocks per stage / blocks per warp) * q_pad warps.
+__host__ __device__ __forceinline__ int q_pad_of(int q_len) { return q_len <= 1 ? 1 : (q_len <= 2 ? 2 : 4); }
 
 __device__ __forceinline__ int32_t tiles_of(int32_t L, int32_t tl) {
   return L > 0 ? static_cast<int32_t>(static_cast<uint32_t>(L - 1) / static_cast<uint32_t>(tl) + 1) : 0;
 }
 
-__device__ __forceinline__ bool len_ok(int32_t L, int32_t max_seq_len) {
-  return L >= 0 && (max_seq_len <= 0 || L <= max_seq_len);
+// A length is valid when it is 0 (no tiles, zero output) or holds the step's q_len new tokens
+// and fits the block table.
+__device__ __forceinline__ bool len_ok(int32_t L, int32_t max_seq_len, int32_t q_len = 1) {
+  return L >= 0 && (L == 0 || L >= q_len) && (max_seq_len <= 0 || L <= max_seq_len);
 }
 
 template <int D, bool FP8>
@@ -182,7 +190,7 @@ struct WalkCursor {
         do {
           ++r;
           const int32_t Ln = p.seq_lens[r];
-          nt = len_ok(Ln, p.max_seq_len) ? tiles_of(Ln, p.tile_len) : 0;
+          nt = len_ok(Ln, p.max_seq_len, p.q_len) ? tiles_of(Ln, p.tile_len) : 0;
         } while (nt == 0);
       }
     }
@@ -401,7 +409,7 @@ __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_s
   uint32_t bad = 0;
   for (int r = r0; r < r1; ++r) {
     const int32_t L = p.seq_lens[r];
-    const bool ok = len_ok(L, p.max_seq_len);
+    const bool ok = len_ok(L, p.max_seq_len, p.q_len);
     if (!ok) bad |= HPC_DEV_BAD_SEQLEN;
     run += ok ? tiles_of(L, p.tile_len) : 0;
   }
@@ -429,7 +437,7 @@ __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_s
   for (int r = r0; r < r1; ++r) {
     s_pre[r] = pre;
     const int32_t L = p.seq_lens[r];
-    pre += len_ok(L, p.max_seq_len) ? tiles_of(L, p.tile_len) : 0;
+    pre += len_ok(L, p.max_seq_len, p.q_len) ? tiles_of(L, p.tile_len) : 0;
   }
   if (tid == 0) s_pre[B] = s_scan[nwarps];
   __syncthreads();
@@ -480,9 +488,10 @@ template <int D>
 __device__ void zero_empty_requests(const AttnParams& p, int tid, int nthr) {
   for (int r = blockIdx.x; r < p.batch; r += gridDim.x) {
     const int32_t L = p.seq_lens[r];
-    if (len_ok(L, p.max_seq_len) && L > 0) continue;
-    const int64_t base = static_cast<int64_t>(r) * p.num_heads * D;
-    for (int i = tid; i < p.num_heads * D; i += nthr) {
+    if (len_ok(L, p.max_seq_len, p.q_len) && L > 0) continue;
+    const int64_t rows = static_cast<int64_t>(p.q_len) * p.num_heads * D;
+    const int64_t base = static_cast<int64_t>(r) * rows;
+    for (int64_t i = tid; i < rows; i += nthr) {
       if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[base + i] = __float2bfloat16_rn(0.f);
       else reinterpret_cast<float*>(p.out)[base + i] = 0.f;
     }
@@ -500,15 +509,19 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
                               float* s_buf, int buf_floats) {
   const int64_t g1 = x.U / chunk, g2 = (x.U + x.nt - 1) / chunk;
   const int64_t first_slot = (x.U > g1 * chunk) ? 2 * g1 + 1 : 2 * g1;
-  const int grp = p.group;
+  // rows of a piece: query token t, head h -> row t * group + h
+  const int grp = p.group * p.q_len;
   const int n = static_cast<int>(g2 - g1 + 1);
   auto slot_of = [&](int i) -> int64_t { return i == 0 ? first_slot : 2 * (g1 + i); };
-  const int64_t orow = (static_cast<int64_t>(x.req) * p.num_heads + x.kvh * grp) * D;
+  auto out_at = [&](int idx) -> int64_t {  // idx = row * D + d
+    const int row = idx / D, t = row / p.group, h = row - t * p.group;
+    return ((static_cast<int64_t>(x.req) * p.q_len + t) * p.num_heads + x.kvh * p.group + h) * D + (idx - row * D);
+  };
   float* s_m = s_buf;
   float* s_w = s_buf + n * grp;
   float* s_M = s_w + n * grp;
-  float* s_iL = s_M + 8;
-  if (2 * n * grp + 16 <= buf_floats) {
+  float* s_iL = s_M + grp;
+  if (2 * n * grp + 2 * grp <= buf_floats) {
     for (int k = tid; k < n * grp; k += nthr) {
       const int i = k / grp, h = k - i * grp;
       const float* ml = p.partial_ml + 2 * (slot_of(i) * grp + h);
@@ -542,8 +555,8 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
       }
       for (; i < n; ++i) a0 += s_w[i * grp + h] * __ldcg(p.partial_o + slot_of(i) * grp * D + idx);
       const float val = (a0 + a1) + (a2 + a3);
-      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow + idx] = __float2bfloat16_rn(val);
-      else reinterpret_cast<float*>(p.out)[orow + idx] = val;
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[out_at(idx)] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(p.out)[out_at(idx)] = val;
     }
     return;
   }
@@ -560,8 +573,8 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
       acc += e * __ldcg(p.partial_o + pi * D + (idx - h * D));
     }
     const float val = Ls > 0.f ? acc / Ls : 0.f;
-    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[orow + idx] = __float2bfloat16_rn(val);
-    else reinterpret_cast<float*>(p.out)[orow + idx] = val;
+    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[out_at(idx)] = __float2bfloat16_rn(val);
+    else reinterpret_cast<float*>(p.out)[out_at(idx)] = val;
   }
 }
 
@@ -707,11 +720,15 @@ __device__ __forceinline__ void q_from_qkv(const AttnParams& p, int req, int hea
   }
 }
 
-template <int D, bool FP8, bool FUSED, bool PRO>
+template <int D, bool FP8, bool FUSED, bool PRO, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                             const AttnParams p) {
   static_assert(FUSED || !PRO, "the prologue is folded into the single-launch step only");
+  static_assert(FUSED || !MULTI, "several new tokens per request run in the single-launch step only");
+  static_assert(!(PRO && MULTI), "the folded prologue takes one new token per request");
+  // query tokens per request: a compile-time 1 unless this is the several-new-tokens kernel
+  const int q_len = MULTI ? p.q_len : 1;
   using S = Shape<D, FP8>;
   using Cursor = typename CursorOf<FUSED>::type;
   extern __shared__ uint8_t smem_raw[];
@@ -735,8 +752,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barriers in order, and a parity wait can never match a phase two behind.
   uint64_t* bars = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * 8);
   const int bpc = p.chunk_tokens / 16;          // 16-token blocks per stage
-  const int nb = blocks_per_warp(bpc, FP8);     // 16-token blocks per warp per stage
-  const int wps = bpc / nb;                     // warps per stage
+  const int q_pad = MULTI ? q_pad_of(q_len) : 1;  // warp slots per block range: one per query token
+  const int nb = blocks_per_warp(bpc, FP8, q_pad);  // 16-token blocks per warp per stage
+  const int wtok = bpc / nb;                    // warps that split a stage's blocks
+  const int wps = wtok * q_pad;                 // warps per stage
   const int groups = kConsumerWarps / wps;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -866,7 +885,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 16-token blocks. Only those warps wait on it and release it (empty-barrier count = wps).
   const int g = lane >> 2, c = lane & 3;  // MMA fragment row / column pair
   constexpr int KSTEPS = D / 16;
-  const int my_group = warp / wps, my_first = (warp % wps) * nb;
+  // warp = (group, query token, block range): group * wps + my_t * wtok + block range
+  const int my_group = warp / wps, my_t = MULTI ? (warp % wps) / wtok : 0, my_first = (warp % wtok) * nb;
+  const bool t_live = !MULTI || my_t < q_len;
   const uint32_t my_full0 = full0 + 8 * my_group;  // + 8 * groups * slot
   const int ctid = threadIdx.x, cthreads = kConsumerWarps * 32;
   int stage = 0, gidx = 0;
@@ -905,6 +926,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kvh = x.kvh;
     const int head0 = kvh * p.group;
     const int64_t tok0 = x.tok0, tok1 = x.tok1;
+    // causal limit of this warp's query token: it sits at position L - q_len + my_t
+    int64_t lim = tok1;
+    if (MULTI) {
+      const int64_t last = static_cast<int64_t>(p.seq_lens[x.req]) - q_len + my_t + 1;
+      lim = last < tok1 ? last : tok1;
+    }
 
     // Q^T fragments (B operand): lane (g, c) holds query head head0 + g.
     uint32_t qf[KSTEPS][2];
@@ -920,9 +947,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         rope_table<D>(static_cast<int64_t>(p.seq_lens[y.req]) - 1, s_invf, nt, nt + D / 2, ctid);
       }
     } else {
-      const bool live = g < p.group;
+      const bool live = g < p.group && t_live;
       const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          p.q + (static_cast<int64_t>(x.req) * p.num_heads + head0 + (live ? g : 0)) * D);
+          p.q + ((static_cast<int64_t>(x.req) * q_len + (t_live ? my_t : 0)) * p.num_heads + head0 +
+                 (live ? g : 0)) * D);
 #pragma unroll
       for (int ks = 0; ks < KSTEPS; ++ks) {
         if (!FP8) {
@@ -951,17 +979,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         wait_par ^= 1u << stage;
         const int64_t tb = t + 16 * my_first;
-        if (ok && tb < tok1) {
+        if (ok && t_live && tb < lim) {
           const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
           const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
           if (FP8 && nb == 4)
-            consume_blocks<D, FP8, 4>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
+            consume_blocks<D, FP8, 4>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, qf, score_scale, m0, m1,
                                       l0, l1, o, lane);
           else if (nb == 2)
-            consume_blocks<D, FP8, 2>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
+            consume_blocks<D, FP8, 2>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, qf, score_scale, m0, m1,
                                       l0, l1, o, lane);
           else
-            consume_blocks<D, FP8, 1>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, tok1, qf, score_scale, m0, m1,
+            consume_blocks<D, FP8, 1>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, qf, score_scale, m0, m1,
                                       l0, l1, o, lane);
         }
         __syncwarp();
@@ -999,15 +1027,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_barrier_sync(1, cthreads);
     const float vs = FP8 ? p.v_scale[kvh] : 1.f;
-    for (int idx = ctid; idx < p.group * D; idx += cthreads) {
-      const int h = idx / D, d = idx - h * D;
+    // output row (query token tq, head h) combines the warps that computed query token tq
+    for (int idx = ctid; idx < q_len * p.group * D; idx += cthreads) {
+      const int row = idx / D, d = idx - row * D;
+      const int tq = MULTI ? row / p.group : 0, h = row - tq * p.group;
       float M = -INFINITY;
 #pragma unroll
-      for (int wq = 0; wq < kConsumerWarps; ++wq) M = fmaxf(M, red_m[wq * 8 + h]);
+      for (int wq = 0; wq < kConsumerWarps; ++wq)
+        if (!MULTI || (wq % wps) / wtok == tq) M = fmaxf(M, red_m[wq * 8 + h]);
       float Ls = 0.f, acc = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
         for (int wq = 0; wq < kConsumerWarps; ++wq) {
+          if (MULTI && (wq % wps) / wtok != tq) continue;
           const float e = exp2f(red_m[wq * 8 + h] - M);
           Ls += e * red_l[wq * 8 + h];
           acc += e * red_o[(wq * 8 + h) * S::kRedStride + (d ^ (4 * h))];
@@ -1016,11 +1048,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc *= vs;
       if (x.direct) {
         const float val = Ls > 0.f ? acc / Ls : 0.f;
-        const int64_t oi = (static_cast<int64_t>(x.req) * p.num_heads + head0 + h) * D + d;
+        const int64_t oi = ((static_cast<int64_t>(x.req) * q_len + tq) * p.num_heads + head0 + h) * D + d;
         if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
         else reinterpret_cast<float*>(p.out)[oi] = val;
       } else {
-        const int64_t pi = x.slot * p.group + h;
+        const int64_t pi = (x.slot * q_len + tq) * p.group + h;
         p.partial_o[pi * D + d] = acc;
         if (d == 0) {
           p.partial_ml[2 * pi] = M * kLn2;  // natural-log units
@@ -1122,12 +1154,13 @@ struct LaunchShape {
 // norm weights, frequencies and rotation tables.
 inline int static_smem_bytes(int D, bool pro) { return 512 + (pro ? D * 4 + D / 2 * 8 + 2 * D * 4 + 64 : 0); }
 
-int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls, bool pro = false) {
+int launch_shape(int D, bool fp8, int C, int ctas_per_sm, LaunchShape* ls, bool pro = false, int q_len = 1) {
   const int elt = fp8 ? 1 : 2;
   const int planes = D * elt / 128;
   const int plane_bytes = C * 128;
   const int stage_bytes = 2 * planes * plane_bytes;
-  const int bpc = C / 16, nb = blocks_per_warp(bpc, fp8), groups = kConsumerWarps / (bpc / nb);
+  const int q_pad = q_pad_of(q_len);
+  const int bpc = C / 16, nb = blocks_per_warp(bpc, fp8, q_pad), groups = kConsumerWarps / ((bpc / nb) * q_pad);
   const int red = kConsumerWarps * 8 * D * 4 + 2 * kConsumerWarps * 8 * 4;
   const int budget = kSmemLimit / (ctas_per_sm < 1 ? 1 : ctas_per_sm) - static_smem_bytes(D, pro);
   int stages = kMaxStages;
@@ -1149,10 +1182,10 @@ inline int chunk_tokens(int tile_len, int page_size) {
   return C > 64 ? 64 : C;
 }
 
-template <int D, bool FP8, bool FUSED, bool PRO = false>
+template <int D, bool FP8, bool FUSED, bool PRO = false, bool MULTI = false>
 int launch(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid, int smem,
            cudaStream_t stream) {
-  auto kern = decode_attention_kernel<D, FP8, FUSED, PRO>;
+  auto kern = decode_attention_kernel<D, FP8, FUSED, PRO, MULTI>;
   static int configured[64] = {0};  // per device: largest dynamic smem already allowed
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1206,7 +1239,7 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
             int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
             int32_t tile_len, int32_t grid, bool persistent, float sm_scale, void* out, hpc_dtype out_dtype,
             uint32_t* status, CUtensorMap* mk, CUtensorMap* mv, LaunchShape* ls, AttnParams* prm,
-            bool pro = false) {
+            bool pro = false, int q_len = 1) {
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !status)
     return fail(HPC_ERR_ARG, "null pointer argument");
   if (kv_dtype != HPC_BF16 && kv_dtype != HPC_E4M3) return fail(HPC_ERR_DTYPE, "kv_dtype must be BF16 or E4M3");
@@ -1235,7 +1268,7 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   int ctas_per_sm = (persistent && sms > 0) ? (grid + sms - 1) / sms : 1;
   if (ctas_per_sm < 1) ctas_per_sm = 1;
   if (ctas_per_sm > 4) ctas_per_sm = 4;
-  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, ls, pro);
+  int rc = launch_shape(head_dim, fp8, C, ctas_per_sm, ls, pro, q_len);
   if (rc) return rc;
   if ((rc = make_pool_map(mk, k_pages, fp8, nhd, head_dim, page_size, kv_heads, num_pages, C))) return rc;
   if ((rc = make_pool_map(mv, v_pages, fp8, nhd, head_dim, page_size, kv_heads, num_pages, C))) return rc;
@@ -1263,28 +1296,32 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   prm->kv_heads = kv_heads;
   prm->max_seq_len = max_pages_per_req * page_size;
   prm->nhd = nhd ? 1 : 0;
+  prm->q_len = q_len;
   return HPC_OK;
 }
 
-template <bool FUSED, bool PRO = false>
+template <bool FUSED, bool PRO = false, bool MULTI = false>
 int dispatch(int head_dim, bool fp8, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
              int smem, cudaStream_t st) {
-  if (fp8) return launch<128, true, FUSED, PRO>(mk, mv, prm, grid, smem, st);
-  if (head_dim == 128) return launch<128, false, FUSED, PRO>(mk, mv, prm, grid, smem, st);
-  return launch<64, false, FUSED, PRO>(mk, mv, prm, grid, smem, st);
+  if (fp8) return launch<128, true, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
+  if (head_dim == 128) return launch<128, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
+  return launch<64, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
 }
 
 struct StepLayout {
   size_t tickets, partial_o, partial_ml, total;
 };
 
-StepLayout step_layout(int32_t batch, int32_t group, int32_t kv_heads, int32_t head_dim, int32_t num_ctas) {
+// Rows of a partial slot: group heads for each of the q_len query tokens.
+StepLayout step_layout(int32_t batch, int32_t group, int32_t kv_heads, int32_t head_dim, int32_t num_ctas,
+                       int32_t q_len = 1) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t rows = static_cast<size_t>(group) * q_len;
   StepLayout L;
   L.tickets = 0;
   L.partial_o = up(static_cast<size_t>(batch) * kv_heads * sizeof(int32_t));
-  L.partial_ml = L.partial_o + up(2 * static_cast<size_t>(num_ctas) * group * head_dim * sizeof(float));
-  L.total = L.partial_ml + up(2 * static_cast<size_t>(num_ctas) * group * 2 * sizeof(float));
+  L.partial_ml = L.partial_o + up(2 * static_cast<size_t>(num_ctas) * rows * head_dim * sizeof(float));
+  L.total = L.partial_ml + up(2 * static_cast<size_t>(num_ctas) * rows * 2 * sizeof(float));
   return L;
 }
 
@@ -1340,8 +1377,10 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
               int32_t kv_heads, int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
               const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas, float sm_scale,
               void* workspace, size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
-              void* stream, const PrologueArgs* pro) {
+              void* stream, const PrologueArgs* pro, int32_t q_len = 1) {
   if (!workspace) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (q_len < 1 || q_len > 4) return fail(HPC_ERR_SHAPE, "q_len must be 1 to 4");
+  if (pro && q_len != 1) return fail(HPC_ERR_SHAPE, "the folded prologue takes one new token per request");
   if (batch < 1) return fail(HPC_ERR_ARG, "batch must be >= 1");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return fail(HPC_ERR_ALIGN, "workspace must be 256-byte aligned");
   if (kv_heads > 32767 || static_cast<int64_t>(batch) * kv_heads > (1ll << 30))
@@ -1352,20 +1391,23 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   int rc = prepare(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads,
                    head_dim, block_table, max_pages_per_req, seq_lens, tile_len, num_ctas, true, sm_scale, out,
-                   out_dtype, status, &mk, &mv, &ls, &prm, pro != nullptr);
+                   out_dtype, status, &mk, &mv, &ls, &prm, pro != nullptr, q_len);
   if (rc) return rc;
   // the per-request tile prefix lives in the reduce buffer while the CTA plans
   const size_t red_bytes = static_cast<size_t>(kConsumerWarps) * 8 * head_dim * sizeof(float);
   if ((static_cast<size_t>(batch) + 1) * sizeof(int64_t) > red_bytes)
     return fail(HPC_ERR_SHAPE, "batch %d is above the single-launch limit %zu; plan with hpc_decode_plan", batch,
                 red_bytes / sizeof(int64_t) - 1);
-  const StepLayout L = step_layout(batch, num_heads / kv_heads, kv_heads, head_dim, num_ctas);
+  const StepLayout L = step_layout(batch, num_heads / kv_heads, kv_heads, head_dim, num_ctas, q_len);
   if (workspace_bytes < L.total) return fail(HPC_ERR_CAPACITY, "step workspace %zu < %zu bytes", workspace_bytes, L.total);
   char* ws = static_cast<char*>(workspace);
   prm.tickets = reinterpret_cast<int32_t*>(ws + L.tickets);
   prm.partial_o = reinterpret_cast<float*>(ws + L.partial_o);
   prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
   prm.batch = batch;
+  if (!pro && q_len > 1)
+    return dispatch<true, false, true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
+                                       static_cast<cudaStream_t>(stream));
   if (!pro)
     return dispatch<true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
                           static_cast<cudaStream_t>(stream));
@@ -1392,6 +1434,26 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
   return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
                    workspace, workspace_bytes, out, out_dtype, status, stream, nullptr);
+}
+
+extern "C" size_t hpc_decode_step_multi_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_heads,
+                                                        int32_t kv_heads, int32_t head_dim, int32_t num_ctas) {
+  if (batch < 1 || q_len < 1 || num_heads < 1 || kv_heads < 1 || head_dim < 1 || num_ctas < 1 || num_heads % kv_heads)
+    return 0;
+  return step_layout(batch, num_heads / kv_heads, kv_heads, head_dim, num_ctas, q_len).total;
+}
+
+extern "C" int hpc_decode_step_multi(const void* q, int32_t q_len, const void* k_pages, const void* v_pages,
+                                     hpc_dtype kv_dtype, hpc_kv_layout kv_layout, const float* k_scale,
+                                     const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads,
+                                     int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                                     int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch,
+                                     int32_t tile_len, int32_t num_ctas, float sm_scale, void* workspace,
+                                     size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
+                                     void* stream) {
+  return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
+                   workspace, workspace_bytes, out, out_dtype, status, stream, nullptr, q_len);
 }
 
 extern "C" int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,

@@ -31,7 +31,8 @@ def declared_symbols():
 def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ("hpc_decode_plan", "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue",
-              "hpc_plan_cpu", "hpc_decode_plan_static", "hpc_decode_step", "hpc_decode_step_prologue"):
+              "hpc_plan_cpu", "hpc_decode_plan_static", "hpc_decode_step", "hpc_decode_step_prologue",
+              "hpc_decode_step_multi"):
         assert n in names
 
 
@@ -43,7 +44,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 3
+    assert B._lib.hpc_abi_version() == 4
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -67,6 +68,13 @@ def test_host_argument_errors_return_codes(B):
     rc = B._lib.hpc_decode_step_prologue(w, w, w, 1e-6, -1.0, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1,
                                          32, 4, 0.1, w, 0, w, 1, w, None)
     assert rc == B.HPC_ERR_ARG and "rope_theta" in B._lib.hpc_last_error().decode()
+    # several new tokens: q_len outside 1..4 and zero-size workspace queries
+    rc = B._lib.hpc_decode_step_multi(w, 5, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1, 32, 4, 0.1, w, 1 << 20,
+                                      w, 1, w, None)
+    assert rc == B.HPC_ERR_SHAPE and "q_len" in B._lib.hpc_last_error().decode()
+    assert B._lib.hpc_decode_step_multi_workspace_bytes(4, 0, 8, 2, 64, 148) == 0
+    assert (B._lib.hpc_decode_step_multi_workspace_bytes(4, 1, 8, 2, 64, 148)
+            == B._lib.hpc_decode_step_workspace_bytes(4, 8, 2, 64, 148))
     # bad tile_len on the host planner
     lens = torch.tensor([5, 7], dtype=torch.int32)
     with pytest.raises(B.HpcError, match="tile_len"):
