@@ -1,0 +1,386 @@
+// Device code shared by the attention kernels of libhpcdecode: kernel parameters, the work
+// cursors (a materialised plan, or the planner's closed form walked in the kernel), the
+// in-kernel plan prefix, the zero rows of empty requests and the ticket merge of split
+// (request, kv head) segments. The mma.sync kernel (attention.cu) and the tcgen05 kernel for
+// E4M3 caches (attention_tc.cu) both include it.
+#pragma once
+
+#include <math.h>
+#include <stdlib.h>
+
+#include "hpc_common.cuh"
+
+namespace hpc {
+namespace attn {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxStages = 16;
+constexpr int kSmemLimit = 232448;  // 227 KB per block on sm_100
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnParams {
+  const __nv_bfloat16* q;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const hpc_work_item* items;
+  const int32_t* cta_indptr;
+  const float* k_scale;
+  const float* v_scale;
+  float* partial_o;
+  float* partial_ml;
+  void* out;
+  uint32_t* status;
+  int64_t max_pages;
+  int32_t num_pages, page_size, tile_len, chunk_tokens, num_heads, group;
+  int32_t stages, out_bf16;
+  uint32_t plane_bytes, stage_bytes;
+  float score_scale;  // sm_scale * log2(e)
+  int32_t q_len;      // new tokens per request (single-launch step); 1 elsewhere
+  int32_t nhd;        // cache layout: token stride Hkv*D (NHD) or D (HND); only the TMA coordinates differ
+  // single-launch step only: the plan is derived in the kernel from seq_lens
+  int32_t batch, kv_heads, max_seq_len;
+  int32_t* tickets;  // [batch * kv_heads], zero between steps
+  // single-launch step with the prologue folded in: q comes from qkv through RMSNorm and RoPE,
+  // and the new token's K/V are written into the cache
+  const __nv_bfloat16* qkv;  // [batch][num_heads + 2 kv_heads][D]
+  const float* q_norm_w;
+  const float* k_norm_w;
+  void* k_pages_w;  // the caches, for the new token's write
+  void* v_pages_w;
+  float eps;
+  double rope_theta;
+};
+
+// One work item as the producer and the consumers see it.
+struct ItemInfo {
+  int32_t req, kvh;
+  int64_t tok0, tok1;  // tokens to stream
+  bool direct;         // covers its whole (request, kv head): writes the output itself
+  int64_t slot;        // partial-state slot of a split item
+  int64_t U;           // single-launch step: first unit of the (request, kv head) segment
+  int32_t nt;          // and its tile count
+};
+
+// 16-token blocks that one consumer warp takes from a stage of `bpc` blocks. Two blocks give
+// two independent MMA chains. An E4M3 stage carries half the bytes per token, so the fixed
+// per-call softmax work (row max across lanes, rescale factors) and the stage handshake weigh
+// twice as much per byte: there a warp takes up to four blocks, a whole 64-token stage.
+__host__ __device__ __forceinline__ int blocks_per_warp(int bpc, bool fp8, int q_pad = 1) {
+  if (fp8 && bpc >= 4 && q_pad == 1) return 4;
+  return bpc >= 2 ? 2 : 1;
+}
+
+// Several new tokens per request: q_len query tokens take q_pad = 1, 2 or 4 warp slots of each
+// stage (q_len 3 leaves one slot idle). Each warp computes one query token's rows over its
+// blocks, so a stage is read by (blocks per stage / blocks per warp) * q_pad warps.
+__host__ __device__ __forceinline__ int q_pad_of(int q_len) { return q_len <= 1 ? 1 : (q_len <= 2 ? 2 : 4); }
+
+__device__ __forceinline__ int32_t tiles_of(int32_t L, int32_t tl) {
+  return L > 0 ? static_cast<int32_t>(static_cast<uint32_t>(L - 1) / static_cast<uint32_t>(tl) + 1) : 0;
+}
+
+// A length is valid when it is 0 (no tiles, zero output) or holds the step's q_len new tokens
+// and fits the block table.
+__device__ __forceinline__ bool len_ok(int32_t L, int32_t max_seq_len, int32_t q_len = 1) {
+  return L >= 0 && (L == 0 || L >= q_len) && (max_seq_len <= 0 || L <= max_seq_len);
+}
+
+template <int D, bool FP8>
+struct Shape {
+  static constexpr int kElt = FP8 ? 1 : 2;
+  static constexpr int kPlanes = D * kElt / 128;  // 128-byte swizzle planes per token row
+  static constexpr int kRedStride = D;  // floats per (warp, head) row; columns XOR 4h against bank conflicts
+};
+
+// Output row index of accumulator register `half` (0: c0/c1, 1: c2/c3) for lane row g
+// inside a 16-row block. bf16 V comes from ldmatrix.trans in natural order (rows g, g+8).
+// E4M3 V comes from ldmatrix.trans on byte pairs, so rows g and g+8 hold d = 2g and 2g+1.
+template <bool FP8>
+__device__ __forceinline__ int out_row(int g, int half) {
+  if (FP8) return 2 * g + half;
+  return g + 8 * half;
+}
+
+// One past the last token of an item: its last tile, clipped to the request length and to
+// what the block table can address (a plan built for other lengths cannot read past it).
+__device__ __forceinline__ int64_t item_end(const hpc_work_item& w, int32_t L, int tl, int64_t capacity) {
+  int64_t e = static_cast<int64_t>(w.tile_end) * tl;
+  if (e > L) e = L;
+  if (e > capacity) e = capacity;
+  return e;
+}
+
+// Items of one CTA, read from a device plan (hpc_decode_plan / hpc_decode_plan_static).
+struct PlanCursor {
+  int it, it_end;
+  __device__ bool next(const AttnParams& p, ItemInfo& x) {
+    if (it >= it_end) return false;
+    const hpc_work_item w = p.items[it];
+    x.req = w.req;
+    x.kvh = w.kv_head;
+    x.tok0 = static_cast<int64_t>(w.tile_begin) * p.tile_len;
+    x.tok1 = item_end(w, p.seq_lens[w.req], p.tile_len, p.max_pages * p.page_size);
+    x.direct = (w.flags & HPC_ITEM_DIRECT) != 0;
+    x.slot = it;
+    x.U = 0;
+    x.nt = 0;
+    ++it;
+    return true;
+  }
+};
+
+// Items of one CTA, derived in the kernel by the planner's closed form: the CTA owns units
+// [u, u_end) of the request -> kv head -> tile enumeration and cuts them at (request, kv head)
+// boundaries. A split (request, kv head) is always this CTA's first or last item, so two
+// partial slots per CTA suffice: 2g for a piece that starts at the CTA's first unit, 2g + 1
+// otherwise.
+struct WalkCursor {
+  int64_t u, u_end, u_first, U_r;
+  int32_t r, kvh, nt, tb, g;
+  __device__ bool next(const AttnParams& p, ItemInfo& x) {
+    if (u >= u_end) return false;
+    const int32_t te = static_cast<int32_t>(min(static_cast<int64_t>(nt), tb + (u_end - u)));
+    const int32_t L = p.seq_lens[r];
+    x.req = r;
+    x.kvh = kvh;
+    x.tok0 = static_cast<int64_t>(tb) * p.tile_len;
+    int64_t e = static_cast<int64_t>(te) * p.tile_len;
+    if (e > L) e = L;
+    x.tok1 = e;
+    x.direct = tb == 0 && te == nt;
+    x.slot = 2 * static_cast<int64_t>(g) + (u == u_first ? 0 : 1);
+    x.U = U_r + static_cast<int64_t>(kvh) * nt;
+    x.nt = nt;
+    u += te - tb;
+    tb = 0;
+    if (u < u_end) {  // step to the next (request, kv head) with tiles
+      if (++kvh == p.kv_heads) {
+        kvh = 0;
+        U_r += static_cast<int64_t>(p.kv_heads) * nt;
+        do {
+          ++r;
+          const int32_t Ln = p.seq_lens[r];
+          nt = len_ok(Ln, p.max_seq_len, p.q_len) ? tiles_of(Ln, p.tile_len) : 0;
+        } while (nt == 0);
+      }
+    }
+    return true;
+  }
+};
+
+template <bool FUSED>
+struct CursorOf {
+  using type = PlanCursor;
+};
+template <>
+struct CursorOf<true> {
+  using type = WalkCursor;
+};
+
+// Single-launch step: each CTA finds where its unit range starts. It forms the exclusive
+// prefix sum of per-request tile counts in shared memory (the reduce buffer, unused until
+// the first item ends) and binary-searches it. Requests with no valid tiles get a zero
+// output from CTA r % num_ctas. Returns the walk cursor (all threads get the same one).
+template <int D>
+__device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_scan, int64_t* s_walk,
+                               WalkCursor& cur, int64_t& chunk) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int B = p.batch, Hkv = p.kv_heads, G = gridDim.x, g = blockIdx.x;
+  // per-thread contiguous run of requests, then a block scan of the run totals
+  const int per = (B + nthr - 1) / nthr;
+  const int r0 = min(B, tid * per), r1 = min(B, r0 + per);
+  int64_t run = 0;
+  uint32_t bad = 0;
+  for (int r = r0; r < r1; ++r) {
+    const int32_t L = p.seq_lens[r];
+    const bool ok = len_ok(L, p.max_seq_len, p.q_len);
+    if (!ok) bad |= HPC_DEV_BAD_SEQLEN;
+    run += ok ? tiles_of(L, p.tile_len) : 0;
+  }
+  if (bad && (r0 % G) == g) atomicOr(p.status, bad);
+  const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
+  int64_t x = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_scan[warp] = x;
+  __syncthreads();
+  if (tid == 0) {
+    int64_t acc = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int64_t t = s_scan[w];
+      s_scan[w] = acc;
+      acc += t;
+    }
+    s_scan[nwarps] = acc;
+  }
+  __syncthreads();
+  int64_t pre = s_scan[warp] + x - run;
+  for (int r = r0; r < r1; ++r) {
+    s_pre[r] = pre;
+    const int32_t L = p.seq_lens[r];
+    pre += len_ok(L, p.max_seq_len, p.q_len) ? tiles_of(L, p.tile_len) : 0;
+  }
+  if (tid == 0) s_pre[B] = s_scan[nwarps];
+  __syncthreads();
+  if (tid == 0) {
+    const int64_t T = s_pre[B] * Hkv;
+    const int64_t ch = T > 0 ? (T + G - 1) / G : 0;
+    const int64_t u0 = static_cast<int64_t>(g) * ch;
+    const int64_t u1 = min(u0 + ch, T);
+    int64_t r = 0, kvh = 0, tb = 0, nt = 0, U_r = 0;
+    if (u0 < T) {
+      // largest r with Hkv * s_pre[r] <= u0: the request that holds unit u0
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] * Hkv <= u0) lo = mid;
+        else hi = mid - 1;
+      }
+      r = lo;
+      nt = s_pre[r + 1] - s_pre[r];
+      U_r = s_pre[r] * Hkv;
+      kvh = (u0 - U_r) / nt;
+      tb = u0 - U_r - kvh * nt;
+    }
+    s_walk[0] = u0;
+    s_walk[1] = u1;
+    s_walk[2] = U_r;
+    s_walk[3] = r;
+    s_walk[4] = kvh;
+    s_walk[5] = nt;
+    s_walk[6] = tb;
+    s_walk[7] = ch;
+  }
+  __syncthreads();
+  cur.u = s_walk[0];
+  cur.u_first = s_walk[0];
+  cur.u_end = s_walk[1];
+  cur.U_r = s_walk[2];
+  cur.r = static_cast<int32_t>(s_walk[3]);
+  cur.kvh = static_cast<int32_t>(s_walk[4]);
+  cur.nt = static_cast<int32_t>(s_walk[5]);
+  cur.tb = static_cast<int32_t>(s_walk[6]);
+  cur.g = g;
+  chunk = s_walk[7];
+}
+
+// Zero output rows of requests that own no tiles (L = 0 or an invalid length).
+template <int D>
+__device__ void zero_empty_requests(const AttnParams& p, int tid, int nthr) {
+  for (int r = blockIdx.x; r < p.batch; r += gridDim.x) {
+    const int32_t L = p.seq_lens[r];
+    if (len_ok(L, p.max_seq_len, p.q_len) && L > 0) continue;
+    const int64_t rows = static_cast<int64_t>(p.q_len) * p.num_heads * D;
+    const int64_t base = static_cast<int64_t>(r) * rows;
+    for (int64_t i = tid; i < rows; i += nthr) {
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[base + i] = __float2bfloat16_rn(0.f);
+      else reinterpret_cast<float*>(p.out)[base + i] = 0.f;
+    }
+  }
+}
+
+// Log-sum-exp merge of a split (request, kv head) by the CTA that finished its last piece.
+// Piece slots follow the walk cursor's rule: the piece in CTA gg is slot 2gg, except the first
+// piece when it starts inside CTA g1's range (slot 2 g1 + 1). All (piece, head) states are
+// loaded at once into shared memory (the reduce buffer, free at this point) and turned into
+// weights exp(m_i - M) / L. The output is then a weighted sum over independent loads. The
+// other CTAs' partial states are read through L2 (ld.global.cg) after the ticket's fence.
+template <int D>
+__device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t chunk, int tid, int nthr,
+                              float* s_buf, int buf_floats) {
+  const int64_t g1 = x.U / chunk, g2 = (x.U + x.nt - 1) / chunk;
+  const int64_t first_slot = (x.U > g1 * chunk) ? 2 * g1 + 1 : 2 * g1;
+  // rows of a piece: query token t, head h -> row t * group + h
+  const int grp = p.group * p.q_len;
+  const int n = static_cast<int>(g2 - g1 + 1);
+  auto slot_of = [&](int i) -> int64_t { return i == 0 ? first_slot : 2 * (g1 + i); };
+  auto out_at = [&](int idx) -> int64_t {  // idx = row * D + d
+    const int row = idx / D, t = row / p.group, h = row - t * p.group;
+    return ((static_cast<int64_t>(x.req) * p.q_len + t) * p.num_heads + x.kvh * p.group + h) * D + (idx - row * D);
+  };
+  float* s_m = s_buf;
+  float* s_w = s_buf + n * grp;
+  float* s_M = s_w + n * grp;
+  float* s_iL = s_M + grp;
+  if (2 * n * grp + 2 * grp <= buf_floats) {
+    for (int k = tid; k < n * grp; k += nthr) {
+      const int i = k / grp, h = k - i * grp;
+      const float* ml = p.partial_ml + 2 * (slot_of(i) * grp + h);
+      s_m[k] = __ldcg(ml);
+      s_w[k] = __ldcg(ml + 1);
+    }
+    named_barrier_sync(1, nthr);
+    if (tid < grp) {
+      float M = -INFINITY;
+      for (int i = 0; i < n; ++i) M = fmaxf(M, s_m[i * grp + tid]);
+      float L = 0.f;
+      for (int i = 0; i < n; ++i) L += expf(s_m[i * grp + tid] - M) * s_w[i * grp + tid];
+      s_M[tid] = M;
+      s_iL[tid] = L > 0.f ? 1.f / L : 0.f;
+    }
+    named_barrier_sync(1, nthr);
+    for (int k = tid; k < n * grp; k += nthr) {
+      const int h = k % grp;
+      s_w[k] = expf(s_m[k] - s_M[h]) * s_iL[h];
+    }
+    named_barrier_sync(1, nthr);
+    for (int idx = tid; idx < grp * D; idx += nthr) {
+      const int h = idx / D;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      int i = 0;
+      for (; i + 4 <= n; i += 4) {
+        a0 += s_w[(i + 0) * grp + h] * __ldcg(p.partial_o + slot_of(i + 0) * grp * D + idx);
+        a1 += s_w[(i + 1) * grp + h] * __ldcg(p.partial_o + slot_of(i + 1) * grp * D + idx);
+        a2 += s_w[(i + 2) * grp + h] * __ldcg(p.partial_o + slot_of(i + 2) * grp * D + idx);
+        a3 += s_w[(i + 3) * grp + h] * __ldcg(p.partial_o + slot_of(i + 3) * grp * D + idx);
+      }
+      for (; i < n; ++i) a0 += s_w[i * grp + h] * __ldcg(p.partial_o + slot_of(i) * grp * D + idx);
+      const float val = (a0 + a1) + (a2 + a3);
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[out_at(idx)] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(p.out)[out_at(idx)] = val;
+    }
+    return;
+  }
+  // more pieces than the buffer holds: two passes over the partial states per output
+  for (int idx = tid; idx < grp * D; idx += nthr) {
+    const int h = idx / D;
+    float M = -INFINITY;
+    for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(p.partial_ml + 2 * (slot_of(i) * grp + h)));
+    float Ls = 0.f, acc = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const int64_t pi = slot_of(i) * grp + h;
+      const float e = expf(__ldcg(p.partial_ml + 2 * pi) - M);
+      Ls += e * __ldcg(p.partial_ml + 2 * pi + 1);
+      acc += e * __ldcg(p.partial_o + pi * D + (idx - h * D));
+    }
+    const float val = Ls > 0.f ? acc / Ls : 0.f;
+    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[out_at(idx)] = __float2bfloat16_rn(val);
+    else reinterpret_cast<float*>(p.out)[out_at(idx)] = val;
+  }
+}
+
+// E4M3 caches run on the mma.sync kernel; HPC_E4M3_TCGEN05=1 in the environment selects the
+// tcgen05 kernel (attention_tc.cu) where it applies. Measured on the large-batch E4M3 workload
+// the mma.sync kernel is the faster one (775 against 1278 us per step): with N = 16 per product
+// and 128 tokens per stage, the tcgen05 pipeline is bound by its per-stage round trips.
+inline bool e4m3_on_tensor_cores() {
+  const char* e = getenv("HPC_E4M3_TCGEN05");
+  return e && e[0] == '1';
+}
+
+// The tcgen05 kernel for E4M3 caches (attention_tc.cu). It serves the one-token single-launch
+// step and the three-launch attention when the cache is E4M3, head_dim is 128 and the group is
+// at most 8 heads. Returns an hpc_status.
+bool tc_supported(int head_dim, bool fp8, int group, int q_len, bool pro);
+int tc_smem_bytes(int ctas_per_sm);
+int tc_threads();
+int launch_attention_tc(bool fused, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
+                        cudaStream_t stream);
+
+}  // namespace attn
+}  // namespace hpc

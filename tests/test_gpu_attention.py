@@ -2,11 +2,14 @@
 element (several tiles, ragged tails, every supported shape), the named workloads at full
 size on sampled requests, plus invariances (page permutation, run-to-run determinism,
 plan choice) and edge cases (L = 1, L = 0, NaN in unused slots, bad page ids)."""
+import os
+
 import numpy as np
 import pytest
 import torch
 
 from load_balanced_split_step_b200 import workloads as W
+from oracle import fp8 as OF
 from tests.helpers import assert_bf16_tol, errors, oracle_out, run_attention, to_device
 
 pytestmark = pytest.mark.gpu
@@ -52,22 +55,66 @@ def test_shapes_ragged(B, Hq, Hkv, D, P, tl):
         assert_bf16_tol(out, ref, what=f"{(Hq, Hkv, D, P, tl, G)}")
 
 
+@pytest.mark.parametrize("consumer", ["mma.sync", "tcgen05"])
 @pytest.mark.parametrize("Hq,Hkv,P,tl", [
     (8, 8, 16, 16), (16, 2, 16, 48), (16, 4, 32, 32), (32, 8, 32, 64), (8, 2, 64, 64), (64, 8, 64, 128),
     (32, 8, 128, 128), (16, 4, 128, 256),
 ])
-def test_e4m3_shapes_ragged(B, Hq, Hkv, P, tl):
-    """E4M3 cache over every stage size (16, 32 and 64 tokens: one, two and four 16-token
-    blocks per consumer warp) and every GQA group size."""
+def test_e4m3_shapes_ragged(B, Hq, Hkv, P, tl, consumer):
+    """E4M3 cache over every stage size (mma.sync: 16, 32 and 64 tokens, one, two and four
+    16-token blocks per consumer warp; tcgen05: 128-token stages of 16-, 32- and 64-token boxes)
+    and every GQA group size, on both E4M3 kernels, three-launch and single-launch paths."""
     lens = (1, 15, 16, 17, 63, 64, 65, 129, 300, 1000, 2049)
     spec, case = _case(lens, Hq, Hkv, 128, P, tl, seed=Hq + P + tl, kv="e4m3")
     dc = to_device(case)
     ref = oracle_out(case)
-    for G in (5, 148):
-        out, _, st = run_attention(B, spec, dc, num_ctas=G)
+    if consumer == "tcgen05":
+        os.environ["HPC_E4M3_TCGEN05"] = "1"
+    try:
+        for G in (5, 148):
+            out, _, st = run_attention(B, spec, dc, num_ctas=G)
+            assert st == 0
+            mx, _ = errors(out, ref)
+            assert mx <= 5e-2, (consumer, Hq, Hkv, P, tl, G, mx)
+            out, st_t, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
+                                               dc["seq_lens"], Hq, Hkv, tl, kv_dtype="e4m3", k_scale=dc["k_scale"],
+                                               v_scale=dc["v_scale"], num_ctas=G)
+            torch.cuda.synchronize()
+            assert int(st_t.item()) == 0
+            mx, _ = errors(out, ref)
+            assert mx <= 5e-2, (consumer, "fused", Hq, Hkv, P, tl, G, mx)
+    finally:
+        os.environ.pop("HPC_E4M3_TCGEN05", None)
+
+
+@pytest.mark.parametrize("path", ["split", "fused"])
+def test_e4m3_both_consumers(B, path):
+    """An E4M3 cache runs on the mma.sync kernel; HPC_E4M3_TCGEN05=1 selects the tcgen05
+    kernel. Both must meet the E4M3 tolerance on the same ragged batch, on both step paths."""
+    spec, case = _case((1, 2, 15, 16, 17, 127, 128, 129, 255, 256, 257, 4000), 32, 4, 128, 32, 64, seed=77,
+                       kv="e4m3")
+    dc = to_device(case)
+    ref = oracle_out(case)
+    outs = {}
+    for consumer in ("tcgen05", "mma.sync"):
+        if consumer == "tcgen05":
+            os.environ["HPC_E4M3_TCGEN05"] = "1"
+        try:
+            if path == "split":
+                out, _, st = run_attention(B, spec, dc, num_ctas=37)
+            else:
+                out, st_t, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
+                                                   dc["seq_lens"], 32, 4, 64, kv_dtype="e4m3", k_scale=dc["k_scale"],
+                                                   v_scale=dc["v_scale"], num_ctas=37)
+                torch.cuda.synchronize()
+                st = int(st_t.item())
+        finally:
+            os.environ.pop("HPC_E4M3_TCGEN05", None)
         assert st == 0
-        mx, _ = errors(out, ref)
-        assert mx <= 5e-2, (Hq, Hkv, P, tl, G, mx)
+        mx, mean = errors(out, ref)
+        assert mx <= 5e-2, (consumer, mx)
+        outs[consumer] = out
+    assert not torch.equal(outs["tcgen05"], outs["mma.sync"])  # two kernels really ran
 
 
 def test_bf16_output_within_one_ulp(B):
@@ -174,10 +221,17 @@ def test_e4m3_cache_small(B):
         assert st == 0
         mx, mean = errors(out, ref)
         assert mx <= 5e-2, mx
-    # the split must not matter beyond fp32 rounding
+    # The split moves only the running maxima against which p is rounded before the P.V
+    # product. The mma.sync kernel rounds p to f16 (11 bits); the tcgen05 kernel sends p (scaled
+    # by 2^8, so p <= 256) as an E4M3 high code plus an E4M3 residual code, off by at most
+    # 2^-8 p + 2^-10 (the residual's subnormal spacing is 2^-9) against a normaliser l of at
+    # least 256 (the maximum's own p). For the coarser of the two, one split's output is within
+    # max|v| (2^-8 + L 2^-18) of the exact mix, and two splits within twice that.
     o1, _, _ = run_attention(B, spec, dc, num_ctas=1)
     o2, _, _ = run_attention(B, spec, dc, num_ctas=148)
-    assert torch.max(torch.abs(o1 - o2)).item() < 1e-4
+    vmax = float(np.nanmax(np.abs(OF.decode_array(case.v_pages.numpy())) * case.v_scale.numpy()[None, :, None, None]))
+    bound = 2 * vmax * (2.0**-8 + max(spec.seq_lens) * 2.0**-18)
+    assert torch.max(torch.abs(o1 - o2)).item() <= bound
 
 
 # ---------------------------------------------------------------- full-size workloads
