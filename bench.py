@@ -61,6 +61,9 @@ def parse_args(argv=None):
                          "plan, attention and merge kernels")
     ap.add_argument("--q-len", type=int, default=1,
                     help="new tokens per request, attending causally (1 to 4; single-launch path)")
+    ap.add_argument("--shard", action="store_true",
+                    help="request-sharded placement of ONE batch over the ranks (strong scaling): each rank runs its "
+                         "parts, (out, lse) are all-gathered and split requests merged; default: independent replicas")
     ap.add_argument("--no-extras", action="store_true", help="skip static split-k, e2e and CPU baseline legs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     return ap.parse_args(argv)
@@ -256,6 +259,35 @@ class Step:
         return (1 if self.fused else 3) + pro
 
 
+class ShardStep:
+    """The step of one batch placed over the ranks by request (load_balanced_split_step_b200.shard):
+    local parts through hpc_decode_step_lse, one all-gather of (out, lse), hpc_merge_lse."""
+
+    def __init__(self, B, spec, dc, num_ctas, tile_len, rank, world):
+        from load_balanced_split_step_b200 import shard as SH
+        self.spec, self.dc, self.tl = spec, dc, tile_len
+        self.status = torch.zeros(1, dtype=torch.int32, device=dc["seq_lens"].device)
+        compute = SH.library_compute(spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype, k_scale=dc["k_scale"],
+                                     v_scale=dc["v_scale"], num_ctas=num_ctas, status=self.status)
+        self.st = SH.ShardedStep(spec.seq_lens, world, rank, spec.page_size, spec.num_heads, spec.head_dim,
+                                 compute=compute)
+        self.out = None
+
+    def __call__(self, seq_lens=None, ev=None, q=None):
+        d = self.dc
+        if ev is not None:
+            ev[0].record()
+        self.out = self.st.step(d["q"] if q is None else q, d["k_pages"], d["v_pages"], d["block_table"], self.tl)
+        if ev is not None:
+            ev[1].record()
+        return self.out
+
+    @property
+    def launches(self):
+        split = sum(1 for places in self.st.where.values() if len(places) > 1)
+        return 1 + split  # the step, then one merge per split request
+
+
 def step_lengths(dc, spec):
     """Device length vectors for each decode step (heavy-tailed grows by one per step)."""
     return [dc["seq_lens"] + i for i in range(spec.steps)]
@@ -293,6 +325,31 @@ def static_leg(B, spec, dc, tl, steps, sms, layout="HND"):
     return {"splits_rule": "S = max(1, ceil(2*SMs/(B*Hkv)))", "S": S0, "us_per_step": round(res[S0], 2),
             "best_S": best, "best_us_per_step": round(res[best], 2),
             "sweep_us": {str(k): round(v, 2) for k, v in res.items()}}
+
+
+def shard_e2e_leg(step, case, dc, steps, world):
+    """The sharded step with q copied in from pinned host memory and the output copied out,
+    every step, in order on one stream (the exchange is inside the step)."""
+    dev = dc["seq_lens"].device
+    q_host = case.q.pin_memory()
+    q_dev = torch.empty_like(q_host, device=dev)
+    host = None
+    for _ in range(3):
+        q_dev.copy_(q_host, non_blocking=True)
+        out = step(q=q_dev)
+        host = out.to("cpu", non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        q_dev.copy_(q_host, non_blocking=True)
+        out = step(q=q_dev)
+        host = out.to("cpu", non_blocking=True)
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return a.elapsed_time(b), q_host.numel() * q_host.element_size(), host.numel() * host.element_size()
 
 
 def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND", folded=False):
@@ -454,7 +511,7 @@ def load_peaks():
 def kernel_source_hash():
     import hashlib
     h = hashlib.sha256()
-    for name in ("attention.cu", "hpc_common.cuh"):
+    for name in ("attention.cu", "attention_common.cuh", "hpc_common.cuh"):
         with open(os.path.join(ROOT, "load_balanced_split_step_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -495,7 +552,13 @@ def run_ours(args, rank, world, local):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     tl = args.tile_len or spec.tile_len
     G = sms * args.ctas_per_sm
-    step = Step(B, spec, dc, G, tl, fused=args.path == "fused", folded=args.path == "folded", layout=args.layout)
+    if args.shard:
+        if spec.prologue or spec.q_len != 1 or spec.steps != 1 or args.layout != "HND":
+            raise SystemExit("--shard runs one-step, one-token workloads without the prologue, HND cache")
+        step = ShardStep(B, spec, dc, G, tl, rank, world)
+    else:
+        step = Step(B, spec, dc, G, tl, fused=args.path == "fused", folded=args.path == "folded",
+                    layout=args.layout)
     lens = step_lengths(dc, spec)
     K, W_ = args.steps, max(3, args.warmup)
 
@@ -512,14 +575,17 @@ def run_ours(args, rank, world, local):
     total_ms = max_over_ranks(total_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
     bytes_step = float(np.mean([W.algorithmic_bytes(spec, i % spec.steps) for i in range(spec.steps)]))
-    value = world * bytes_step * K / (total_ms / 1e3) / 1e9
+    jobs = 1 if args.shard else world  # sharded: the ranks share one batch
+    value = jobs * bytes_step * K / (total_ms / 1e3) / 1e9
     ms_step = total_ms / K
     peak, peak_kind = load_peaks()
     achieved = bytes_step / (kern_ms / 1e3) / 1e9
+    if args.shard:  # per GPU: its share of the batch over the step, exchange and merge included
+        achieved = bytes_step / world / (kern_ms / 1e3) / 1e9
     clocks = clk.summary()
 
     extra = {}
-    if not args.no_extras:
+    if not args.no_extras and not args.shard:
         # graph replay of the same step (host launch overhead removed)
         g = torch.cuda.CUDAGraph()
         s = torch.cuda.Stream()
@@ -545,11 +611,14 @@ def run_ours(args, rank, world, local):
             extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms, args.layout)
             extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step),
                                                        3)
-    e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, max(50, K // 4), world, fused=args.path != "split",
-                               layout=args.layout, folded=args.path == "folded")
-    e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_steps = max(50, K // 4)
-    e2e_val = world * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
+    if args.shard:
+        e2e_ms, h2d, d2h = shard_e2e_leg(step, case, dc, e2e_steps, world)
+    else:
+        e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, e2e_steps, world, fused=args.path != "split",
+                                   layout=args.layout, folded=args.path == "folded")
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_val = jobs * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
@@ -559,7 +628,8 @@ def run_ours(args, rank, world, local):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W_,
         "ms_per_step": round(ms_step, 5), "us_per_step": round(1000 * ms_step, 2), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if spec.kv_dtype == "bf16" else "e4m3/f16",
+        "scaling": "strong" if args.shard else "weak", "vs_baseline": None,
+        "dtype": "bf16" if spec.kv_dtype == "bf16" else "e4m3/f16",
         "data": "synthetic (seeded N(0,1), bf16-rounded; random page permutation)",
         "config": {"workload": WORKLOAD_TEXT[args.workload] + qlen_text(args), "tile_len": tl, "num_ctas": G,
                    "plan": "dynamic (re-planned on the device every step)",
@@ -570,7 +640,9 @@ def run_ours(args, rank, world, local):
                                       + (" after the prologue kernel" if spec.prologue else "")}[args.path]),
                    "kv_layout": args.layout,
                    "l2": f"inputs larger than L2 ({bytes_step / 1e9:.2f} GB per step), no flush",
-                   "parallelism": f"{world} independent replica(s), no collective"},
+                   "parallelism": (f"one batch request-sharded over {world} GPU(s): one all-gather of (out, lse), "
+                                   "log-sum-exp merge of split requests") if args.shard
+                   else f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8000": round(achieved / 8000.0, 4),

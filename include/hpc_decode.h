@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 4
+#define HPC_DECODE_ABI_VERSION 5
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -250,6 +250,29 @@ HPC_API int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, con
                                      const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
                                      float sm_scale, void* workspace, size_t workspace_bytes, void* out,
                                      hpc_dtype out_dtype, uint32_t* status, void* stream);
+
+/* hpc_decode_step that also writes the log-sum-exp of every output row:
+ *   lse[r][h] = log sum_j exp(sm_scale * q[r,h] . k_j)   (natural log; -inf when L_r = 0),
+ * the quantity that combines outputs over disjoint parts of one request's keys (see
+ * hpc_merge_lse). lse: device float [batch][num_heads]. Everything else as hpc_decode_step. */
+HPC_API int hpc_decode_step_lse(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                                hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages,
+                                int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
+                                const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
+                                int32_t batch, int32_t tile_len, int32_t num_ctas, float sm_scale, void* workspace,
+                                size_t workspace_bytes, void* out, hpc_dtype out_dtype, float* lse, uint32_t* status,
+                                void* stream);
+
+/* Log-sum-exp merge of outputs computed over disjoint parts of the same keys (a request split
+ * across GPUs in request-sharded placement; the pages describe the split of a request's tiles
+ * across processing units but no merge step, so this extends the in-GPU merge to parts made
+ * elsewhere). For each row r:
+ *   LSE = log sum_i exp(lses[i][r]),   out[r] = sum_i exp(lses[i][r] - LSE) outs[i][r].
+ * A row whose parts are all -inf gets zeros and -inf.
+ *   outs: device float [parts][rows][head_dim]; lses: device float [parts][rows].
+ *   out:  device float [rows][head_dim]; lse_out: device float [rows], or NULL. */
+HPC_API int hpc_merge_lse(const float* outs, const float* lses, int32_t parts, int64_t rows, int32_t head_dim,
+                          float* out, float* lse_out, void* stream);
 
 /* ---- several new tokens per request ----------------------------------------------------- */
 

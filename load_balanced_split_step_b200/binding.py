@@ -30,7 +30,8 @@ EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_d
            "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue", "hpc_attention_launch_info",
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
            "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue",
-           "hpc_decode_step_multi", "hpc_decode_step_multi_workspace_bytes")
+           "hpc_decode_step_multi", "hpc_decode_step_multi_workspace_bytes", "hpc_decode_step_lse",
+           "hpc_merge_lse")
 
 
 class HpcError(RuntimeError):
@@ -84,6 +85,9 @@ def _load():
         "hpc_decode_step_multi": (ctypes.c_int, [vp, i32, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32,
                                                  i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp,
                                                  vp]),
+        "hpc_decode_step_lse": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32,
+                                               vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp, vp]),
+        "hpc_merge_lse": (ctypes.c_int, [vp, vp, i32, ctypes.c_int64, i32, vp, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -436,6 +440,51 @@ def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile
         workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
         _stream(dev)), "hpc_decode_step_multi")
     return out, status, workspace
+
+
+def decode_step_lse(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",
+                    kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None, lse=None,
+                    status=None, workspace=None):
+    """``hpc_decode_step_lse``: the single-launch step, plus the natural-log log-sum-exp of
+    every output row. Returns (out fp32 [B, Hq, D], lse fp32 [B, Hq], status, workspace)."""
+    _need(q, "q", torch.bfloat16)
+    dev = q.device
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    code = _kv_code(kv_dtype, k_pages)
+    B, Hq, D = q.shape
+    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
+    if num_ctas is None:
+        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
+    _need(lse, "lse", torch.float32, dev)
+    status = new_status(dev) if status is None else status
+    if workspace is None:
+        workspace = step_workspace(B, Hq, Hkv, D, num_ctas, dev)
+    scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    _check(_lib.hpc_decode_step_lse(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
+        workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(lse), _ptr(status),
+        _stream(dev)), "hpc_decode_step_lse")
+    return out, lse, status, workspace
+
+
+def merge_lse(outs, lses, out=None, lse_out=None):
+    """``hpc_merge_lse``: outs fp32 [parts, rows..., D], lses fp32 [parts, rows...] -> (out, lse)."""
+    _need(outs, "outs", torch.float32)
+    dev = outs.device
+    _need(lses, "lses", torch.float32, dev)
+    parts, D = outs.shape[0], outs.shape[-1]
+    rows = lses[0].numel()
+    if outs[0].numel() != rows * D:
+        raise HpcError("outs and lses disagree on the rows")
+    out = torch.empty(outs.shape[1:], dtype=torch.float32, device=dev) if out is None else out
+    lse_out = torch.empty(lses.shape[1:], dtype=torch.float32, device=dev) if lse_out is None else lse_out
+    _check(_lib.hpc_merge_lse(_ptr(outs), _ptr(lses), parts, rows, D, _ptr(out), _ptr(lse_out), _stream(dev)),
+           "hpc_merge_lse")
+    return out, lse_out
 
 
 def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",

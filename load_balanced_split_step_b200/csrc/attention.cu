@@ -702,6 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t oi = ((static_cast<int64_t>(x.req) * q_len + tq) * p.num_heads + head0 + h) * D + d;
         if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
         else reinterpret_cast<float*>(p.out)[oi] = val;
+        if (!MULTI && p.lse && d == 0)  // log-sum-exp in natural-log units (M is in log2 units)
+          p.lse[static_cast<int64_t>(x.req) * p.num_heads + head0 + h] = Ls > 0.f ? M * kLn2 + logf(Ls) : -INFINITY;
       } else {
         const int64_t pi = (x.slot * q_len + tq) * p.group + h;
         p.partial_o[pi * D + d] = acc;
@@ -1038,8 +1040,9 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
               int32_t kv_heads, int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
               const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas, float sm_scale,
               void* workspace, size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
-              void* stream, const PrologueArgs* pro, int32_t q_len = 1) {
+              void* stream, const PrologueArgs* pro, int32_t q_len = 1, float* lse = nullptr) {
   if (!workspace) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (lse && (q_len != 1 || pro)) return fail(HPC_ERR_ARG, "the log-sum-exp output is for the one-token step");
   if (q_len < 1 || q_len > 4) return fail(HPC_ERR_SHAPE, "q_len must be 1 to 4");
   if (pro && q_len != 1) return fail(HPC_ERR_SHAPE, "the folded prologue takes one new token per request");
   if (batch < 1) return fail(HPC_ERR_ARG, "batch must be >= 1");
@@ -1066,6 +1069,7 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.partial_o = reinterpret_cast<float*>(ws + L.partial_o);
   prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
   prm.batch = batch;
+  prm.lse = lse;
   if (!pro && q_len > 1)
     return dispatch<true, false, true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
                                        static_cast<cudaStream_t>(stream));
@@ -1095,6 +1099,19 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
   return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
                    workspace, workspace_bytes, out, out_dtype, status, stream, nullptr);
+}
+
+extern "C" int hpc_decode_step_lse(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                                   hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale,
+                                   int32_t num_pages, int32_t page_size, int32_t num_heads, int32_t kv_heads,
+                                   int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
+                                   const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
+                                   float sm_scale, void* workspace, size_t workspace_bytes, void* out,
+                                   hpc_dtype out_dtype, float* lse, uint32_t* status, void* stream) {
+  if (!lse) return fail(HPC_ERR_ARG, "null pointer argument");
+  return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
+                   workspace, workspace_bytes, out, out_dtype, status, stream, nullptr, 1, lse);
 }
 
 extern "C" size_t hpc_decode_step_multi_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_heads,

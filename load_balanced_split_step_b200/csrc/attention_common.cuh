@@ -38,6 +38,7 @@ struct AttnParams {
   uint32_t plane_bytes, stage_bytes;
   float score_scale;  // sm_scale * log2(e)
   int32_t q_len;      // new tokens per request (single-launch step); 1 elsewhere
+  float* lse;         // optional [batch][num_heads]: natural log of sum_j exp(score_j) (one-token step)
   int32_t nhd;        // cache layout: token stride Hkv*D (NHD) or D (HND); only the TMA coordinates differ
   // single-launch step only: the plan is derived in the kernel from seq_lens
   int32_t batch, kv_heads, max_seq_len;
@@ -277,6 +278,8 @@ __device__ void zero_empty_requests(const AttnParams& p, int tid, int nthr) {
     if (len_ok(L, p.max_seq_len, p.q_len) && L > 0) continue;
     const int64_t rows = static_cast<int64_t>(p.q_len) * p.num_heads * D;
     const int64_t base = static_cast<int64_t>(r) * rows;
+    if (p.lse)
+      for (int h = tid; h < p.num_heads; h += nthr) p.lse[static_cast<int64_t>(r) * p.num_heads + h] = -INFINITY;
     for (int64_t i = tid; i < rows; i += nthr) {
       if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[base + i] = __float2bfloat16_rn(0.f);
       else reinterpret_cast<float*>(p.out)[base + i] = 0.f;
@@ -322,6 +325,9 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
       for (int i = 0; i < n; ++i) L += expf(s_m[i * grp + tid] - M) * s_w[i * grp + tid];
       s_M[tid] = M;
       s_iL[tid] = L > 0.f ? 1.f / L : 0.f;
+      if (p.lse) {  // one new token per request: row tid is head kvh * group + tid
+        p.lse[static_cast<int64_t>(x.req) * p.num_heads + x.kvh * p.group + tid] = L > 0.f ? M + logf(L) : -INFINITY;
+      }
     }
     named_barrier_sync(1, nthr);
     for (int k = tid; k < n * grp; k += nthr) {
@@ -361,6 +367,8 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
     const float val = Ls > 0.f ? acc / Ls : 0.f;
     if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[out_at(idx)] = __float2bfloat16_rn(val);
     else reinterpret_cast<float*>(p.out)[out_at(idx)] = val;
+    if (p.lse && idx - h * D == 0)
+      p.lse[static_cast<int64_t>(x.req) * p.num_heads + x.kvh * p.group + h] = Ls > 0.f ? M + logf(Ls) : -INFINITY;
   }
 }
 

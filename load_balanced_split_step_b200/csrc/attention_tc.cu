@@ -549,6 +549,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int64_t oi = (static_cast<int64_t>(x.req) * p.num_heads + head0 + h) * kTcD + i;
             if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
             else reinterpret_cast<float*>(p.out)[oi] = val;
+            if (p.lse && i == 0)  // natural-log units; l carries 2^8
+              p.lse[static_cast<int64_t>(x.req) * p.num_heads + head0 + h] =
+                  Lh > 0.f ? M * kLn2 + logf(Lh * (1.f / 256.f)) : -INFINITY;
           } else {
             // partial state in natural-log units, without the 2^8 that p carries
             const int64_t pi = x.slot * p.group + h;

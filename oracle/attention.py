@@ -163,3 +163,39 @@ def decode_attention_multi(q, k_pages, v_pages, block_table, seq_lens, sm_scale=
                     p = p / p.sum()
                     out[r, t, h] = p @ V[:n]
     return out
+
+
+def decode_lse(q, k_pages, v_pages, block_table, seq_lens, sm_scale=None, kv_dtype="bf16", k_scale=None,
+               requests=None):
+    """Log-sum-exp of each request and query head's scores, in natural log:
+
+        lse[r, h] = log sum_{j < L_r} exp(sm_scale * q[r,h] . k_j)    (-inf when L_r = 0),
+
+    the weight that combines outputs computed over disjoint parts of the keys: with parts i,
+    LSE = log sum_i exp(lse_i) and out = sum_i exp(lse_i - LSE) out_i. Returns float64 [B, Hq].
+    """
+    qf = to_f64(q)
+    B, Hq, D = qf.shape
+    if kv_dtype == "e4m3":
+        kp = np.asarray(k_pages.cpu().numpy() if isinstance(k_pages, torch.Tensor) else k_pages, dtype=np.uint8)
+        ks = to_f64(k_scale)
+    else:
+        kp, ks = k_pages, None
+    Hkv = kp.shape[1]
+    grp = Hq // Hkv
+    bt = np.asarray(block_table.cpu().numpy() if isinstance(block_table, torch.Tensor) else block_table, dtype=np.int64)
+    lens = np.asarray(seq_lens.cpu().numpy() if isinstance(seq_lens, torch.Tensor) else seq_lens, dtype=np.int64)
+    scale = (1.0 / math.sqrt(D)) if sm_scale is None else float(sm_scale)
+    out = np.full((B, Hq), -np.inf)
+    for r in (range(B) if requests is None else requests):
+        L = int(lens[r])
+        if L == 0:
+            continue
+        for g in range(Hkv):
+            K = _kv_values(kp, kv_dtype, ks, bt, r, g, L) if kv_dtype == "e4m3" else \
+                to_f64(_torch_gather(kp, bt, r, g, L))
+            for h in range(g * grp, (g + 1) * grp):
+                s = scale * (K @ qf[r, h])
+                m = s.max()
+                out[r, h] = m + math.log(np.exp(s - m).sum())
+    return out

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ("hpc_decode_plan", "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue",
               "hpc_plan_cpu", "hpc_decode_plan_static", "hpc_decode_step", "hpc_decode_step_prologue",
-              "hpc_decode_step_multi"):
+              "hpc_decode_step_multi", "hpc_decode_step_lse", "hpc_merge_lse"):
         assert n in names
 
 
@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 4
+    assert B._lib.hpc_abi_version() == 5
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -75,6 +75,13 @@ def test_host_argument_errors_return_codes(B):
     assert B._lib.hpc_decode_step_multi_workspace_bytes(4, 0, 8, 2, 64, 148) == 0
     assert (B._lib.hpc_decode_step_multi_workspace_bytes(4, 1, 8, 2, 64, 148)
             == B._lib.hpc_decode_step_workspace_bytes(4, 8, 2, 64, 148))
+    # log-sum-exp step and merge: null outputs, bad sizes
+    rc = B._lib.hpc_decode_step_lse(w, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1, 32, 4, 0.1, w, 1 << 20, w,
+                                    1, None, w, None)
+    assert rc == B.HPC_ERR_ARG
+    assert B._lib.hpc_merge_lse(None, None, 2, 10, 64, None, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_merge_lse(w, w, 0, 10, 64, w, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_merge_lse(w, w, 2, 0, 64, w, None, None) == B.HPC_OK  # nothing to do
     # bad tile_len on the host planner
     lens = torch.tensor([5, 7], dtype=torch.int32)
     with pytest.raises(B.HpcError, match="tile_len"):

@@ -1,0 +1,91 @@
+"""Log-sum-exp output, the log-sum-exp merge and request-sharded placement, through the
+C ABI on one GPU.
+
+* hpc_decode_step_lse writes the same output as hpc_decode_step, and lse matches the fp64
+  oracle's log-sum-exp.
+* hpc_merge_lse equals its definition (float64 torch) on random parts, -inf parts included.
+* A batch sharded over 2, 3 and 4 ranks gives the unsharded oracle result. The ranks run
+  one after another in this process: each computes its parts, their (out, lse) are stacked
+  as the all-gather would stack them, and split requests are merged. No kernel waits on
+  another rank.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from load_balanced_split_step_b200 import shard as S
+from load_balanced_split_step_b200 import workloads as W
+from oracle import attention as OA
+from tests.helpers import assert_bf16_tol, errors, oracle_out, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from load_balanced_split_step_b200 import binding
+    return binding
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_lse_output(B, kv):
+    spec = W.custom_spec((0, 1, 17, 300, 1000, 4097), 32, 4, 128, 64, 128, kv_dtype=kv, seed=31)
+    case = W.make_case(spec)
+    dc = to_device(case)
+    kw = dict(kv_dtype=kv, k_scale=dc["k_scale"], v_scale=dc["v_scale"], num_ctas=37)
+    out, lse, st, _ = B.decode_step_lse(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"], dc["seq_lens"], 32,
+                                        4, 128, **kw)
+    ref_out, _, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"], dc["seq_lens"], 32,
+                                        4, 128, **kw)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(out, ref_out)
+    ref = OA.decode_lse(case.q, case.k_pages, case.v_pages, case.block_table, case.seq_lens, kv_dtype=kv,
+                        k_scale=case.k_scale)
+    got = lse.cpu().numpy().astype(np.float64)
+    assert np.all(np.isneginf(got[0])) and np.all(np.isneginf(ref[0]))
+    assert np.max(np.abs(got[1:] - ref[1:])) <= 1e-4
+
+
+def test_merge_lse_definition(B):
+    g = torch.Generator().manual_seed(5)
+    parts, rows, D = 5, 70, 128
+    outs = torch.randn(parts, rows, D, generator=g)
+    lses = torch.randn(parts, rows, generator=g) * 4
+    lses[1, :10] = -math.inf
+    lses[:, 20] = -math.inf  # a row with no keys at all
+    o, l = B.merge_lse(outs.cuda(), lses.cuda())
+    torch.cuda.synchronize()
+    ld = lses.double()
+    M = ld.max(0).values
+    Mf = torch.where(torch.isinf(M), torch.zeros_like(M), M)
+    w = torch.exp(ld - Mf)
+    L = Mf + torch.log(w.sum(0))
+    ref = (torch.exp(ld - L)[..., None] * outs.double()).sum(0)
+    ref[20] = 0.0
+    assert torch.max(torch.abs(o.cpu().double() - ref)).item() <= 1e-5
+    lc = l.cpu().double()
+    assert torch.isneginf(lc[20]) and torch.max(torch.abs(lc[:20] - L[:20])).item() <= 1e-5
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_sharded_batch_equals_unsharded(B, world, kv):
+    spec = W.custom_spec((9000, 64, 5, 130, 2047, 700), 32, 4, 128, 64, 128, kv_dtype=kv, seed=40 + world)
+    case = W.make_case(spec)
+    dc = to_device(case)
+    compute = S.library_compute(32, 4, kv_dtype=kv, k_scale=dc["k_scale"], v_scale=dc["v_scale"], num_ctas=37)
+    steps = [S.ShardedStep(spec.seq_lens, world, r, spec.page_size, 32, 128, compute=compute) for r in range(world)]
+    assert sum(len(p) for p in steps[0].plan) > len(spec.seq_lens)  # the 9000-token request is split
+    local = [st.local(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"], spec.tile_len) for st in steps]
+    outs = torch.stack([o for o, _ in local])  # what the all-gather delivers to every rank
+    lses = torch.stack([l for _, l in local])
+    out = steps[0].assemble(outs, lses)
+    torch.cuda.synchronize()
+    ref = oracle_out(case)
+    if kv == "bf16":
+        assert_bf16_tol(out, ref, what=f"sharded over {world}")
+    else:
+        assert errors(out, ref)[0] <= 5e-2
