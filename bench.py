@@ -59,6 +59,8 @@ def parse_args(argv=None):
                     help="fused: one launch per step (in-kernel plan + ticket merge), after the prologue kernel on "
                          "the FP8 workload; folded: the same with the prologue folded into that launch; split: "
                          "plan, attention and merge kernels")
+    ap.add_argument("--requests", type=int, default=0,
+                    help="run only the first N requests of the workload (a bounded sample, e.g. for a profiler)")
     ap.add_argument("--q-len", type=int, default=1,
                     help="new tokens per request, attending causally (1 to 4; single-launch path)")
     ap.add_argument("--shard", action="store_true",
@@ -485,13 +487,18 @@ def cpu_baseline(spec, case, target_s):
 
 
 def qlen_text(args):
-    return "" if args.q_len == 1 else f"; {args.q_len} new tokens per request, causal among themselves"
+    t = "" if args.q_len == 1 else f"; {args.q_len} new tokens per request, causal among themselves"
+    return t + (f"; first {args.requests} requests only" if args.requests else "")
 
 
 def workload_spec(args):
-    """The named workload, with q_len new tokens per request when --q-len > 1."""
+    """The named workload, with q_len new tokens per request when --q-len > 1, and only its
+    first --requests requests when that is set."""
     from dataclasses import replace
     spec = W.config_spec(args.workload)
+    if args.requests and args.requests < spec.batch:
+        spec = replace(spec, seq_lens=tuple(spec.seq_lens[:args.requests]),
+                       name=f"{spec.name}, first {args.requests} requests")
     if args.q_len != 1:
         if spec.prologue:
             raise SystemExit("--q-len > 1 is not combined with the prologue workload")

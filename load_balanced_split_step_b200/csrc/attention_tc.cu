@@ -24,13 +24,15 @@
 //    same layout; Phl is MN-major without swizzle, 16 bytes per token.
 //  * warps 0-7, softmax: two warpgroups take alternate stages, each with its own running state
 //    for the item, combined by log-sum-exp at the item end. In a warpgroup, thread i owns token
-//    row i of S^T and d row i of O^T. Per stage they
-//    read S, take the row max of each head across the 128 tokens (a reduce-scatter over the
-//    warp, then shared memory), write Phl for p = 2^(s - m + 8) (the 2^8 keeps the E4M3 codes
-//    of p away from underflow; p <= 256 < 448), and fold the previous stage's O^T into
-//    registers with the running-max correction. O is never rescaled in tensor memory.
-// Each stage of an item is a separate product with its own output buffer, so the softmax of
-// stage n overlaps the products of stage n + 1. Tensor memory: 64 columns (S[2], O[2]).
+//    row i of S^T and d row i of O^T. Per stage a warpgroup reads S, takes the row max of each
+//    head across the 128 tokens (a reduce-scatter over the warp, then shared memory), folds its
+//    previous stage's O^T into registers with the running-max correction, and writes Phl for
+//    p = 2^(s - m + 8) (the 2^8 keeps the E4M3 codes of p away from underflow; p <= 256 < 448).
+//    O is never rescaled in tensor memory.
+// Each stage is a separate pair of products with its own buffers (two of each), so the softmax
+// of one stage overlaps the products of the next. Tensor memory: 64 columns (S[2], O[2]).
+// Measured, this kernel is slower than the mma.sync one for one new token per request (each
+// stage chains two product round trips through mbarriers, with N = 16), so it is opt-in.
 // Every wait is bounded (2 s) and ends in HPC_DEV_TIMEOUT; tensor memory is freed on every
 // path.
 #include "attention_common.cuh"
