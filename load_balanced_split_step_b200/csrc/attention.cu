@@ -921,6 +921,8 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   const int tl = tile_len;
   if (tl < 16 || tl % 16 || !(tl % page_size == 0 || page_size % tl == 0))
     return fail(HPC_ERR_SHAPE, "tile_len %d must be a multiple of 16 and of page_size %d, or divide it", tl, page_size);
+  if (static_cast<int64_t>(max_pages_per_req) * page_size > INT32_MAX)
+    return fail(HPC_ERR_SHAPE, "max_pages_per_req * page_size must fit in int32");
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out))
     return fail(HPC_ERR_ALIGN, "q, caches and out must be 16-byte aligned");
 
@@ -955,7 +957,7 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
   prm->stage_bytes = ls->stage_bytes;
   prm->score_scale = sm_scale * kLog2e;
   prm->kv_heads = kv_heads;
-  prm->max_seq_len = max_pages_per_req * page_size;
+  prm->max_seq_len = max_pages_per_req * page_size;  // checked above to fit int32
   prm->nhd = nhd ? 1 : 0;
   prm->q_len = q_len;
   return HPC_OK;

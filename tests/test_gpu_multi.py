@@ -106,3 +106,20 @@ def test_heavy_tailed_four_tokens_full_size(B):
     assert_bf16_tol(out[rows], ref, what="heavy-tailed, 4 new tokens")
     again, _, _ = _run(B, spec, dc, 148)
     assert torch.equal(out, again)  # run to run: bit-identical
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_nhd_layout_is_bit_identical(B, kv):
+    """Several new tokens on the vLLM page layout: the same TMA boxes land in shared memory,
+    so the output equals the HND run bit for bit."""
+    spec = W.custom_spec((3, 40, 300, 2049), 32, 8, 128, 64, 128, kv_dtype=kv, seed=97, q_len=3)
+    case = W.make_case(spec)
+    dc = to_device(case)
+    hnd, st1, _ = _run(B, spec, dc, 37)
+    nhd = dict(dc)
+    nhd["k_pages"] = dc["k_pages"].permute(0, 2, 1, 3).contiguous()
+    nhd["v_pages"] = dc["v_pages"].permute(0, 2, 1, 3).contiguous()
+    got, st2, _ = _run(B, spec, nhd, 37, kv_layout="NHD")
+    assert st1 == 0 and st2 == 0
+    assert torch.equal(got, hnd)
+    _check(got, _oracle(case), kv, f"NHD q_len 3 {kv}")
