@@ -315,6 +315,41 @@ def time_steps(step, lens, K, W_, world, kernel_events=True):
     return total_ms, kern_ms
 
 
+def step_distribution(step, lens, n, world):
+    """Distribution of single-step times: CUDA events around each whole step on the launching
+    stream, after three untimed steps. The events between steps stop one step's launch from
+    overlapping the previous one's tail, so the median sits slightly above the back-to-back mean.
+    A workload of several decode steps (lengths growing by one) also gets each step's mean."""
+    for i in range(3):
+        step(lens[i % len(lens)])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        ev[i][0].record()
+        step(lens[i % len(lens)])
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    us = np.array([1000.0 * a.elapsed_time(b) for a, b in ev])
+    p10, p50, p90 = (max_over_ranks(float(np.percentile(us, q)), world) for q in (10, 50, 90))
+    out = {"reps": n, "median_us": round(p50, 2), "p10_us": round(p10, 2), "p90_us": round(p90, 2),
+           "note": "events around every step (max over ranks)"}
+    if len(lens) > 1:
+        out["per_step_mean_us"] = [round(max_over_ranks(float(us[i::len(lens)].mean()), world), 2)
+                                   for i in range(len(lens))]
+    return out
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def static_leg(B, spec, dc, tl, steps, sms, layout="HND"):
     S0 = max(1, -(-2 * sms // (spec.batch * spec.kv_heads)))
     res = {}
@@ -614,6 +649,7 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         extra["graph_us_per_step"] = round(1000.0 * a.elapsed_time(b) / K, 2)
         del g
+        extra["step_time_distribution"] = step_distribution(step, lens, max(50, 8 * len(lens)), world)
         if spec.q_len == 1:  # the static plan drives the three-launch path, which takes one new token
             extra["static_split_k"] = static_leg(B, spec, dc, tl, max(50, K // 10), sms, args.layout)
             extra["speedup_vs_static_split_k"] = round(extra["static_split_k"]["us_per_step"] / (1000 * ms_step),
@@ -630,7 +666,8 @@ def run_ours(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
         v, desc, threads, _ = cpu_baseline(spec, case, args.cpu_seconds)
-        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "cpu_model": cpu_model(), "host_cores": os.cpu_count()}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W_,
@@ -690,7 +727,7 @@ def run_reference(args, rank, world):
                    "plan": "none (exact)",
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": descs[0]},
+                         "sample": descs[0], "cpu_model": cpu_model(), "host_cores": os.cpu_count()},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 5
+#define HPC_DECODE_ABI_VERSION 6
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -377,6 +377,20 @@ HPC_API int hpc_decode_step_noalloc(const void* q, const void* k_pages, const vo
 HPC_API int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, int32_t page_size, int32_t tile_len,
                               int32_t ctas_per_sm, int32_t* stages, int32_t* smem_bytes,
                               int32_t* threads);
+
+/* Diagnostic of the bounded pipeline waits. Every wait in the library's kernels (stage
+ * barriers, the new-token barrier, the final drain) gives up after a time limit, ORs
+ * HPC_DEV_TIMEOUT into the status word and lets the kernel return; the library never
+ * traps. This call runs that same wait in a one-warp kernel on a shared-memory barrier
+ * phase:
+ *   arrive != 0  the phase completes before the wait, which returns at once;
+ *   arrive == 0  nothing completes it; the wait gives up after limit_ns and
+ *                HPC_DEV_TIMEOUT is OR-ed into *status.
+ * limit_ns: 1 .. 2e9 (the kernels' own limit is 2 s), else HPC_ERR_ARG.
+ * status: device uint32 word (required). waited_ns: device uint64 (8-byte aligned) that
+ * receives the wait's duration from %globaltimer, or NULL. Asynchronous on stream. */
+HPC_API int hpc_wait_selftest(uint64_t limit_ns, int32_t arrive, uint32_t* status, uint64_t* waited_ns,
+                              void* stream);
 
 HPC_API const char* hpc_status_string(int status);
 HPC_API const char* hpc_last_error(void); /* message of the calling thread's last failure ("" if none) */

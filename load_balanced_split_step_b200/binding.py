@@ -31,7 +31,7 @@ EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_d
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
            "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue",
            "hpc_decode_step_multi", "hpc_decode_step_multi_workspace_bytes", "hpc_decode_step_lse",
-           "hpc_merge_lse")
+           "hpc_merge_lse", "hpc_wait_selftest")
 
 
 class HpcError(RuntimeError):
@@ -88,6 +88,7 @@ def _load():
         "hpc_decode_step_lse": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32,
                                                vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp, vp]),
         "hpc_merge_lse": (ctypes.c_int, [vp, vp, i32, ctypes.c_int64, i32, vp, vp, vp]),
+        "hpc_wait_selftest": (ctypes.c_int, [ctypes.c_uint64, i32, vp, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -485,6 +486,17 @@ def merge_lse(outs, lses, out=None, lse_out=None):
     _check(_lib.hpc_merge_lse(_ptr(outs), _ptr(lses), parts, rows, D, _ptr(out), _ptr(lse_out), _stream(dev)),
            "hpc_merge_lse")
     return out, lse_out
+
+
+def wait_selftest(limit_ns: int, arrive: bool, device, status=None):
+    """``hpc_wait_selftest``: the library's bounded wait on a barrier phase that completes at once
+    (arrive) or never (not arrive). Returns (status word, waited ns), both device tensors."""
+    dev = torch.device(device)
+    status = new_status(dev) if status is None else status
+    waited = torch.zeros(1, dtype=torch.int64, device=dev)
+    _check(_lib.hpc_wait_selftest(int(limit_ns), 1 if arrive else 0, _ptr(status), _ptr(waited), _stream(dev)),
+           "hpc_wait_selftest")
+    return status, waited
 
 
 def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 5
+    assert B._lib.hpc_abi_version() == 6
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -82,6 +82,11 @@ def test_host_argument_errors_return_codes(B):
     assert B._lib.hpc_merge_lse(None, None, 2, 10, 64, None, None, None) == B.HPC_ERR_ARG
     assert B._lib.hpc_merge_lse(w, w, 0, 10, 64, w, None, None) == B.HPC_ERR_ARG
     assert B._lib.hpc_merge_lse(w, w, 2, 0, 64, w, None, None) == B.HPC_OK  # nothing to do
+    # wait diagnostic: null status, limit outside 1 .. 2 s
+    assert B._lib.hpc_wait_selftest(1000, 0, None, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_wait_selftest(0, 0, w, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_wait_selftest(3_000_000_000, 0, w, None, None) == B.HPC_ERR_ARG
+    assert "limit_ns" in B._lib.hpc_last_error().decode()
     # bad tile_len on the host planner
     lens = torch.tensor([5, 7], dtype=torch.int32)
     with pytest.raises(B.HpcError, match="tile_len"):
