@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using S = Shape<D, FP8>;
   using Cursor = typename CursorOf<FUSED>::type;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int64_t s_scan[16], s_walk[8];
+  __shared__ int64_t s_scan[16], s_walk[9];
   __shared__ int s_flag;
   __shared__ int32_t s_pages[32];
   // folded prologue: q_norm_w, theta^(-2i/D), two rotation tables [cos | sin], new-token barrier
@@ -719,7 +719,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __threadfence();
         named_barrier_sync(1, cthreads);
         if (ctid == 0) {
-          const int64_t pieces = (x.U + x.nt - 1) / chunk - x.U / chunk + 1;
+          int64_t g1, g2, first_slot;
+          segment_ctas(x, p.item_cost, chunk, g1, g2, first_slot);
+          const int64_t pieces = g2 - g1 + 1;
           int32_t* ticket = p.tickets + static_cast<int64_t>(x.req) * p.kv_heads + kvh;
           const int old = atomicAdd(ticket, 1);
           const int last = old == pieces - 1;
@@ -1037,6 +1039,28 @@ struct PrologueArgs {
 
 // Single-launch step; with `pro`, q is formed from qkv in the kernel and the new token's K/V
 // are written into the cache first.
+// Fixed cost of starting an item in the single-launch step's split, in 1/kCostPerTile of a
+// tile. At an item end the consumers combine their states, write the output or a partial
+// state, take the merge ticket (and merge), and load the next item's q; the ring keeps
+// streaming, but only a few stages beyond what covers the memory latency. Per-CTA
+// %globaltimer stamps on B200 put that cost near the time a CTA takes to stream 152 KB of KV
+// at its share of HBM (one new token), and 224 KB with several new tokens, where the
+// consumers are the bound. A CTA that starts many items (many short requests) therefore gets
+// fewer tiles. HPC_ITEM_COST (integer, 1/16 tile) overrides it; 0 splits by tiles alone, the
+// pages' rule.
+int item_cost_units(int head_dim, bool fp8, int tile_len, int q_len) {
+  constexpr int64_t kMax = 64 * kCostPerTile;
+  const char* e = getenv("HPC_ITEM_COST");
+  if (e && *e) {
+    const long v = strtol(e, nullptr, 10);
+    return static_cast<int>(v < 0 ? 0 : (v > kMax ? kMax : v));
+  }
+  const int64_t tile_bytes = static_cast<int64_t>(tile_len) * head_dim * 2 * (fp8 ? 1 : 2);
+  const int64_t item_bytes = (q_len > 1 ? 224 : 152) * 1024;
+  const int64_t c = (kCostPerTile * item_bytes + tile_bytes / 2) / tile_bytes;
+  return static_cast<int>(c > kMax ? kMax : c);
+}
+
 int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype, hpc_kv_layout kv_layout,
               const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads,
               int32_t kv_heads, int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
@@ -1072,6 +1096,7 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
   prm.batch = batch;
   prm.lse = lse;
+  prm.item_cost = item_cost_units(head_dim, kv_dtype == HPC_E4M3, tile_len, q_len);
   if (!pro && q_len > 1)
     return dispatch<true, false, true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
                                        static_cast<cudaStream_t>(stream));

@@ -19,6 +19,11 @@ constexpr int kMaxStages = 16;
 constexpr int kSmemLimit = 232448;  // 227 KB per block on sm_100
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Single-launch step: cost units per tile in the planner's split (item_cost is in the same units)
+constexpr int64_t kCostPerTile = 16;
+// The request prefix packs two sums: valid requests (nt > 0) above bit 44, tiles below it.
+constexpr int kPreShift = 44;
+constexpr int64_t kPreTiles = (int64_t(1) << kPreShift) - 1;
 
 struct AttnParams {
   const __nv_bfloat16* q;
@@ -43,6 +48,7 @@ struct AttnParams {
   // single-launch step only: the plan is derived in the kernel from seq_lens
   int32_t batch, kv_heads, max_seq_len;
   int32_t* tickets;  // [batch * kv_heads], zero between steps
+  int32_t item_cost;  // cost of starting an item, in 1/kCostPerTile of a tile (0: split by tiles alone)
   // single-launch step with the prologue folded in: q comes from qkv through RMSNorm and RoPE,
   // and the new token's K/V are written into the cache
   const __nv_bfloat16* qkv;  // [batch][num_heads + 2 kv_heads][D]
@@ -60,8 +66,9 @@ struct ItemInfo {
   int64_t tok0, tok1;  // tokens to stream
   bool direct;         // covers its whole (request, kv head): writes the output itself
   int64_t slot;        // partial-state slot of a split item
-  int64_t U;           // single-launch step: first unit of the (request, kv head) segment
-  int32_t nt;          // and its tile count
+  int64_t U;           // single-launch step: first unit of the (request, kv head) segment,
+  int32_t nt;          // its tile count
+  int64_t S;           // and its 1-based index among the segments that have tiles
 };
 
 // 16-token blocks that one consumer warp takes from a stage of `bpc` blocks. Two blocks give
@@ -127,6 +134,7 @@ struct PlanCursor {
     x.slot = it;
     x.U = 0;
     x.nt = 0;
+    x.S = 0;
     ++it;
     return true;
   }
@@ -136,9 +144,9 @@ struct PlanCursor {
 // [u, u_end) of the request -> kv head -> tile enumeration and cuts them at (request, kv head)
 // boundaries. A split (request, kv head) is always this CTA's first or last item, so two
 // partial slots per CTA suffice: 2g for a piece that starts at the CTA's first unit, 2g + 1
-// otherwise.
+// otherwise. V counts the requests with tiles before r, which numbers the segments.
 struct WalkCursor {
-  int64_t u, u_end, u_first, U_r;
+  int64_t u, u_end, u_first, U_r, V;
   int32_t r, kvh, nt, tb, g;
   __device__ bool next(const AttnParams& p, ItemInfo& x) {
     if (u >= u_end) return false;
@@ -154,11 +162,13 @@ struct WalkCursor {
     x.slot = 2 * static_cast<int64_t>(g) + (u == u_first ? 0 : 1);
     x.U = U_r + static_cast<int64_t>(kvh) * nt;
     x.nt = nt;
+    x.S = V * p.kv_heads + kvh + 1;
     u += te - tb;
     tb = 0;
     if (u < u_end) {  // step to the next (request, kv head) with tiles
       if (++kvh == p.kv_heads) {
         kvh = 0;
+        ++V;
         U_r += static_cast<int64_t>(p.kv_heads) * nt;
         do {
           ++r;
@@ -180,10 +190,33 @@ struct CursorOf<true> {
   using type = WalkCursor;
 };
 
-// Single-launch step: each CTA finds where its unit range starts. It forms the exclusive
-// prefix sum of per-request tile counts in shared memory (the reduce buffer, unused until
-// the first item ends) and binary-searches it. Requests with no valid tiles get a zero
-// output from CTA r % num_ctas. Returns the walk cursor (all threads get the same one).
+// Where the single-launch step's split puts a unit. Unit u (tile t of segment S, the S-th
+// (request, kv head) with tiles, 1-based) sits at cost position W*u + c*S: every tile costs
+// W = kCostPerTile and every segment start adds c = item_cost, the fixed cost of an item
+// (its combine, partial write, ticket and merge, and the next item's first loads). CTA g owns
+// the units whose positions fall in [g*chunk, (g+1)*chunk), chunk = W * ceil(total / (W*G)).
+// With c = 0 this is the pages' rule: chunk / W = ceil(T / G) units per CTA.
+__device__ __forceinline__ int64_t unit_pos(int64_t u, int64_t S, int64_t c) { return kCostPerTile * u + c * S; }
+
+// CTAs that own the first and the last tile of an item's segment, and the partial slot of the
+// segment's first piece (2 g1 when the segment starts CTA g1's range, 2 g1 + 1 otherwise).
+// Every CTA between g1 and g2 owns at least one tile of the segment (chunk >= W), so the
+// segment has g2 - g1 + 1 pieces, and the piece in CTA g1 + i (i >= 1) is in slot 2 (g1 + i).
+__device__ __forceinline__ void segment_ctas(const ItemInfo& x, int64_t c, int64_t chunk, int64_t& g1, int64_t& g2,
+                                             int64_t& first_slot) {
+  const int64_t p_first = unit_pos(x.U, x.S, c);
+  g1 = p_first / chunk;
+  g2 = (p_first + kCostPerTile * (x.nt - 1)) / chunk;
+  // the unit before the segment is the last tile of segment S - 1
+  const bool starts_cta = x.U == 0 || unit_pos(x.U - 1, x.S - 1, c) / chunk != g1;
+  first_slot = starts_cta ? 2 * g1 : 2 * g1 + 1;
+}
+
+// Single-launch step: each CTA finds its unit range. It forms the exclusive prefix sums of
+// per-request tile counts and of requests with tiles (packed in one int64, kPreShift) in
+// shared memory (the reduce buffer, unused until the first item ends) and binary-searches
+// them. Requests with no valid tiles get a zero output from CTA r % num_ctas. Returns the
+// walk cursor (all threads get the same one) and the split's chunk in cost units.
 template <int D>
 __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_scan, int64_t* s_walk,
                                WalkCursor& cur, int64_t& chunk) {
@@ -198,7 +231,8 @@ __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_s
     const int32_t L = p.seq_lens[r];
     const bool ok = len_ok(L, p.max_seq_len, p.q_len);
     if (!ok) bad |= HPC_DEV_BAD_SEQLEN;
-    run += ok ? tiles_of(L, p.tile_len) : 0;
+    const int32_t nt = ok ? tiles_of(L, p.tile_len) : 0;
+    run += nt > 0 ? (int64_t(1) << kPreShift) + nt : 0;
   }
   if (bad && (r0 % G) == g) atomicOr(p.status, bad);
   const int lane = tid & 31, warp = tid >> 5, nwarps = (nthr + 31) >> 5;
@@ -224,27 +258,49 @@ __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_s
   for (int r = r0; r < r1; ++r) {
     s_pre[r] = pre;
     const int32_t L = p.seq_lens[r];
-    pre += len_ok(L, p.max_seq_len, p.q_len) ? tiles_of(L, p.tile_len) : 0;
+    const int32_t nt = len_ok(L, p.max_seq_len, p.q_len) ? tiles_of(L, p.tile_len) : 0;
+    pre += nt > 0 ? (int64_t(1) << kPreShift) + nt : 0;
   }
   if (tid == 0) s_pre[B] = s_scan[nwarps];
   __syncthreads();
   if (tid == 0) {
-    const int64_t T = s_pre[B] * Hkv;
-    const int64_t ch = T > 0 ? (T + G - 1) / G : 0;
-    const int64_t u0 = static_cast<int64_t>(g) * ch;
-    const int64_t u1 = min(u0 + ch, T);
-    int64_t r = 0, kvh = 0, tb = 0, nt = 0, U_r = 0;
-    if (u0 < T) {
-      // largest r with Hkv * s_pre[r] <= u0: the request that holds unit u0
+    auto tiles = [&](int i) -> int64_t { return s_pre[i] & kPreTiles; };
+    auto valid = [&](int i) -> int64_t { return s_pre[i] >> kPreShift; };
+    const int64_t c = p.item_cost, W = kCostPerTile;
+    const int64_t T = tiles(B) * Hkv;
+    const int64_t total = W * T + c * valid(B) * Hkv;
+    const int64_t ch = T > 0 ? W * ((total + W * G - 1) / (W * G)) : 0;
+    // first unit whose cost position is >= P (T if none)
+    auto first_unit_at = [&](int64_t P) -> int64_t {
+      if (T == 0 || P <= 0) return 0;
+      if (P > unit_pos(T - 1, valid(B) * Hkv, c)) return T;
+      // largest r whose cost prefix is <= P: the request whose segments hold position P
+      auto cost_pre = [&](int i) -> int64_t { return (W * tiles(i) + c * valid(i)) * Hkv; };
       int lo = 0, hi = B - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (s_pre[mid] * Hkv <= u0) lo = mid;
+        if (cost_pre(mid) <= P) lo = mid;
+        else hi = mid - 1;
+      }
+      const int64_t nt = tiles(lo + 1) - tiles(lo), seg = c + W * nt;
+      const int64_t off = P - cost_pre(lo), kv = off / seg, o = off - kv * seg;
+      const int64_t t = o <= c ? 0 : min(nt, (o - c + W - 1) / W);  // nt: the next segment's first unit
+      return tiles(lo) * Hkv + kv * nt + t;
+    };
+    const int64_t u0 = first_unit_at(static_cast<int64_t>(g) * ch);
+    const int64_t u1 = max(u0, first_unit_at(static_cast<int64_t>(g + 1) * ch));
+    int64_t r = 0, kvh = 0, tb = 0, nt = 0, U_r = 0;
+    if (u0 < T) {
+      // largest r with Hkv * tiles(r) <= u0: the request that holds unit u0
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tiles(mid) * Hkv <= u0) lo = mid;
         else hi = mid - 1;
       }
       r = lo;
-      nt = s_pre[r + 1] - s_pre[r];
-      U_r = s_pre[r] * Hkv;
+      nt = tiles(r + 1) - tiles(r);
+      U_r = tiles(r) * Hkv;
       kvh = (u0 - U_r) / nt;
       tb = u0 - U_r - kvh * nt;
     }
@@ -256,6 +312,7 @@ __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_s
     s_walk[5] = nt;
     s_walk[6] = tb;
     s_walk[7] = ch;
+    s_walk[8] = u0 < T ? valid(static_cast<int>(r)) : 0;
   }
   __syncthreads();
   cur.u = s_walk[0];
@@ -266,6 +323,7 @@ __device__ void plan_in_kernel(const AttnParams& p, int64_t* s_pre, int64_t* s_s
   cur.kvh = static_cast<int32_t>(s_walk[4]);
   cur.nt = static_cast<int32_t>(s_walk[5]);
   cur.tb = static_cast<int32_t>(s_walk[6]);
+  cur.V = s_walk[8];
   cur.g = g;
   chunk = s_walk[7];
 }
@@ -296,8 +354,8 @@ __device__ void zero_empty_requests(const AttnParams& p, int tid, int nthr) {
 template <int D>
 __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t chunk, int tid, int nthr,
                               float* s_buf, int buf_floats) {
-  const int64_t g1 = x.U / chunk, g2 = (x.U + x.nt - 1) / chunk;
-  const int64_t first_slot = (x.U > g1 * chunk) ? 2 * g1 + 1 : 2 * g1;
+  int64_t g1, g2, first_slot;
+  segment_ctas(x, p.item_cost, chunk, g1, g2, first_slot);
   // rows of a piece: query token t, head h -> row t * group + h
   const int grp = p.group * p.q_len;
   const int n = static_cast<int>(g2 - g1 + 1);

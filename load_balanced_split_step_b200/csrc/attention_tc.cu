@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                const AttnParams p) {
   using Cursor = typename CursorOf<FUSED>::type;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int64_t s_scan[16], s_walk[8];
+  __shared__ int64_t s_scan[16], s_walk[9];
   __shared__ int s_flag;
   __shared__ int32_t s_pages[32];
   __shared__ uint32_t s_tmem;
@@ -570,7 +570,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __threadfence();
             named_barrier_sync(1, kSoftmax);
             if (i == 0) {
-              const int64_t pieces = (x.U + x.nt - 1) / chunk - x.U / chunk + 1;
+              int64_t g1, g2, first_slot;
+              segment_ctas(x, p.item_cost, chunk, g1, g2, first_slot);
+              const int64_t pieces = g2 - g1 + 1;
               int32_t* ticket = p.tickets + static_cast<int64_t>(x.req) * p.kv_heads + kvh;
               const int old = atomicAdd(ticket, 1);
               const int last = old == pieces - 1;

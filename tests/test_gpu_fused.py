@@ -61,6 +61,25 @@ def test_shapes_ragged(B, Hq, Hkv, D, P, tl):
         assert _tickets_zero(ws, spec.batch, spec.kv_heads)
 
 
+@pytest.mark.parametrize("cost", ["0", "16", "200", "1024"])
+def test_item_cost_split(B, monkeypatch, cost):
+    """The split of the single-launch step with a fixed cost per item (HPC_ITEM_COST, in 1/16 of
+    a tile; 0 is the pages' split by tiles alone). Whatever the cost, every tile lands in
+    exactly one CTA, every split segment's piece count and partial slots agree (the merge
+    tickets end at zero) and the output equals the oracle, for CTA counts from 1 to 2 per SM."""
+    monkeypatch.setenv("HPC_ITEM_COST", cost)
+    lens = (1, 15, 16, 17, 63, 64, 65, 129, 300, 1000, 2049, 0, 5000)
+    spec = W.custom_spec(lens, 16, 4, 128, 64, 64, seed=61)
+    case = W.make_case(spec)
+    dc = to_device(case)
+    ref = oracle_out(case)
+    for G in (1, 3, 8, 37, 148, 296):
+        out, st, ws = _fused(B, spec, dc, num_ctas=G)
+        assert st == 0
+        assert_bf16_tol(out, ref, what=f"fused, item cost {cost}, G={G}")
+        assert _tickets_zero(ws, spec.batch, spec.kv_heads)
+
+
 def test_empty_and_invalid_requests(B):
     spec = W.custom_spec((0, 40, 5, 200), 8, 2, 64, 16, 32, seed=51)
     case = W.make_case(spec)
@@ -81,7 +100,9 @@ def test_empty_and_invalid_requests(B):
     assert torch.all(out2[2] == 0) and torch.isfinite(out2).all()
 
 
-def test_matches_three_launch_path_and_is_deterministic(B):
+def test_matches_three_launch_path_and_is_deterministic(B, monkeypatch):
+    # with no item cost the single launch splits the tiles exactly as the planner does
+    monkeypatch.setenv("HPC_ITEM_COST", "0")
     spec = W.custom_spec((5000, 40, 999, 131, 7777), 64, 8, 128, 64, 128, seed=52)
     case = W.make_case(spec)
     dc = to_device(case)
