@@ -204,7 +204,12 @@ HPC_API size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads,
  * SGLang …" (remio.ai), section "Tres señales …", lists megakernels; "vLLM × HPC-Ops"
  * describes PDL-chained stages.
  *  - Planning: each of the num_ctas persistent CTAs reads seq_lens and derives its own items
- *    with the same closed form as hpc_decode_plan (same tiles, same CTA assignment).
+ *    with a closed form over the same tiles and unit order as hpc_decode_plan. The CTAs take
+ *    contiguous unit runs of equal cost, where a tile costs 16 and each (request, kv head)
+ *    segment start adds the fixed cost of an item: 152 KB worth of KV streaming with one new
+ *    token, 224 KB with several (2.4 tiles of bf16 KV at tile_len 128, head_dim 128). The
+ *    environment variable HPC_ITEM_COST (integer, in 1/16 of a tile, 0 .. 1024) overrides it;
+ *    0 assigns exactly hpc_decode_plan's ranges (ceil(T / num_ctas) units per CTA).
  *  - Merge: a split (request, kv head) is merged by the CTA that finishes its last piece. It
  *    finds out via an atomic ticket; there is no wait.
  *  - Requests with no tiles (L = 0, or an invalid length with HPC_DEV_BAD_SEQLEN) get a
