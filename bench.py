@@ -263,7 +263,8 @@ class Step:
 
 class ShardStep:
     """The step of one batch placed over the ranks by request (load_balanced_split_step_b200.shard):
-    local parts through hpc_decode_step_lse, one all-gather of (out, lse), hpc_merge_lse."""
+    q rows of the local parts gathered (hpc_gather_rows), the parts through hpc_decode_step_lse,
+    one all-gather of (out, lse), every request formed from its parts (hpc_merge_lse_gather)."""
 
     def __init__(self, B, spec, dc, num_ctas, tile_len, rank, world):
         from load_balanced_split_step_b200 import shard as SH
@@ -272,7 +273,8 @@ class ShardStep:
         compute = SH.library_compute(spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype, k_scale=dc["k_scale"],
                                      v_scale=dc["v_scale"], num_ctas=num_ctas, status=self.status)
         self.st = SH.ShardedStep(spec.seq_lens, world, rank, spec.page_size, spec.num_heads, spec.head_dim,
-                                 compute=compute)
+                                 compute=compute, merge=SH.library_merge(self.status),
+                                 gather=SH.library_gather(self.status))
         self.out = None
 
     def __call__(self, seq_lens=None, ev=None, q=None):
@@ -286,8 +288,8 @@ class ShardStep:
 
     @property
     def launches(self):
-        split = sum(1 for places in self.st.where.values() if len(places) > 1)
-        return 1 + split  # the step, then one merge per split request
+        local = 2 if self.st.plan[self.st.rank] else 0  # q gather and the step, when the rank has parts
+        return local + 1  # then the indexed merge
 
 
 def step_lengths(dc, spec):
@@ -365,28 +367,48 @@ def static_leg(B, spec, dc, tl, steps, sms, layout="HND"):
 
 
 def shard_e2e_leg(step, case, dc, steps, world):
-    """The sharded step with q copied in from pinned host memory and the output copied out,
-    every step, in order on one stream (the exchange is inside the step)."""
+    """The sharded step with q copied in from pinned host memory and the output copied out every
+    step, overlapped as in e2e_leg: copy-in, compute (the exchange included) and copy-out
+    streams with two buffer sets, ordered by events."""
     dev = dc["seq_lens"].device
     q_host = case.q.pin_memory()
-    q_dev = torch.empty_like(q_host, device=dev)
-    host = None
-    for _ in range(3):
-        q_dev.copy_(q_host, non_blocking=True)
-        out = step(q=q_dev)
-        host = out.to("cpu", non_blocking=True)
+    nbuf = 2
+    q_dev = [torch.empty_like(q_host, device=dev) for _ in range(nbuf)]
+    hosts = [torch.empty(tuple(q_host.shape), dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_cmp = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+    def one(i):
+        b = i % nbuf
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[b])  # step i-2 has finished reading this q buffer
+            q_dev[b].copy_(q_host, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            s_cmp.wait_event(ev_out[b])  # step i-2's output has left its host buffer
+            out = step(q=q_dev[b])
+            ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            out.record_stream(s_out)  # allocated on the compute stream, read here
+            hosts[b].copy_(out, non_blocking=True)
+            ev_out[b].record(s_out)
+
+    for i in range(4):
+        one(i)
     torch.cuda.synchronize()
     barrier(world)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        q_dev.copy_(q_host, non_blocking=True)
-        out = step(q=q_dev)
-        host = out.to("cpu", non_blocking=True)
-    b.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for i in range(steps):
+        one(i)
+    t1.record(s_out)
     torch.cuda.synchronize()
     barrier(world)
-    return a.elapsed_time(b), q_host.numel() * q_host.element_size(), host.numel() * host.element_size()
+    return t0.elapsed_time(t1), q_host.numel() * q_host.element_size(), hosts[0].numel() * hosts[0].element_size()
 
 
 def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND", folded=False):

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 6
+#define HPC_DECODE_ABI_VERSION 7
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -86,6 +86,7 @@ typedef enum { HPC_HND = 0, HPC_NHD = 1 } hpc_kv_layout;
 #define HPC_DEV_BAD_PAGE 0x2u   /* a block_table entry outside [0, num_pages); reads there return zeros */
 #define HPC_DEV_CAPACITY 0x4u   /* more work items than the plan can hold (cannot happen for a valid plan) */
 #define HPC_DEV_TIMEOUT 0x8u    /* a bounded pipeline wait expired; the kernel gave up and returned */
+#define HPC_DEV_BAD_INDEX 0x10u /* a row index outside its table (hpc_gather_rows, hpc_merge_lse_gather) */
 
 /* One unit of a CTA's work: tiles [tile_begin, tile_end) of one (request, kv head). */
 typedef struct {
@@ -278,6 +279,29 @@ HPC_API int hpc_decode_step_lse(const void* q, const void* k_pages, const void* 
  *   out:  device float [rows][head_dim]; lse_out: device float [rows], or NULL. */
 HPC_API int hpc_merge_lse(const float* outs, const float* lses, int32_t parts, int64_t rows, int32_t head_dim,
                           float* out, float* lse_out, void* stream);
+
+/* The log-sum-exp merge with its parts found through an index, for a request-sharded batch:
+ * the all-gathered parts of every rank are rows of outs / lses, and each request lists its
+ * rows. For request r and head h, with p_k = part_index[r][k] over the k < max_parts where
+ * p_k >= 0:
+ *   LSE = log sum_k exp(lses[p_k][h]),  out[r][h][:] = sum_k exp(lses[p_k][h] - LSE) outs[p_k][h][:].
+ * A request with one part gets that part's row exactly (weight exp(0) = 1); a request with
+ * none gets zeros and LSE = -inf. An index >= part_rows is skipped and sets HPC_DEV_BAD_INDEX.
+ *   outs:       device fp32 [part_rows][num_heads][head_dim]; lses: fp32 [part_rows][num_heads].
+ *   part_index: device int32 [batch][max_parts], -1 for unused entries.
+ *   out:        fp32 [batch][num_heads][head_dim]; lse_out: fp32 [batch][num_heads] or NULL.
+ *   status:     device uint32 word or NULL.
+ * One warp per (request, head); lanes split head_dim. */
+HPC_API int hpc_merge_lse_gather(const float* outs, const float* lses, int64_t part_rows, const int32_t* part_index,
+                                 int32_t max_parts, int32_t batch, int32_t num_heads, int32_t head_dim, float* out,
+                                 float* lse_out, uint32_t* status, void* stream);
+
+/* Row gather: dst[j] = src[index[j]] for j < n, rows of row_bytes bytes (a multiple of 16;
+ * src and dst 16-byte aligned). A request-sharded rank uses it to collect the q rows of its
+ * parts. An index outside [0, src_rows) gives a zero row and sets HPC_DEV_BAD_INDEX in
+ * *status (device uint32, or NULL). */
+HPC_API int hpc_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* index, int64_t n,
+                            void* dst, uint32_t* status, void* stream);
 
 /* ---- several new tokens per request ----------------------------------------------------- */
 

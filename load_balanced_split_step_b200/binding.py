@@ -21,7 +21,7 @@ HPC_OK, HPC_ERR_ARG, HPC_ERR_SHAPE, HPC_ERR_DTYPE, HPC_ERR_ALIGN, HPC_ERR_CUDA, 
 HPC_BF16, HPC_FP32, HPC_E4M3 = 0, 1, 2
 HPC_HND, HPC_NHD = 0, 1
 _LAYOUTS = {"HND": HPC_HND, "NHD": HPC_NHD}
-DEV_STATUS = {"bad_seqlen": 0x1, "bad_page": 0x2, "capacity": 0x4, "timeout": 0x8}
+DEV_STATUS = {"bad_seqlen": 0x1, "bad_page": 0x2, "capacity": 0x4, "timeout": 0x8, "bad_index": 0x10}
 ITEM_DTYPE = np.dtype([("req", "<i4"), ("kv_head", "<i2"), ("flags", "<i2"),
                        ("tile_begin", "<i4"), ("tile_end", "<i4")])
 
@@ -31,7 +31,7 @@ EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_d
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
            "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue",
            "hpc_decode_step_multi", "hpc_decode_step_multi_workspace_bytes", "hpc_decode_step_lse",
-           "hpc_merge_lse", "hpc_wait_selftest")
+           "hpc_merge_lse", "hpc_wait_selftest", "hpc_merge_lse_gather", "hpc_gather_rows")
 
 
 class HpcError(RuntimeError):
@@ -89,6 +89,8 @@ def _load():
                                                vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp, vp]),
         "hpc_merge_lse": (ctypes.c_int, [vp, vp, i32, ctypes.c_int64, i32, vp, vp, vp]),
         "hpc_wait_selftest": (ctypes.c_int, [ctypes.c_uint64, i32, vp, vp, vp]),
+        "hpc_merge_lse_gather": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, vp, vp, vp, vp]),
+        "hpc_gather_rows": (ctypes.c_int, [vp, ctypes.c_int64, ctypes.c_int64, vp, ctypes.c_int64, vp, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -486,6 +488,40 @@ def merge_lse(outs, lses, out=None, lse_out=None):
     _check(_lib.hpc_merge_lse(_ptr(outs), _ptr(lses), parts, rows, D, _ptr(out), _ptr(lse_out), _stream(dev)),
            "hpc_merge_lse")
     return out, lse_out
+
+
+def merge_lse_gather(outs, lses, part_index, out=None, lse_out=None, status=None):
+    """``hpc_merge_lse_gather``: outs fp32 [part_rows, Hq, D], lses fp32 [part_rows, Hq], part_index
+    int32 [B, max_parts] (-1 unused) -> (out [B, Hq, D], lse [B, Hq])."""
+    _need(outs, "outs", torch.float32)
+    dev = outs.device
+    _need(lses, "lses", torch.float32, dev)
+    _need(part_index, "part_index", torch.int32, dev)
+    rows, Hq, D = outs.shape
+    if tuple(lses.shape) != (rows, Hq) or part_index.dim() != 2:
+        raise HpcError("outs [rows, Hq, D], lses [rows, Hq] and part_index [B, max_parts] disagree")
+    Bn, mp = part_index.shape
+    out = torch.empty((Bn, Hq, D), dtype=torch.float32, device=dev) if out is None else out
+    lse_out = torch.empty((Bn, Hq), dtype=torch.float32, device=dev) if lse_out is None else lse_out
+    _need(out, "out", torch.float32, dev)
+    _need(lse_out, "lse_out", torch.float32, dev)
+    _check(_lib.hpc_merge_lse_gather(_ptr(outs), _ptr(lses), rows, _ptr(part_index), mp, Bn, Hq, D, _ptr(out),
+                                     _ptr(lse_out), _ptr(status), _stream(dev)), "hpc_merge_lse_gather")
+    return out, lse_out
+
+
+def gather_rows(src, index, out=None, status=None):
+    """``hpc_gather_rows``: out[j] = src[index[j]] along the first dimension (rows a multiple of 16 bytes)."""
+    _need(src, "src")
+    dev = src.device
+    _need(index, "index", torch.int32, dev)
+    n = index.numel()
+    out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=dev) if out is None else out
+    _need(out, "out", src.dtype, dev)
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else out[0].numel() * out.element_size()
+    _check(_lib.hpc_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out), _ptr(status),
+                                _stream(dev)), "hpc_gather_rows")
+    return out
 
 
 def wait_selftest(limit_ns: int, arrive: bool, device, status=None):

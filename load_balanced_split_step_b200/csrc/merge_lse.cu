@@ -44,6 +44,82 @@ __global__ void __launch_bounds__(kMergeLseThreads)
   }
 }
 
+// The same merge, with each output row's parts found through an index: row (r, h) combines
+// rows part_index[r][k] (k < max_parts, index >= 0) of outs / lses at head h. One part is copied
+// exactly (its weight is exp(0) = 1 and the sum is 1); no part gives zeros and -inf. An index
+// at or past part_rows is skipped and sets HPC_DEV_BAD_INDEX.
+__global__ void __launch_bounds__(kMergeLseThreads)
+    merge_lse_gather_kernel(const float* __restrict__ outs, const float* __restrict__ lses,
+                            const int32_t* __restrict__ part_index, int32_t max_parts, int64_t part_rows,
+                            int32_t batch, int32_t num_heads, int32_t head_dim, float* __restrict__ out,
+                            float* __restrict__ lse_out, uint32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(batch) * num_heads;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    const int64_t r = row / num_heads;
+    const int h = static_cast<int>(row - r * num_heads);
+    const int32_t* idx = part_index + r * max_parts;
+    float M = -INFINITY;
+    bool bad = false;
+    for (int k = 0; k < max_parts; ++k) {
+      const int32_t i = idx[k];
+      if (i < 0) continue;
+      if (i >= part_rows) {
+        bad = true;
+        continue;
+      }
+      M = fmaxf(M, lses[static_cast<int64_t>(i) * num_heads + h]);
+    }
+    float S = 0.f;
+    if (M != -INFINITY)
+      for (int k = 0; k < max_parts; ++k) {
+        const int32_t i = idx[k];
+        if (i >= 0 && i < part_rows) S += expf(lses[static_cast<int64_t>(i) * num_heads + h] - M);
+      }
+    const float inv = S > 0.f ? 1.f / S : 0.f;
+    for (int d = lane; d < head_dim; d += 32) {
+      float acc = 0.f;
+      if (M != -INFINITY)
+        for (int k = 0; k < max_parts; ++k) {
+          const int32_t i = idx[k];
+          if (i < 0 || i >= part_rows) continue;
+          const int64_t pr = static_cast<int64_t>(i) * num_heads + h;
+          acc += expf(lses[pr] - M) * outs[pr * head_dim + d];
+        }
+      out[row * head_dim + d] = acc * inv;
+    }
+    if (lane == 0) {
+      if (lse_out) lse_out[row] = S > 0.f ? M + logf(S) : -INFINITY;
+      if (bad && status) atomicOr(status, HPC_DEV_BAD_INDEX);
+    }
+  }
+}
+
+// dst row j = src row index[j], rows of row_bytes (a multiple of 16) bytes. An index outside
+// [0, src_rows) gives a zero row and sets HPC_DEV_BAD_INDEX.
+__global__ void __launch_bounds__(kMergeLseThreads)
+    gather_rows_kernel(const uint4* __restrict__ src, int64_t src_rows, const int32_t* __restrict__ index,
+                       int64_t n, int64_t row_vecs, uint4* __restrict__ dst, uint32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t total = n * row_vecs;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = t / row_vecs, v = t - j * row_vecs;
+    const int32_t i = index[j];
+    if (i < 0 || i >= src_rows) {
+      dst[t] = make_uint4(0u, 0u, 0u, 0u);
+      if (v == 0 && status) atomicOr(status, HPC_DEV_BAD_INDEX);
+      continue;
+    }
+    dst[t] = src[static_cast<int64_t>(i) * row_vecs + v];
+  }
+}
+
 }  // namespace
 }  // namespace hpc
 
@@ -63,4 +139,46 @@ extern "C" int hpc_merge_lse(const float* outs, const float* lses, int32_t parts
                                    static_cast<cudaStream_t>(stream), outs, lses, parts, rows, head_dim, out, lse_out);
   if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "merge_lse_kernel: %s", cudaGetErrorString(e));
   return check_launch("merge_lse_kernel");
+}
+
+extern "C" int hpc_merge_lse_gather(const float* outs, const float* lses, int64_t part_rows, const int32_t* part_index,
+                                    int32_t max_parts, int32_t batch, int32_t num_heads, int32_t head_dim, float* out,
+                                    float* lse_out, uint32_t* status, void* stream) {
+  if (!outs || !lses || !part_index || !out) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (part_rows < 0 || max_parts < 1 || batch < 0 || num_heads < 1 || head_dim < 1)
+    return fail(HPC_ERR_ARG, "part_rows, max_parts, batch, num_heads and head_dim must be in range");
+  if (batch == 0) return HPC_OK;
+  const int64_t rows = static_cast<int64_t>(batch) * num_heads;
+  const int64_t per_block = kMergeLseThreads / 32;
+  int64_t blocks = (rows + per_block - 1) / per_block;
+  const int sms = device_sm_count();
+  const int64_t cap = sms > 0 ? static_cast<int64_t>(sms) * 8 : 1024;
+  if (blocks > cap) blocks = cap;
+  const cudaError_t e =
+      launch_pdl(merge_lse_gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kMergeLseThreads), 0,
+                 static_cast<cudaStream_t>(stream), outs, lses, part_index, max_parts, part_rows, batch, num_heads,
+                 head_dim, out, lse_out, status);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "merge_lse_gather_kernel: %s", cudaGetErrorString(e));
+  return check_launch("merge_lse_gather_kernel");
+}
+
+extern "C" int hpc_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* index, int64_t n,
+                               void* dst, uint32_t* status, void* stream) {
+  if (!src || !index || !dst) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (src_rows < 0 || n < 0 || row_bytes <= 0) return fail(HPC_ERR_ARG, "src_rows, n and row_bytes must be in range");
+  if (row_bytes % 16) return fail(HPC_ERR_SHAPE, "row_bytes must be a multiple of 16");
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15)
+    return fail(HPC_ERR_ALIGN, "src and dst must be 16-byte aligned");
+  if (n == 0) return HPC_OK;
+  const int64_t row_vecs = row_bytes / 16, total = n * row_vecs;
+  int64_t blocks = (total + kMergeLseThreads - 1) / kMergeLseThreads;
+  const int sms = device_sm_count();
+  const int64_t cap = sms > 0 ? static_cast<int64_t>(sms) * 8 : 1024;
+  if (blocks > cap) blocks = cap;
+  const cudaError_t e =
+      launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kMergeLseThreads), 0,
+                 static_cast<cudaStream_t>(stream), static_cast<const uint4*>(src), src_rows, index, n, row_vecs,
+                 static_cast<uint4*>(dst), status);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "gather_rows_kernel: %s", cudaGetErrorString(e));
+  return check_launch("gather_rows_kernel");
 }

@@ -32,7 +32,8 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ("hpc_decode_plan", "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue",
               "hpc_plan_cpu", "hpc_decode_plan_static", "hpc_decode_step", "hpc_decode_step_prologue",
-              "hpc_decode_step_multi", "hpc_decode_step_lse", "hpc_merge_lse"):
+              "hpc_decode_step_multi", "hpc_decode_step_lse", "hpc_merge_lse", "hpc_merge_lse_gather",
+              "hpc_gather_rows", "hpc_wait_selftest"):
         assert n in names
 
 
@@ -44,7 +45,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 6
+    assert B._lib.hpc_abi_version() == 7
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -82,6 +83,14 @@ def test_host_argument_errors_return_codes(B):
     assert B._lib.hpc_merge_lse(None, None, 2, 10, 64, None, None, None) == B.HPC_ERR_ARG
     assert B._lib.hpc_merge_lse(w, w, 0, 10, 64, w, None, None) == B.HPC_ERR_ARG
     assert B._lib.hpc_merge_lse(w, w, 2, 0, 64, w, None, None) == B.HPC_OK  # nothing to do
+    # indexed merge and row gather: nulls, sizes, alignment
+    assert B._lib.hpc_merge_lse_gather(None, w, 4, w, 2, 3, 8, 64, w, None, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_merge_lse_gather(w, w, 4, w, 0, 3, 8, 64, w, None, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_merge_lse_gather(w, w, 4, w, 2, 0, 8, 64, w, None, None, None) == B.HPC_OK  # nothing to do
+    assert B._lib.hpc_gather_rows(w, 4, 256, None, 2, w, None, None) == B.HPC_ERR_ARG
+    assert B._lib.hpc_gather_rows(w, 4, 200, w, 2, w, None, None) == B.HPC_ERR_SHAPE
+    assert B._lib.hpc_gather_rows(ctypes.c_void_p(24), 4, 256, w, 2, w, None, None) == B.HPC_ERR_ALIGN
+    assert B._lib.hpc_gather_rows(w, 4, 256, w, 0, w, None, None) == B.HPC_OK
     # wait diagnostic: null status, limit outside 1 .. 2 s
     assert B._lib.hpc_wait_selftest(1000, 0, None, None, None) == B.HPC_ERR_ARG
     assert B._lib.hpc_wait_selftest(0, 0, w, None, None) == B.HPC_ERR_ARG

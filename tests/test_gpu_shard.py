@@ -4,6 +4,8 @@ C ABI on one GPU.
 * hpc_decode_step_lse writes the same output as hpc_decode_step, and lse matches the fp64
   oracle's log-sum-exp.
 * hpc_merge_lse equals its definition (float64 torch) on random parts, -inf parts included.
+* hpc_merge_lse_gather (parts found through an index) equals its definition; a single part is
+  copied bit for bit. hpc_gather_rows is an exact row gather. Both flag indices out of range.
 * A batch sharded over 2, 3 and 4 ranks gives the unsharded oracle result. The ranks run
   one after another in this process: each computes its parts, their (out, lse) are stacked
   as the all-gather would stack them, and split requests are merged. No kernel waits on
@@ -68,6 +70,62 @@ def test_merge_lse_definition(B):
     assert torch.max(torch.abs(o.cpu().double() - ref)).item() <= 1e-5
     lc = l.cpu().double()
     assert torch.isneginf(lc[20]) and torch.max(torch.abs(lc[:20] - L[:20])).item() <= 1e-5
+
+
+def test_merge_lse_gather_definition(B):
+    g = torch.Generator().manual_seed(6)
+    rows, Hq, D = 23, 8, 128
+    outs = torch.randn(rows, Hq, D, generator=g)
+    lses = torch.randn(rows, Hq, generator=g) * 4
+    lses[3, :2] = -math.inf  # a part with no mass for two heads
+    idx = torch.tensor([[-1, -1, -1, -1],   # no part: zeros, -inf
+                        [7, -1, -1, -1],    # one part: copied exactly
+                        [-1, 2, -1, 11],    # two parts, unused entries between
+                        [3, 0, 22, 5],      # four parts
+                        [3, -1, -1, -1]],   # one part whose lse is -inf for two heads
+                       dtype=torch.int32)
+    st = B.new_status("cuda")
+    o, l = B.merge_lse_gather(outs.cuda(), lses.cuda(), idx.cuda(), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    o, l = o.cpu().double(), l.cpu().double()
+    for r in range(idx.shape[0]):
+        parts = [int(i) for i in idx[r] if int(i) >= 0]
+        if not parts:
+            assert torch.all(o[r] == 0) and torch.all(torch.isneginf(l[r]))
+            continue
+        ld = lses[parts].double()
+        L = torch.logsumexp(ld, 0)
+        ref = (torch.exp(ld - L)[..., None] * outs[parts].double()).sum(0)
+        ref = torch.where(torch.isneginf(L)[..., None], torch.zeros_like(ref), ref)
+        assert torch.max(torch.abs(o[r] - ref)).item() <= 1e-5, r
+        fin = torch.isfinite(L)
+        assert torch.equal(torch.isneginf(l[r]), ~fin)
+        assert torch.max(torch.abs(l[r][fin] - L[fin])).item() <= 1e-5
+    assert torch.equal(o[1].float(), outs[7])  # a single part is a copy
+    # an index past the parts is skipped and flagged
+    bad = idx.clone()
+    bad[2, 0] = 99
+    st = B.new_status("cuda")
+    o2, _ = B.merge_lse_gather(outs.cuda(), lses.cuda(), bad.cuda(), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == B.DEV_STATUS["bad_index"]
+    assert torch.max(torch.abs(o2.cpu()[2].double() - o[2])).item() <= 1e-6
+
+
+def test_gather_rows(B):
+    g = torch.Generator().manual_seed(7)
+    src = torch.randn(10, 8, 128, generator=g).bfloat16().cuda()
+    index = torch.tensor([3, 0, 9, 3, 5], dtype=torch.int32, device="cuda")
+    st = B.new_status("cuda")
+    out = B.gather_rows(src, index, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and torch.equal(out, src[index.long()])
+    index[1] = 10  # outside the source: a zero row and the status bit
+    out = B.gather_rows(src, index, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == B.DEV_STATUS["bad_index"]
+    assert torch.all(out[1] == 0) and torch.equal(out[2:], src[index[2:].long()])
 
 
 @pytest.mark.parametrize("kv", ["bf16", "e4m3"])

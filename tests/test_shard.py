@@ -75,14 +75,25 @@ def _oracle_compute(case):
     return compute
 
 
-def _merge_by_definition(outs, lses):
-    """LSE = log sum_i exp(lse_i); out = sum_i exp(lse_i - LSE) out_i (float64)."""
-    l = lses.double()
-    M = l.max(0).values
-    w = torch.exp(l - M)
-    L = M + torch.log(w.sum(0))
-    out = (torch.exp(l - L)[..., None] * outs.double()).sum(0)
-    return out.float(), L.float()
+def _merge_by_definition(outs, lses, part_index):
+    """For each request, its parts' rows: LSE = log sum_i exp(lse_i); out = sum_i exp(lse_i - LSE)
+    out_i (float64). A request with no part gets zeros."""
+    B, Hq, D = part_index.shape[0], outs.shape[1], outs.shape[2]
+    out = torch.zeros((B, Hq, D), dtype=torch.float64)
+    lse = torch.full((B, Hq), -math.inf, dtype=torch.float64)
+    for r in range(B):
+        rows = [int(i) for i in part_index[r] if int(i) >= 0]
+        if not rows:
+            continue
+        l = lses[rows].double()
+        L = torch.logsumexp(l, 0)
+        out[r] = (torch.exp(l - L)[..., None] * outs[rows].double()).sum(0)
+        lse[r] = L
+    return out.float(), lse.float()
+
+
+def _gather_rows(src, index):
+    return src.index_select(0, index.long())
 
 
 def _worker(rank, world, port, q):
@@ -94,7 +105,7 @@ def _worker(rank, world, port, q):
         spec = W.custom_spec((700, 64, 5, 2000, 33), 16, 2, 64, 16, 32, seed=11)
         case = W.make_case(spec)
         st = S.ShardedStep(spec.seq_lens, world, rank, spec.page_size, 16, 64, compute=_oracle_compute(case),
-                           merge=_merge_by_definition)
+                           merge=_merge_by_definition, gather=_gather_rows)
         out = st.step(case.q, case.k_pages, case.v_pages, case.block_table, spec.tile_len)
         q.put((rank, out.numpy(), [len(p) for p in st.plan]))
     finally:
