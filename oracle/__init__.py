@@ -20,7 +20,8 @@ definitions by eye:
 * ``fp8``: OCP E4M3 decode and encode (round to nearest even, saturating).
 
 Pins (tests/test_oracle_*.py) tie each function to something other than itself:
-library routines, closed forms, brute force and invariants. The one function without
-a value pin is the attention value beyond those invariants and the library
-cross-check; its header says "parity unpinned" for exactly that part.
+library routines, closed forms, brute force on tiny inputs, invariants, and planted
+mistakes that the pins must catch. The pages print no worked numerical example for the
+attention value, so its pins are the definition's own: fp64 SDPA, brute force and closed
+forms.
 """

@@ -24,10 +24,11 @@ Readings where the pages are silent:
 * An E4M3 cache holds codes; the value is decode(code) * scale[g].
 * A request with L_r = 0 attends over nothing; its output is defined as 0.
 
-Parity unpinned beyond the invariants and library cross-check listed in
-tests/test_oracle_attention.py (torch SDPA in fp64, pure-Python loops on tiny inputs,
-single key, identical keys, q = 0, split invariance). The pages print no worked
-numerical example.
+Pins (tests/test_oracle_attention.py, tests/test_oracle_multi.py): torch SDPA in fp64,
+pure-Python loops on tiny inputs, closed forms (a single key returns v; identical keys or
+q = 0 give the mean of v; no keys give 0), split invariance, and planted mistakes (a wrong
+page index, GQA map or scale) that the pins catch. The pages print no worked numerical
+example, so the pins tie the oracle to the definition itself.
 """
 from __future__ import annotations
 
