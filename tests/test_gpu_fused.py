@@ -80,6 +80,36 @@ def test_item_cost_split(B, monkeypatch, cost):
         assert _tickets_zero(ws, spec.batch, spec.kv_heads)
 
 
+@pytest.mark.parametrize("D,Bmax", [(128, 4095), (64, 2047)])
+def test_largest_batch(B, monkeypatch, D, Bmax):
+    """The single launch keeps the per-request prefix (tile and segment counts packed in one
+    int64) in shared memory. Its largest batch, 4095 requests at head_dim 128 and 2047 at 64,
+    runs with short ragged lengths and empty requests, with and without the item cost, and
+    matches the oracle on sampled requests. One request more is refused before launch."""
+    rng = np.random.default_rng(D)
+    lens = [int(x) for x in rng.integers(0, 80, size=Bmax)]
+    spec = W.custom_spec(lens, 8, 2, D, 16, 32, seed=D + 7)
+    case = W.make_case(spec)
+    dc = to_device(case)
+    empty = [i for i, L in enumerate(lens) if L == 0][:3]
+    rows = sorted(set([0, 1, 2, Bmax // 2, Bmax - 2, Bmax - 1] + empty + [int(x) for x in rng.integers(0, Bmax, 6)]))
+    ref = oracle_out(W.make_case(spec, requests=rows))
+    for cost in ("0", None):
+        if cost is None:
+            monkeypatch.delenv("HPC_ITEM_COST", raising=False)
+        else:
+            monkeypatch.setenv("HPC_ITEM_COST", cost)
+        out, st, ws = _fused(B, spec, dc)
+        assert st == 0
+        assert_bf16_tol(out[rows], ref, what=f"largest batch {Bmax}, D {D}, cost {cost}")
+        assert _tickets_zero(ws, spec.batch, spec.kv_heads)
+    more = torch.cat([dc["seq_lens"], dc["seq_lens"][:1]])
+    bt = torch.cat([dc["block_table"], dc["block_table"][:1]])
+    q = torch.cat([dc["q"], dc["q"][:1]])
+    with pytest.raises(B.HpcError, match="single-launch limit"):
+        B.decode_step_fused(q, dc["k_pages"], dc["v_pages"], bt, more, 8, 2, 32)
+
+
 def test_empty_and_invalid_requests(B):
     spec = W.custom_spec((0, 40, 5, 200), 8, 2, 64, 16, 32, seed=51)
     case = W.make_case(spec)
