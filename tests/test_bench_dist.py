@@ -73,3 +73,10 @@ def test_reference_arm_prints_on_rank0_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    # the JSON contract of the line
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["higher_is_better"] is True and line["vs_baseline"] is None and "workload" in line["config"]
+    assert {"value", "unit", "cores", "kind", "sample"} <= set(line["cpu_baseline"])
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["d2h_bytes_per_step"] == 0
