@@ -125,3 +125,89 @@ def plan_static(seq_lens, kv_heads: int, tile_len: int, splits: int) -> Plan:
 def static_splits(batch: int, kv_heads: int, num_sms: int) -> int:
     """S = max(1, ceil(2 * num_SMs / (B * Hkv))): enough CTAs for two waves."""
     return max(1, -(-2 * num_sms // (batch * kv_heads)))
+
+
+# ---------------------------------------------------------------------------------------------
+# The single-launch step's split: tiles plus a fixed cost per item start.
+#
+# Reading 21 of the path's spec. The pages balance CTAs by "current load" (remio.ai, section
+# "Por qué Tencent HPC importa …") and leave the measure of load open; reading 7 takes tile
+# counts. The single-launch step counts each item start as a fixed number of tile-equivalents
+# as well. Step by step:
+#
+# 1. Units and segments as in plan_dynamic: units u = 0..T-1 enumerate request -> kv head ->
+#    tile; a segment is one (request, kv head) with tiles, numbered S = 1, 2, ... in unit order.
+# 2. Every tile costs W = 16 and every segment start adds c = item_cost. Unit u, a tile of
+#    segment S, sits at cost position W*u + c*S.
+# 3. total = W*T + c*(number of segments); chunk = W * ceil(total / (W*G)), in cost units.
+# 4. Unit u belongs to CTA floor(position(u) / chunk). Positions grow with u, so every CTA owns
+#    one contiguous run of units (possibly empty).
+# 5. A CTA's run is cut into items at segment boundaries. An item covering its whole segment is
+#    DIRECT. Any other item writes a partial state: slot 2g if it is CTA g's first item, else
+#    slot 2g + 1 (a split segment can only be the first or the last item of its CTA's run).
+# With c = 0 the owners are u // ceil(T/G), the units of plan_dynamic.
+# ---------------------------------------------------------------------------------------------
+
+COST_PER_TILE = 16
+FLAG_SECOND_SLOT = 2  # item record flag: the partial slot is 2g + 1 (else 2g)
+
+
+@dataclass
+class CostSplit:
+    unit_begin: np.ndarray  # int64 [G]: first unit of each CTA's run
+    unit_end: np.ndarray  # int64 [G]: one past its last unit
+    items: list  # per CTA: ITEM_DTYPE array of its items, in order (flags DIRECT / SECOND_SLOT)
+    slots: list  # per CTA: partial slot of each item, -1 for a DIRECT item
+    chunk: int  # cost units per CTA
+    n_units: int
+    item_cost: int
+
+
+def plan_cost_split(seq_lens, kv_heads: int, tile_len: int, num_ctas: int, item_cost: int) -> CostSplit:
+    """Steps 1-5 above, unit by unit. seq_lens are the lengths that get tiles (0 for none)."""
+    lens = [int(x) for x in seq_lens]
+    G, W, c = int(num_ctas), COST_PER_TILE, int(item_cost)
+    units = []  # (r, kvh, tile, S)
+    S = 0
+    for r, L in enumerate(lens):
+        nt = num_tiles(L, tile_len)
+        for kvh in range(kv_heads):
+            if nt == 0:
+                continue
+            S += 1
+            for t in range(nt):
+                units.append((r, kvh, t, S))
+    T = len(units)
+    total = W * T + c * S
+    chunk = W * (-(-total // (W * G))) if T > 0 else 0
+    owner = [(W * u + c * s) // chunk for u, (_, _, _, s) in enumerate(units)]
+    begin = np.full(G, T, dtype=np.int64)
+    end = np.full(G, T, dtype=np.int64)
+    rows = [[] for _ in range(G)]  # [r, kvh, tb, te]
+    for u, (r, kvh, t, _) in enumerate(units):
+        g = owner[u]
+        if not rows[g]:
+            begin[g] = u
+        end[g] = u + 1
+        last = rows[g][-1] if rows[g] else None
+        if last is not None and last[0] == r and last[1] == kvh:
+            last[3] = t + 1
+        else:
+            rows[g].append([r, kvh, t, t + 1])
+    # CTAs with no units sit where the next owner starts: [T, T) at the end, or an empty run
+    # at the first unit after the previous CTA's run
+    for g in range(G - 1, -1, -1):
+        if not rows[g]:
+            begin[g] = end[g] = begin[g + 1] if g + 1 < G else T
+    items, slots = [], []
+    for g in range(G):
+        arr = np.zeros(len(rows[g]), dtype=ITEM_DTYPE)
+        sl = []
+        for k, (r, kvh, tb, te) in enumerate(rows[g]):
+            direct = tb == 0 and te == num_tiles(lens[r], tile_len)
+            flags = FLAG_DIRECT if direct else (FLAG_SECOND_SLOT if k > 0 else 0)
+            arr[k] = (r, kvh, flags, tb, te)
+            sl.append(-1 if direct else 2 * g + (1 if k > 0 else 0))
+        items.append(arr)
+        slots.append(sl)
+    return CostSplit(begin, end, items, slots, chunk, T, c)
