@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 7
+#define HPC_DECODE_ABI_VERSION 8
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -83,7 +83,8 @@ typedef enum { HPC_HND = 0, HPC_NHD = 1 } hpc_kv_layout;
 
 /* Bits the kernels OR into the caller's device status word. */
 #define HPC_DEV_BAD_SEQLEN 0x1u /* seq_len < 0 or > max tokens; the request gets no tiles and a zero output */
-#define HPC_DEV_BAD_PAGE 0x2u   /* a block_table entry outside [0, num_pages); reads there return zeros */
+#define HPC_DEV_BAD_PAGE 0x2u   /* a block_table entry outside [0, num_pages); no load is issued for that page
+                                   and its tokens are left out of the request's softmax */
 #define HPC_DEV_CAPACITY 0x4u   /* more work items than the plan can hold (cannot happen for a valid plan) */
 #define HPC_DEV_TIMEOUT 0x8u    /* a bounded pipeline wait expired; the kernel gave up and returned */
 #define HPC_DEV_BAD_INDEX 0x10u /* a row index outside its table (hpc_gather_rows, hpc_merge_lse_gather) */
@@ -99,6 +100,9 @@ typedef struct {
 } hpc_work_item;
 
 #define HPC_ITEM_DIRECT 1
+/* Set only in hpc_cta_record items: the item's partial state goes to slot 2g + 1 of its CTA g
+ * (without it, a non-DIRECT item uses slot 2g). */
+#define HPC_ITEM_SECOND_SLOT 2
 
 /* A plan is a host struct of device pointers into one caller-owned workspace. Layout:
  *   counts       int64[4]             n_items, n_merge, n_units, chunk (written on the device)
@@ -116,6 +120,64 @@ typedef struct {
   int32_t* merge_indptr;
   int32_t* merge_list;
 } hpc_plan;
+
+/* ---- per-call options (ABI 8) ----------------------------------------------------------- */
+
+/* Record of one CTA's share of a single-launch step, written when a caller asks for it (tests,
+ * debugging). CTA g writes the record at byte offset g * hpc_step_record_bytes(1, record_items):
+ * this header, then min(n_items, record_items) hpc_work_item entries in the order the CTA ran
+ * them. An entry's flags hold HPC_ITEM_DIRECT, or HPC_ITEM_SECOND_SLOT for a split item whose
+ * partial state went to slot 2g + 1 (slot 2g without it). */
+typedef struct {
+  int64_t unit_begin, unit_end; /* the CTA's run [begin, end) of the request -> kv head -> tile units */
+  int64_t chunk;                /* cost units per CTA of the split */
+  int32_t item_cost;            /* cost of an item start used by the split, in 1/16 tile */
+  int32_t n_items;              /* items the CTA ran */
+} hpc_cta_record;
+
+#define HPC_ITEM_COST_DEFAULT (-1)
+#define HPC_ITEM_COST_MAX 1024
+#define HPC_E4M3_MMA 0     /* E4M3 caches on the mma.sync consumers (the default) */
+#define HPC_E4M3_TCGEN05 1 /* E4M3 caches on the tcgen05 kernel, where it applies */
+#define HPC_TRACE_WORDS 8  /* uint64 words per CTA in a trace buffer */
+#define HPC_BUILD_TRACE 1u /* hpc_build_flags(): the library was built with HPC_TRACE */
+
+/* Options of one call. A NULL options pointer selects the defaults, as does a struct set from
+ * HPC_STEP_OPTIONS_INIT (note that item_cost 0 is not the default). The library reads no
+ * environment variables.
+ *   item_cost:    single-launch steps only. The fixed cost of starting an item in the split of
+ *                 units over CTAs, in 1/16 of a tile, 0 .. HPC_ITEM_COST_MAX. 0 splits by tiles
+ *                 alone (exactly hpc_decode_plan's CTA ranges). HPC_ITEM_COST_DEFAULT: the time
+ *                 one item start takes, as KV bytes a CTA streams meanwhile: 152 KB with one new
+ *                 token, 224 KB with several, converted to tiles of the call's shape (rounded).
+ *   e4m3_kernel:  HPC_E4M3_MMA or HPC_E4M3_TCGEN05. The tcgen05 kernel serves E4M3 caches with
+ *                 head_dim 128 in hpc_decode_attention, hpc_decode_step and hpc_decode_step_lse;
+ *                 elsewhere the choice is ignored.
+ *   record:       single-launch steps only: device buffer of hpc_step_record_bytes(num_ctas,
+ *                 record_items) bytes that receives every CTA's hpc_cta_record, or NULL.
+ *   trace:        device uint64 [num_ctas][HPC_TRACE_WORDS], or NULL. Only a library built with
+ *                 HPC_TRACE (hpc_build_flags() & HPC_BUILD_TRACE) accepts it; the default build
+ *                 returns HPC_ERR_ARG, and its kernels carry no trace code. Per CTA, from
+ *                 %globaltimer (ns): [0] entry, [1] plan ready (after the wait on the previous
+ *                 kernel), [2] first stage consumed, [3] last item finished by the consumers,
+ *                 [4] producer done; then [5] items, [6] pipeline stages, [7] SM id. Words [2]
+ *                 and [3] stay 0 for a CTA without work. The mma.sync kernel writes it. */
+typedef struct {
+  int32_t item_cost;
+  int32_t e4m3_kernel;
+  void* record;
+  int32_t record_items;
+  int32_t reserved;
+  uint64_t* trace;
+} hpc_step_options;
+
+#define HPC_STEP_OPTIONS_INIT {HPC_ITEM_COST_DEFAULT, HPC_E4M3_MMA, NULL, 0, 0, NULL}
+
+/* Bytes of a record buffer for num_ctas CTAs with record_items entries each. */
+HPC_API size_t hpc_step_record_bytes(int32_t num_ctas, int32_t record_items);
+
+/* Bit set of build options: HPC_BUILD_TRACE. */
+HPC_API uint32_t hpc_build_flags(void);
 
 /* ---- planning ------------------------------------------------------------------------ */
 
@@ -185,13 +247,16 @@ HPC_API size_t hpc_partial_ml_bytes(const hpc_plan* plan, int32_t num_heads);
  *             writes slot k with natural-log state m = max score, l = sum exp(s - m),
  *             o = sum exp(s - m) v.
  *   out:      device [batch][num_heads][head_dim], out_dtype HPC_FP32 or HPC_BF16. DIRECT
- *             items write it here; hpc_merge_states writes the rest. */
+ *             items write it here; hpc_merge_states writes the rest.
+ *   options:  NULL, or hpc_step_options: e4m3_kernel and trace apply here; item_cost must be
+ *             HPC_ITEM_COST_DEFAULT and record NULL (they belong to the single-launch steps). */
 HPC_API int hpc_decode_attention(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
                          hpc_kv_layout kv_layout, const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
                          int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                          int32_t max_pages_per_req, const int32_t* seq_lens, const hpc_plan* plan,
                          float sm_scale, float* partial_o, float* partial_ml, void* out,
-                         hpc_dtype out_dtype, uint32_t* status, void* stream);
+                         hpc_dtype out_dtype, const hpc_step_options* options,
+                                 uint32_t* status, void* stream);
 
 /* ---- single-launch step ---------------------------------------------------------------- */
 
@@ -208,9 +273,11 @@ HPC_API size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads,
  *    with a closed form over the same tiles and unit order as hpc_decode_plan. The CTAs take
  *    contiguous unit runs of equal cost, where a tile costs 16 and each (request, kv head)
  *    segment start adds the fixed cost of an item: 152 KB worth of KV streaming with one new
- *    token, 224 KB with several (2.4 tiles of bf16 KV at tile_len 128, head_dim 128). The
- *    environment variable HPC_ITEM_COST (integer, in 1/16 of a tile, 0 .. 1024) overrides it;
- *    0 assigns exactly hpc_decode_plan's ranges (ceil(T / num_ctas) units per CTA).
+ *    token, 224 KB with several (2.4 tiles of bf16 KV at tile_len 128, head_dim 128).
+ *    options->item_cost (1/16 of a tile, 0 .. HPC_ITEM_COST_MAX) sets it per call; 0 assigns
+ *    exactly hpc_decode_plan's ranges (ceil(T / num_ctas) units per CTA).
+ *  - options: NULL for the defaults, or see hpc_step_options (item cost, E4M3 kernel, per-CTA
+ *    record of the split, trace).
  *  - Merge: a split (request, kv head) is merged by the CTA that finishes its last piece. It
  *    finds out via an atomic ticket; there is no wait.
  *  - Requests with no tiles (L = 0, or an invalid length with HPC_DEV_BAD_SEQLEN) get a
@@ -228,7 +295,8 @@ HPC_API int hpc_decode_step(const void* q, const void* k_pages, const void* v_pa
                             int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                             int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
                             int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
-                            hpc_dtype out_dtype, uint32_t* status, void* stream);
+                            hpc_dtype out_dtype, const hpc_step_options* options,
+                            uint32_t* status, void* stream);
 
 /* hpc_decode_step with the decode prologue folded in ("vLLM × HPC-Ops" summary: "RoPE +
  * QK-Norm + KV-write" in front of attention). One launch does what hpc_decode_prologue followed
@@ -255,7 +323,8 @@ HPC_API int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, con
                                      int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
                                      const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
                                      float sm_scale, void* workspace, size_t workspace_bytes, void* out,
-                                     hpc_dtype out_dtype, uint32_t* status, void* stream);
+                                     hpc_dtype out_dtype, const hpc_step_options* options,
+                                     uint32_t* status, void* stream);
 
 /* hpc_decode_step that also writes the log-sum-exp of every output row:
  *   lse[r][h] = log sum_j exp(sm_scale * q[r,h] . k_j)   (natural log; -inf when L_r = 0),
@@ -266,7 +335,8 @@ HPC_API int hpc_decode_step_lse(const void* q, const void* k_pages, const void* 
                                 int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
                                 const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
                                 int32_t batch, int32_t tile_len, int32_t num_ctas, float sm_scale, void* workspace,
-                                size_t workspace_bytes, void* out, hpc_dtype out_dtype, float* lse, uint32_t* status,
+                                size_t workspace_bytes, void* out, hpc_dtype out_dtype, float* lse, const hpc_step_options* options,
+                                uint32_t* status,
                                 void* stream);
 
 /* Log-sum-exp merge of outputs computed over disjoint parts of the same keys (a request split
@@ -332,7 +402,8 @@ HPC_API int hpc_decode_step_multi(const void* q, int32_t q_len, const void* k_pa
                                   int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                                   int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch,
                                   int32_t tile_len, int32_t num_ctas, float sm_scale, void* workspace,
-                                  size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
+                                  size_t workspace_bytes, void* out, hpc_dtype out_dtype, const hpc_step_options* options,
+                                  uint32_t* status,
                                   void* stream);
 
 /* ---- merge --------------------------------------------------------------------------- */
@@ -402,9 +473,10 @@ HPC_API int hpc_decode_step_noalloc(const void* q, const void* k_pages, const vo
 /* ---- misc ---------------------------------------------------------------------------- */
 
 /* Launch shape the attention kernel would use: pipeline stages, dynamic shared memory
- * bytes and threads per CTA. For introspection and benchmarking. */
+ * bytes and threads per CTA. e4m3_kernel as in hpc_step_options. For introspection and
+ * benchmarking. */
 HPC_API int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, int32_t page_size, int32_t tile_len,
-                              int32_t ctas_per_sm, int32_t* stages, int32_t* smem_bytes,
+                              int32_t ctas_per_sm, int32_t e4m3_kernel, int32_t* stages, int32_t* smem_bytes,
                               int32_t* threads);
 
 /* Diagnostic of the bounded pipeline waits. Every wait in the library's kernels (stage

@@ -24,8 +24,15 @@ _LAYOUTS = {"HND": HPC_HND, "NHD": HPC_NHD}
 DEV_STATUS = {"bad_seqlen": 0x1, "bad_page": 0x2, "capacity": 0x4, "timeout": 0x8, "bad_index": 0x10}
 ITEM_DTYPE = np.dtype([("req", "<i4"), ("kv_head", "<i2"), ("flags", "<i2"),
                        ("tile_begin", "<i4"), ("tile_end", "<i4")])
+ITEM_DIRECT, ITEM_SECOND_SLOT = 1, 2
+RECORD_DTYPE = np.dtype([("unit_begin", "<i8"), ("unit_end", "<i8"), ("chunk", "<i8"), ("item_cost", "<i4"),
+                         ("n_items", "<i4")])
+ITEM_COST_DEFAULT, ITEM_COST_MAX = -1, 1024
+E4M3_KERNELS = {"mma": 0, "tcgen05": 1}
+TRACE_WORDS = 8
+BUILD_TRACE = 1
 
-EXPORTS = ("hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_decode_plan",
+EXPORTS = ("hpc_step_record_bytes", "hpc_build_flags", "hpc_plan_workspace_bytes", "hpc_plan_static_workspace_bytes", "hpc_decode_plan",
            "hpc_decode_plan_static", "hpc_plan_cpu", "hpc_partial_o_bytes", "hpc_partial_ml_bytes",
            "hpc_decode_attention", "hpc_merge_states", "hpc_decode_prologue", "hpc_attention_launch_info",
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
@@ -46,19 +53,30 @@ class CPlan(ctypes.Structure):
                 ("merge_indptr", ctypes.c_void_p), ("merge_list", ctypes.c_void_p)]
 
 
+class COptions(ctypes.Structure):
+    _fields_ = [("item_cost", ctypes.c_int32), ("e4m3_kernel", ctypes.c_int32), ("record", ctypes.c_void_p),
+                ("record_items", ctypes.c_int32), ("reserved", ctypes.c_int32), ("trace", ctypes.c_void_p)]
+
+
+_path = LIB
+
+
 def library_path() -> str:
-    return LIB
+    return _path
 
 
-def _load():
-    if not os.path.exists(LIB):
-        raise HpcError(f"{LIB} is missing; build it with `python -m load_balanced_split_step_b200.build` "
+def _load(path=LIB):
+    if not os.path.exists(path):
+        raise HpcError(f"{path} is missing; build it with `python -m load_balanced_split_step_b200.build` "
                        "(there is no CPU fallback)")
-    lib = ctypes.CDLL(LIB)
+    lib = ctypes.CDLL(path)
     i32, vp, sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
     fp = ctypes.c_float
     P = ctypes.POINTER(CPlan)
+    O = ctypes.POINTER(COptions)
     sig = {
+        "hpc_step_record_bytes": (sz, [i32, i32]),
+        "hpc_build_flags": (ctypes.c_uint32, []),
         "hpc_plan_workspace_bytes": (sz, [i32, i32, i32]),
         "hpc_plan_static_workspace_bytes": (sz, [i32, i32, i32]),
         "hpc_decode_plan": (ctypes.c_int, [vp, i32, i32, i32, i32, i32, i32, vp, sz, P, vp, vp]),
@@ -67,26 +85,26 @@ def _load():
         "hpc_partial_o_bytes": (sz, [P, i32, i32]),
         "hpc_partial_ml_bytes": (sz, [P, i32]),
         "hpc_decode_attention": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32,
-                                                vp, i32, vp, P, fp, vp, vp, vp, ctypes.c_int, vp, vp]),
+                                                vp, i32, vp, P, fp, vp, vp, vp, ctypes.c_int, O, vp, vp]),
         "hpc_merge_states": (ctypes.c_int, [vp, vp, P, i32, i32, vp, ctypes.c_int, vp, vp]),
         "hpc_decode_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32,
                                                i32, vp, i32, vp, i32, i32, i32, i32, vp, vp]),
-        "hpc_attention_launch_info": (ctypes.c_int, [i32, ctypes.c_int, i32, i32, i32, ctypes.POINTER(i32),
+        "hpc_attention_launch_info": (ctypes.c_int, [i32, ctypes.c_int, i32, i32, i32, i32, ctypes.POINTER(i32),
                                                      ctypes.POINTER(i32), ctypes.POINTER(i32)]),
         "hpc_decode_step_noalloc": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp,
                                                    i32, vp, i32, i32, i32, fp, vp, ctypes.c_int, vp, vp]),
         "hpc_decode_step_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
         "hpc_decode_step": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32, vp,
-                                           i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp]),
+                                           i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, O, vp, vp]),
         "hpc_decode_step_prologue": (ctypes.c_int, [vp, vp, vp, fp, fp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp,
                                                     i32, i32, i32, i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz,
-                                                    vp, ctypes.c_int, vp, vp]),
+                                                    vp, ctypes.c_int, O, vp, vp]),
         "hpc_decode_step_multi_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
         "hpc_decode_step_multi": (ctypes.c_int, [vp, i32, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32,
-                                                 i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp,
-                                                 vp]),
+                                                 i32, i32, vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, O,
+                                                 vp, vp]),
         "hpc_decode_step_lse": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, i32, i32, i32, i32, i32,
-                                               vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, vp, vp]),
+                                               vp, i32, vp, i32, i32, i32, fp, vp, sz, vp, ctypes.c_int, vp, O, vp, vp]),
         "hpc_merge_lse": (ctypes.c_int, [vp, vp, i32, ctypes.c_int64, i32, vp, vp, vp]),
         "hpc_wait_selftest": (ctypes.c_int, [ctypes.c_uint64, i32, vp, vp, vp]),
         "hpc_merge_lse_gather": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, vp, vp, vp, vp]),
@@ -102,6 +120,18 @@ def _load():
 
 
 _lib = _load()
+
+
+def use_library(path: str = LIB):
+    """Switch this module to another build of the library (e.g. the HPC_TRACE build, see
+    ``build.build(trace=True)``); ``use_library()`` goes back to the default build."""
+    global _lib, _path
+    _lib = _load(path)
+    _path = path
+
+
+def build_flags() -> int:
+    return int(_lib.hpc_build_flags())
 
 
 def status_string(code: int) -> str:
@@ -189,9 +219,10 @@ def plan(seq_lens: torch.Tensor, num_heads: int, kv_heads: int, tile_len: int, n
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     status = new_status(dev) if status is None else status
     raw = CPlan()
-    _check(_lib.hpc_decode_plan(_ptr(seq_lens), B, num_heads, kv_heads, tile_len, num_ctas, max_seq_len,
-                                _ptr(workspace), workspace.numel(), ctypes.byref(raw), _ptr(status),
-                                _stream(dev)), "hpc_decode_plan")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_plan(_ptr(seq_lens), B, num_heads, kv_heads, tile_len, num_ctas, max_seq_len,
+                                    _ptr(workspace), workspace.numel(), ctypes.byref(raw), _ptr(status),
+                                    _stream(dev)), "hpc_decode_plan")
     return Plan(raw, workspace)
 
 
@@ -207,9 +238,10 @@ def plan_static(seq_lens: torch.Tensor, num_heads: int, kv_heads: int, tile_len:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     status = new_status(dev) if status is None else status
     raw = CPlan()
-    _check(_lib.hpc_decode_plan_static(_ptr(seq_lens), B, num_heads, kv_heads, tile_len, splits, max_seq_len,
-                                       _ptr(workspace), workspace.numel(), ctypes.byref(raw), _ptr(status),
-                                       _stream(dev)), "hpc_decode_plan_static")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_plan_static(_ptr(seq_lens), B, num_heads, kv_heads, tile_len, splits, max_seq_len,
+                                           _ptr(workspace), workspace.numel(), ctypes.byref(raw), _ptr(status),
+                                           _stream(dev)), "hpc_decode_plan_static")
     return Plan(raw, workspace)
 
 
@@ -264,37 +296,115 @@ def _geometry(k_pages, kv_layout):
     return n, hkv, psz, d, _LAYOUTS[kv_layout]
 
 
+def _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, head_dim, dev):
+    """Checks the two caches against each other, the query's head_dim and the device, and the
+    E4M3 scales. Returns (dtype code, num_pages, kv_heads, page_size, layout code)."""
+    _need(k_pages, "k_pages", device=dev)
+    _need(v_pages, "v_pages", device=dev)
+    code = _kv_code(kv_dtype, k_pages)
+    _kv_code(kv_dtype, v_pages)
+    num_pages, Hkv, P, D, lay = _geometry(k_pages, kv_layout)
+    if tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise HpcError(f"v_pages {tuple(v_pages.shape)} and k_pages {tuple(k_pages.shape)} differ")
+    if D != head_dim:
+        raise HpcError(f"cache head_dim {D} does not match the query's {head_dim}")
+    if code == HPC_E4M3:
+        for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+            _need(t, name, torch.float32, dev)
+            if t.numel() != Hkv:
+                raise HpcError(f"{name} must hold one scale per kv head ({Hkv})")
+    return code, num_pages, Hkv, P, lay
+
+
+def _tables(block_table, seq_lens, batch, dev):
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    if block_table.dim() != 2 or block_table.shape[0] != batch or seq_lens.numel() != batch:
+        raise HpcError(f"block_table [batch, pages] and seq_lens [batch] must match the batch of {batch}")
+
+
+def _output(out, shape, out_dtype, dev):
+    if out is None:
+        return torch.empty(shape, dtype=out_dtype, device=dev)
+    _need(out, "out", (torch.float32, torch.bfloat16), dev)
+    if tuple(out.shape) != tuple(shape):
+        raise HpcError(f"out has shape {tuple(out.shape)}, expected {tuple(shape)}")
+    return out
+
+
+def _out_code(out):
+    return HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32
+
+
+def options(item_cost=None, e4m3_kernel="mma", record=None, record_items=0, trace=None, device=None, num_ctas=None):
+    """A ``hpc_step_options`` struct, or None when every option has its default.
+    item_cost: 1/16 tile per item start (None: the library's default). e4m3_kernel: "mma" or
+    "tcgen05". record: uint8 device tensor of ``record_bytes(num_ctas, record_items)`` bytes.
+    trace: int64 device tensor [num_ctas, TRACE_WORDS] (HPC_TRACE builds only)."""
+    if e4m3_kernel not in E4M3_KERNELS:
+        raise HpcError(f"e4m3_kernel must be one of {list(E4M3_KERNELS)}")
+    if item_cost is None and e4m3_kernel == "mma" and record is None and trace is None:
+        return None
+    o = COptions()
+    o.item_cost = ITEM_COST_DEFAULT if item_cost is None else int(item_cost)
+    o.e4m3_kernel = E4M3_KERNELS[e4m3_kernel]
+    if record is not None:
+        _need(record, "record", torch.uint8, device)
+        o.record, o.record_items = record.data_ptr(), int(record_items)
+        if num_ctas is not None and record.numel() < record_bytes(num_ctas, record_items):
+            raise HpcError(f"record holds {record.numel()} bytes, {record_bytes(num_ctas, record_items)} needed")
+    if trace is not None:
+        _need(trace, "trace", torch.int64, device)
+        if num_ctas is not None and trace.numel() < num_ctas * TRACE_WORDS:
+            raise HpcError(f"trace must hold num_ctas x {TRACE_WORDS} words")
+        o.trace = trace.data_ptr()
+    return o
+
+
+def _opt_ref(o):
+    return None if o is None else ctypes.byref(o)
+
+
+def record_bytes(num_ctas: int, record_items: int) -> int:
+    return int(_lib.hpc_step_record_bytes(num_ctas, record_items))
+
+
+def read_record(record: torch.Tensor, num_ctas: int, record_items: int):
+    """The per-CTA records of a single-launch step: (headers RECORD_DTYPE [G], items list of
+    ITEM_DTYPE arrays, the first min(n_items, record_items) of each CTA)."""
+    raw = record.cpu().numpy()
+    stride = RECORD_DTYPE.itemsize + record_items * ITEM_DTYPE.itemsize
+    heads = np.empty(num_ctas, dtype=RECORD_DTYPE)
+    items = []
+    for g in range(num_ctas):
+        blk = raw[g * stride:(g + 1) * stride]
+        heads[g] = blk[:RECORD_DTYPE.itemsize].view(RECORD_DTYPE)[0]
+        n = min(int(heads[g]["n_items"]), record_items)
+        items.append(blk[RECORD_DTYPE.itemsize:RECORD_DTYPE.itemsize + n * ITEM_DTYPE.itemsize].view(ITEM_DTYPE))
+    return heads, items
+
+
 def attention(q, k_pages, v_pages, block_table, seq_lens, p: Plan, *, kv_dtype="bf16", kv_layout="HND",
               k_scale=None, v_scale=None, sm_scale=None, out=None, out_dtype=torch.float32, partial_o=None,
-              partial_ml=None, status=None):
+              partial_ml=None, status=None, e4m3_kernel="mma", trace=None):
     """Persistent split-KV attention (``hpc_decode_attention``). Returns (out, partial_o, partial_ml)."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
-    for name, t in (("k_pages", k_pages), ("v_pages", v_pages)):
-        _need(t, name, device=dev)
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
-    _kv_code(kv_dtype, v_pages)
     B, Hq, D = q.shape
-    num_pages, Hkv, P, D2, lay = _geometry(k_pages, kv_layout)
-    if D2 != D or v_pages.shape != k_pages.shape:
-        raise HpcError("cache shape does not match q")
-    if out is None:
-        out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
-    _need(out, "out", (torch.float32, torch.bfloat16), dev)
+    code, num_pages, Hkv, P, lay = _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, D, dev)
+    _tables(block_table, seq_lens, B, dev)
+    out = _output(out, (B, Hq, D), out_dtype, dev)
     if partial_o is None or partial_ml is None:
         partial_o, partial_ml = partial_buffers(p, Hq, D, dev)
     status = new_status(dev) if status is None else status
-    if code == HPC_E4M3:
-        _need(k_scale, "k_scale", torch.float32, dev)
-        _need(v_scale, "v_scale", torch.float32, dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    _check(_lib.hpc_decode_attention(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
-        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), ctypes.byref(p.raw), scale, _ptr(partial_o),
-        _ptr(partial_ml), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
-        _stream(dev)), "hpc_decode_attention")
+    opt = options(e4m3_kernel=e4m3_kernel, trace=trace, device=dev, num_ctas=p.num_ctas)
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_attention(
+            _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+            _ptr(block_table), block_table.shape[1], _ptr(seq_lens), ctypes.byref(p.raw), scale, _ptr(partial_o),
+            _ptr(partial_ml), _ptr(out), _out_code(out), _opt_ref(opt), _ptr(status), _stream(dev)),
+            "hpc_decode_attention")
     return out, partial_o, partial_ml
 
 
@@ -306,9 +416,10 @@ def merge(p: Plan, partial_o, partial_ml, out, num_heads: int, status=None):
     _need(out, "out", (torch.float32, torch.bfloat16), dev)
     status = new_status(dev) if status is None else status
     D = out.shape[-1]
-    _check(_lib.hpc_merge_states(_ptr(partial_o), _ptr(partial_ml), ctypes.byref(p.raw), num_heads, D, _ptr(out),
-                                 HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
-                                 _stream(dev)), "hpc_merge_states")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_merge_states(_ptr(partial_o), _ptr(partial_ml), ctypes.byref(p.raw), num_heads, D, _ptr(out),
+                                     HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
+                                     _stream(dev)), "hpc_merge_states")
     return out
 
 
@@ -320,20 +431,27 @@ def prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, n
     dev = qkv.device
     _need(q_norm_w, "q_norm_w", torch.float32, dev)
     _need(k_norm_w, "k_norm_w", torch.float32, dev)
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
     B, H, D = qkv.shape
     if H != num_heads + 2 * kv_heads:
         raise HpcError("qkv must hold num_heads + 2*kv_heads heads")
-    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
+    if q_norm_w.numel() != D or k_norm_w.numel() != D:
+        raise HpcError("norm weights must hold head_dim values")
+    code, num_pages, Hkv, P, lay = _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, D, dev)
+    if Hkv != kv_heads:
+        raise HpcError(f"cache has {Hkv} kv heads, expected {kv_heads}")
+    _tables(block_table, seq_lens, B, dev)
     if q_out is None:
         q_out = torch.empty((B, num_heads, D), dtype=torch.bfloat16, device=dev)
+    _need(q_out, "q_out", torch.bfloat16, dev)
+    if tuple(q_out.shape) != (B, num_heads, D):
+        raise HpcError("q_out must be [batch, num_heads, head_dim]")
     status = new_status(dev) if status is None else status
-    _check(_lib.hpc_decode_prologue(
-        _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(q_out), _ptr(k_pages),
-        _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, _ptr(block_table), block_table.shape[1],
-        _ptr(seq_lens), B, num_heads, kv_heads, D, _ptr(status), _stream(dev)), "hpc_decode_prologue")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_prologue(
+            _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(q_out), _ptr(k_pages),
+            _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, _ptr(block_table),
+            block_table.shape[1], _ptr(seq_lens), B, num_heads, kv_heads, D, _ptr(status), _stream(dev)),
+            "hpc_decode_prologue")
     return q_out
 
 
@@ -345,38 +463,52 @@ def step_workspace(batch, num_heads, kv_heads, head_dim, num_ctas, device):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def _grid(num_ctas, dev):
+    return torch.cuda.get_device_properties(dev).multi_processor_count if num_ctas is None else int(num_ctas)
+
+
+def _workspace(ws, nbytes, dev):
+    if ws is None:
+        return torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    _need(ws, "workspace", torch.uint8, dev)
+    return ws
+
+
 def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *,
                       kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None,
-                      out=None, out_dtype=torch.float32, status=None, workspace=None):
+                      out=None, out_dtype=torch.float32, status=None, workspace=None, item_cost=None,
+                      e4m3_kernel="mma", record=None, record_items=0, trace=None):
     """One decode step in a single launch (``hpc_decode_step``): in-kernel planning, attention
-    and ticket merge. Returns (out, status, workspace); pass the workspace back on later calls."""
+    and ticket merge. Returns (out, status, workspace); pass the workspace back on later calls.
+    item_cost, e4m3_kernel, record / record_items and trace are the call's options."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
     B, Hq, D = q.shape
-    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
-    if num_ctas is None:
-        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
-    if out is None:
-        out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
+    if Hq != num_heads:
+        raise HpcError(f"q has {Hq} heads, expected {num_heads}")
+    code, num_pages, Hkv, P, lay = _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, D, dev)
+    if Hkv != kv_heads:
+        raise HpcError(f"cache has {Hkv} kv heads, expected {kv_heads}")
+    _tables(block_table, seq_lens, B, dev)
+    G = _grid(num_ctas, dev)
+    out = _output(out, (B, Hq, D), out_dtype, dev)
     status = new_status(dev) if status is None else status
-    if workspace is None:
-        workspace = step_workspace(B, Hq, Hkv, D, num_ctas, dev)
+    workspace = _workspace(workspace, _lib.hpc_decode_step_workspace_bytes(B, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    _check(_lib.hpc_decode_step(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
-        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
-        workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
-        _stream(dev)), "hpc_decode_step")
+    opt = options(item_cost, e4m3_kernel, record, record_items, trace, dev, G)
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_step(
+            _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+            _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, G, scale, _ptr(workspace),
+            workspace.numel(), _ptr(out), _out_code(out), _opt_ref(opt), _ptr(status), _stream(dev)),
+            "hpc_decode_step")
     return out, status, workspace
 
 
 def decode_step_prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads,
                          tile_len, *, kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, eps=1e-6,
                          rope_theta=1e6, num_ctas=None, sm_scale=None, out=None, out_dtype=torch.float32,
-                         status=None, workspace=None):
+                         status=None, workspace=None, item_cost=None, record=None, record_items=0, trace=None):
     """One decode step in a single launch with the prologue folded in
     (``hpc_decode_step_prologue``): the new token's K/V go into the cache and q is formed from
     qkv inside the attention kernel. Returns (out, status, workspace)."""
@@ -384,27 +516,27 @@ def decode_step_prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table,
     dev = qkv.device
     _need(q_norm_w, "q_norm_w", torch.float32, dev)
     _need(k_norm_w, "k_norm_w", torch.float32, dev)
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
     B, H, D = qkv.shape
     if H != num_heads + 2 * kv_heads:
         raise HpcError("qkv must hold num_heads + 2*kv_heads heads")
-    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
-    if num_ctas is None:
-        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
-    if out is None:
-        out = torch.empty((B, num_heads, D), dtype=out_dtype, device=dev)
+    if q_norm_w.numel() != D or k_norm_w.numel() != D:
+        raise HpcError("norm weights must hold head_dim values")
+    code, num_pages, Hkv, P, lay = _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, D, dev)
+    if Hkv != kv_heads:
+        raise HpcError(f"cache has {Hkv} kv heads, expected {kv_heads}")
+    _tables(block_table, seq_lens, B, dev)
+    G = _grid(num_ctas, dev)
+    out = _output(out, (B, num_heads, D), out_dtype, dev)
     status = new_status(dev) if status is None else status
-    if workspace is None:
-        workspace = step_workspace(B, num_heads, Hkv, D, num_ctas, dev)
+    workspace = _workspace(workspace, _lib.hpc_decode_step_workspace_bytes(B, num_heads, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    _check(_lib.hpc_decode_step_prologue(
-        _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(k_pages), _ptr(v_pages), code,
-        lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, num_heads, Hkv, D, _ptr(block_table), block_table.shape[1],
-        _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace), workspace.numel(), _ptr(out),
-        HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status), _stream(dev)),
-        "hpc_decode_step_prologue")
+    opt = options(item_cost, "mma", record, record_items, trace, dev, G)
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_step_prologue(
+            _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(k_pages), _ptr(v_pages),
+            code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, num_heads, Hkv, D, _ptr(block_table),
+            block_table.shape[1], _ptr(seq_lens), B, tile_len, G, scale, _ptr(workspace), workspace.numel(),
+            _ptr(out), _out_code(out), _opt_ref(opt), _ptr(status), _stream(dev)), "hpc_decode_step_prologue")
     return out, status, workspace
 
 
@@ -418,59 +550,63 @@ def multi_workspace(batch, q_len, num_heads, kv_heads, head_dim, num_ctas, devic
 
 def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile_len, *, kv_dtype="bf16",
                       kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None,
-                      out_dtype=torch.float32, status=None, workspace=None):
+                      out_dtype=torch.float32, status=None, workspace=None, item_cost=None, record=None,
+                      record_items=0, trace=None):
     """q_len new tokens per request in one launch (``hpc_decode_step_multi``): q is
     [B, q_len, Hq, D]; query token t of request r sits at position L_r - q_len + t and
     attends causally. Returns (out [B, q_len, Hq, D], status, workspace)."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
     B, T, Hq, D = q.shape
-    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
-    if num_ctas is None:
-        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
-    if out is None:
-        out = torch.empty((B, T, Hq, D), dtype=out_dtype, device=dev)
+    code, num_pages, Hkv, P, lay = _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, D, dev)
+    if Hkv != kv_heads:
+        raise HpcError(f"cache has {Hkv} kv heads, expected {kv_heads}")
+    _tables(block_table, seq_lens, B, dev)
+    G = _grid(num_ctas, dev)
+    out = _output(out, (B, T, Hq, D), out_dtype, dev)
     status = new_status(dev) if status is None else status
-    if workspace is None:
-        workspace = multi_workspace(B, T, Hq, Hkv, D, num_ctas, dev)
+    workspace = _workspace(workspace, _lib.hpc_decode_step_multi_workspace_bytes(B, T, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    _check(_lib.hpc_decode_step_multi(
-        _ptr(q), T, _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
-        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
-        workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status),
-        _stream(dev)), "hpc_decode_step_multi")
+    opt = options(item_cost, "mma", record, record_items, trace, dev, G)
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_step_multi(
+            _ptr(q), T, _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv,
+            D, _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, G, scale, _ptr(workspace),
+            workspace.numel(), _ptr(out), _out_code(out), _opt_ref(opt), _ptr(status), _stream(dev)),
+            "hpc_decode_step_multi")
     return out, status, workspace
 
 
 def decode_step_lse(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",
                     kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None, lse=None,
-                    status=None, workspace=None):
+                    status=None, workspace=None, item_cost=None, e4m3_kernel="mma"):
     """``hpc_decode_step_lse``: the single-launch step, plus the natural-log log-sum-exp of
     every output row. Returns (out fp32 [B, Hq, D], lse fp32 [B, Hq], status, workspace)."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
     B, Hq, D = q.shape
-    num_pages, Hkv, P, _, lay = _geometry(k_pages, kv_layout)
-    if num_ctas is None:
-        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
-    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev) if out is None else out
+    if Hq != num_heads:
+        raise HpcError(f"q has {Hq} heads, expected {num_heads}")
+    code, num_pages, Hkv, P, lay = _cache(k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, D, dev)
+    if Hkv != kv_heads:
+        raise HpcError(f"cache has {Hkv} kv heads, expected {kv_heads}")
+    _tables(block_table, seq_lens, B, dev)
+    G = _grid(num_ctas, dev)
+    out = _output(out, (B, Hq, D), torch.float32, dev)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=dev) if lse is None else lse
     _need(lse, "lse", torch.float32, dev)
+    if tuple(lse.shape) != (B, Hq):
+        raise HpcError("lse must be [batch, num_heads]")
     status = new_status(dev) if status is None else status
-    if workspace is None:
-        workspace = step_workspace(B, Hq, Hkv, D, num_ctas, dev)
+    workspace = _workspace(workspace, _lib.hpc_decode_step_workspace_bytes(B, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    _check(_lib.hpc_decode_step_lse(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
-        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(workspace),
-        workspace.numel(), _ptr(out), HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(lse), _ptr(status),
-        _stream(dev)), "hpc_decode_step_lse")
+    opt = options(item_cost, e4m3_kernel, device=dev)
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_step_lse(
+            _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+            _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, G, scale, _ptr(workspace),
+            workspace.numel(), _ptr(out), _out_code(out), _ptr(lse), _opt_ref(opt), _ptr(status), _stream(dev)),
+            "hpc_decode_step_lse")
     return out, lse, status, workspace
 
 
@@ -485,8 +621,9 @@ def merge_lse(outs, lses, out=None, lse_out=None):
         raise HpcError("outs and lses disagree on the rows")
     out = torch.empty(outs.shape[1:], dtype=torch.float32, device=dev) if out is None else out
     lse_out = torch.empty(lses.shape[1:], dtype=torch.float32, device=dev) if lse_out is None else lse_out
-    _check(_lib.hpc_merge_lse(_ptr(outs), _ptr(lses), parts, rows, D, _ptr(out), _ptr(lse_out), _stream(dev)),
-           "hpc_merge_lse")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_merge_lse(_ptr(outs), _ptr(lses), parts, rows, D, _ptr(out), _ptr(lse_out), _stream(dev)),
+               "hpc_merge_lse")
     return out, lse_out
 
 
@@ -505,8 +642,9 @@ def merge_lse_gather(outs, lses, part_index, out=None, lse_out=None, status=None
     lse_out = torch.empty((Bn, Hq), dtype=torch.float32, device=dev) if lse_out is None else lse_out
     _need(out, "out", torch.float32, dev)
     _need(lse_out, "lse_out", torch.float32, dev)
-    _check(_lib.hpc_merge_lse_gather(_ptr(outs), _ptr(lses), rows, _ptr(part_index), mp, Bn, Hq, D, _ptr(out),
-                                     _ptr(lse_out), _ptr(status), _stream(dev)), "hpc_merge_lse_gather")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_merge_lse_gather(_ptr(outs), _ptr(lses), rows, _ptr(part_index), mp, Bn, Hq, D, _ptr(out),
+                                         _ptr(lse_out), _ptr(status), _stream(dev)), "hpc_merge_lse_gather")
     return out, lse_out
 
 
@@ -519,8 +657,9 @@ def gather_rows(src, index, out=None, status=None):
     out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=dev) if out is None else out
     _need(out, "out", src.dtype, dev)
     row_bytes = src[0].numel() * src.element_size() if src.shape[0] else out[0].numel() * out.element_size()
-    _check(_lib.hpc_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out), _ptr(status),
-                                _stream(dev)), "hpc_gather_rows")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out), _ptr(status),
+                                    _stream(dev)), "hpc_gather_rows")
     return out
 
 
@@ -530,14 +669,15 @@ def wait_selftest(limit_ns: int, arrive: bool, device, status=None):
     dev = torch.device(device)
     status = new_status(dev) if status is None else status
     waited = torch.zeros(1, dtype=torch.int64, device=dev)
-    _check(_lib.hpc_wait_selftest(int(limit_ns), 1 if arrive else 0, _ptr(status), _ptr(waited), _stream(dev)),
-           "hpc_wait_selftest")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_wait_selftest(int(limit_ns), 1 if arrive else 0, _ptr(status), _ptr(waited), _stream(dev)),
+               "hpc_wait_selftest")
     return status, waited
 
 
 def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",
                 kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, out=None, out_dtype=torch.float32,
-                status=None, static_splits=None):
+                status=None, static_splits=None, e4m3_kernel="mma"):
     """plan -> attention -> merge (three launches) for one decode step; returns (out, plan, status)."""
     dev = q.device
     status = new_status(dev) if status is None else status
@@ -547,7 +687,8 @@ def decode_step(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads,
     else:
         p = plan(seq_lens, num_heads, kv_heads, tile_len, num_ctas, max_seq, status)
     out, po, pml = attention(q, k_pages, v_pages, block_table, seq_lens, p, kv_dtype=kv_dtype, kv_layout=kv_layout,
-                             k_scale=k_scale, v_scale=v_scale, out=out, out_dtype=out_dtype, status=status)
+                             k_scale=k_scale, v_scale=v_scale, out=out, out_dtype=out_dtype, status=status,
+                             e4m3_kernel=e4m3_kernel)
     merge(p, po, pml, out, num_heads, status)
     return out, p, status
 
@@ -561,31 +702,32 @@ def decode_step_noalloc(q, k_pages, v_pages, block_table, seq_lens, num_heads, k
     """One decode step through ``hpc_decode_step_noalloc``: the library keeps the plan and
     partial states in its own static device array, for callers that cannot allocate device
     memory. Returns (out, status). Calls that overlap on the GPU share that array; keep
-    them on one stream."""
+    them on one stream. The cache is HND."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
-    _need(block_table, "block_table", torch.int32, dev)
-    _need(seq_lens, "seq_lens", torch.int32, dev)
-    code = _kv_code(kv_dtype, k_pages)
     B, Hq, D = q.shape
-    num_pages, Hkv, P, _ = k_pages.shape
-    if num_ctas is None:
-        num_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
-    if out is None:
-        out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
+    if Hq != num_heads:
+        raise HpcError(f"q has {Hq} heads, expected {num_heads}")
+    code, num_pages, Hkv, P, _ = _cache(k_pages, v_pages, kv_dtype, "HND", k_scale, v_scale, D, dev)
+    if Hkv != kv_heads:
+        raise HpcError(f"cache has {Hkv} kv heads, expected {kv_heads}")
+    _tables(block_table, seq_lens, B, dev)
+    G = _grid(num_ctas, dev)
+    out = _output(out, (B, Hq, D), out_dtype, dev)
     status = new_status(dev) if status is None else status
+    _need(status, "status", torch.int32, dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    _check(_lib.hpc_decode_step_noalloc(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
-        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, num_ctas, scale, _ptr(out),
-        HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32, _ptr(status), _stream(dev)),
-        "hpc_decode_step_noalloc")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_decode_step_noalloc(
+            _ptr(q), _ptr(k_pages), _ptr(v_pages), code, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
+            _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, tile_len, G, scale, _ptr(out),
+            _out_code(out), _ptr(status), _stream(dev)), "hpc_decode_step_noalloc")
     return out, status
 
 
-def launch_info(head_dim, kv_dtype, page_size, tile_len, ctas_per_sm=1):
+def launch_info(head_dim, kv_dtype, page_size, tile_len, ctas_per_sm=1, e4m3_kernel="mma"):
     st, sm, th = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
     _check(_lib.hpc_attention_launch_info(head_dim, _KV_DTYPES[kv_dtype], page_size, tile_len, ctas_per_sm,
-                                          ctypes.byref(st), ctypes.byref(sm), ctypes.byref(th)),
-           "hpc_attention_launch_info")
+                                          E4M3_KERNELS[e4m3_kernel], ctypes.byref(st), ctypes.byref(sm),
+                                          ctypes.byref(th)), "hpc_attention_launch_info")
     return {"stages": st.value, "smem_bytes": sm.value, "threads": th.value}

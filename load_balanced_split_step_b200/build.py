@@ -1,6 +1,10 @@
 """Builds libhpcdecode.so in-tree with nvcc for sm_100a.
 
-    python -m load_balanced_split_step_b200.build [--force] [--ptxas-v]
+    python -m load_balanced_split_step_b200.build [--force] [--ptxas-v] [--trace]
+
+--trace builds libhpcdecode_trace.so instead: the same library compiled with HPC_TRACE, whose
+attention kernel writes per-CTA timestamps into a caller's trace buffer (hpc_step_options). The
+default build carries no trace code.
 """
 from __future__ import annotations
 
@@ -16,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libhpcdecode.so")
+TRACE_LIB = os.path.join(PKG, "libhpcdecode_trace.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
@@ -46,7 +51,7 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False, lib: str = LIB, defines=()) -> str:
-    if not force and not ptxas_verbose and not defines and up_to_date(lib):
+    if not force and not ptxas_verbose and up_to_date(lib):
         return lib
     cmd = [nvcc(), *ARCH, *FLAGS, f"-I{INCLUDE}", "-shared", "-o", lib + ".tmp", *sources()]
     cmd += [f"-D{d}" for d in defines]
@@ -61,9 +66,18 @@ def build(force: bool = False, ptxas_verbose: bool = False, lib: str = LIB, defi
     return lib
 
 
+def build_trace(force: bool = False) -> str:
+    """libhpcdecode_trace.so: the library with the HPC_TRACE stamps compiled in."""
+    return build(force=force, lib=TRACE_LIB, defines=("HPC_TRACE",))
+
+
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true")
+    ap.add_argument("--trace", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, ptxas_verbose=a.ptxas_v))
+    if a.trace:
+        print(build_trace(force=a.force))
+    else:
+        print(build(force=a.force, ptxas_verbose=a.ptxas_v))

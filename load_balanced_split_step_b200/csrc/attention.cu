@@ -386,6 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int64_t s_scan[16], s_walk[9];
   __shared__ int s_flag;
   __shared__ int32_t s_pages[32];
+  // per ring slot: the stage's page id was outside the pool, so page 0 stood in for it and the
+  // consumers skip the stage (written before the fill's arrive, read after its wait)
+  __shared__ uint8_t s_bad[kMaxStages];
+  __shared__ int s_rec_n;  // items this CTA has run (written by consumer thread 0)
   // folded prologue: q_norm_w, theta^(-2i/D), two rotation tables [cos | sin], new-token barrier
   __shared__ float s_qw[PRO ? D : 1];
   __shared__ double s_invf[PRO ? D / 2 : 1];
@@ -413,7 +417,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t ring_u32 = smem_u32(ring);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + stages * groups);
 
+#ifdef HPC_TRACE
+  uint64_t* trace = p.trace ? p.trace + static_cast<size_t>(blockIdx.x) * HPC_TRACE_WORDS : nullptr;
+  if (trace && threadIdx.x == 0) {
+    trace[0] = global_timer_ns();
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    trace[7] = smid;
+    trace[2] = trace[3] = 0;
+  }
+#endif
   if (threadIdx.x == 0) {
+    s_rec_n = 0;
     for (int s = 0; s < stages * groups; ++s) mbar_init(full0 + 8 * s, 1);
     for (int s = 0; s < stages; ++s) mbar_init(empty0 + 8 * s, wps);
     if (PRO) mbar_init(smem_u32(&s_pro_bar), kConsumerWarps);
@@ -437,6 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     cursor.it = p.cta_indptr[blockIdx.x];
     cursor.it_end = p.cta_indptr[blockIdx.x + 1];
   }
+#ifdef HPC_TRACE
+  if (trace && threadIdx.x == 0) trace[1] = global_timer_ns();
+#endif
   const int C = p.chunk_tokens;
   const int P = p.page_size;
 
@@ -467,9 +485,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           bad |= HPC_DEV_TIMEOUT;
           return false;
         }
-        const int32_t page = s_pages[k];
+        int32_t page = s_pages[k];
         const int off = static_cast<int>((off0 + (cb + k) * C) & (P - 1));
-        if (page < 0 || page >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;  // TMA fills zeros there
+        // a page id outside the pool is never handed to the copy engine: page 0 stands in, and
+        // the consumers leave the stage's tokens out (a stage never spans two pages)
+        const bool page_ok = page >= 0 && page < p.num_pages;
+        if (!page_ok) {
+          bad |= HPC_DEV_BAD_PAGE;
+          page = 0;
+        }
+        s_bad[stage] = page_ok ? 0 : 1;
         const int bi = stage * groups + gidx;
         const uint32_t full = full0 + 8 * bi;
         if (bi < 64) par_lo ^= uint64_t(1) << bi;
@@ -527,6 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(full0 + 8 * bi, par)) bad |= HPC_DEV_TIMEOUT;
       }
       if (bad) atomicOr(p.status, bad);
+#ifdef HPC_TRACE
+      if (trace) {
+        trace[4] = global_timer_ns();
+        trace[6] = static_cast<uint64_t>(issued);
+      }
+#endif
     }
     return;
   }
@@ -576,6 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   while (cursor.next(p, x)) {
     const int kvh = x.kvh;
     const int head0 = kvh * p.group;
+    if (ctid == 0) {  // items this CTA ran (its record, and the trace's count)
+      if (FUSED && p.record) record_item(p, s_rec_n, x);
+      ++s_rec_n;
+    }
     const int64_t tok0 = x.tok0, tok1 = x.tok1;
     // causal limit of this warp's query token: it sits at position L - q_len + my_t
     int64_t lim = tok1;
@@ -629,8 +664,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) atomicOr(p.status, HPC_DEV_TIMEOUT);
         }
         wait_par ^= 1u << stage;
+#ifdef HPC_TRACE
+        if (trace && warp == 0 && lane == 0 && trace[2] == 0) trace[2] = global_timer_ns();
+#endif
         const int64_t tb = t + 16 * my_first;
-        if (ok && t_live && tb < lim) {
+        if (ok && t_live && tb < lim && !s_bad[stage]) {
           const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
           const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
           if (FP8 && nb == 4)
@@ -738,6 +776,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_barrier_sync(1, cthreads);  // reduce buffers are reused by the next item
     it_par ^= 1;
   }
+  if constexpr (FUSED) {
+    // s_walk still holds this CTA's unit run and the chunk from plan_in_kernel
+    if (p.record && ctid == 0) record_header(p, s_walk[0], s_walk[1], s_walk[7], s_rec_n);
+  }
+#ifdef HPC_TRACE
+  if (trace && ctid == 0) {
+    if (s_rec_n > 0) trace[3] = global_timer_ns();
+    trace[5] = static_cast<uint64_t>(s_rec_n);
+  }
+#endif
 }
 
 // ----------------------------------------------------------------------------- host side
@@ -870,12 +918,12 @@ extern "C" size_t hpc_partial_ml_bytes(const hpc_plan* plan, int32_t num_heads) 
 }
 
 extern "C" int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, int32_t page_size, int32_t tile_len,
-                                         int32_t ctas_per_sm, int32_t* stages, int32_t* smem_bytes,
-                                         int32_t* threads) {
+                                         int32_t ctas_per_sm, int32_t e4m3_kernel, int32_t* stages,
+                                         int32_t* smem_bytes, int32_t* threads) {
   if (tile_len <= 0 || page_size <= 0) return fail(HPC_ERR_ARG, "bad tile/page size");
   LaunchShape ls;
   const int C = chunk_tokens(tile_len, page_size);
-  if (kv_dtype == HPC_E4M3 && e4m3_on_tensor_cores() && tc_supported(head_dim, true, 8, 1, false)) {
+  if (kv_dtype == HPC_E4M3 && e4m3_kernel == HPC_E4M3_TCGEN05 && tc_supported(head_dim, true, 8, 1, false)) {
     const int sm = tc_smem_bytes(ctas_per_sm);
     if (!sm) return fail(HPC_ERR_SHAPE, "tensor-core E4M3 attention does not fit shared memory");
     if (stages) *stages = (sm - 12288 - 1024) / (2 * 128 * 128);
@@ -891,8 +939,54 @@ extern "C" int hpc_attention_launch_info(int32_t head_dim, hpc_dtype kv_dtype, i
   return HPC_OK;
 }
 
+extern "C" size_t hpc_step_record_bytes(int32_t num_ctas, int32_t record_items) {
+  if (num_ctas < 1 || record_items < 0) return 0;
+  return static_cast<size_t>(num_ctas) * record_stride(record_items);
+}
+
+extern "C" uint32_t hpc_build_flags(void) {
+#ifdef HPC_TRACE
+  return HPC_BUILD_TRACE;
+#else
+  return 0u;
+#endif
+}
+
 namespace hpc {
 namespace {
+
+// Per-call options, checked. single_launch: the call is one of the hpc_decode_step entry points,
+// where the item cost and the record apply.
+struct Options {
+  int32_t item_cost = HPC_ITEM_COST_DEFAULT;
+  bool tc = false;
+  uint8_t* record = nullptr;
+  int32_t record_items = 0;
+  uint64_t* trace = nullptr;
+};
+
+int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
+  *out = Options{};
+  if (!o) return HPC_OK;
+  if (o->item_cost != HPC_ITEM_COST_DEFAULT && (o->item_cost < 0 || o->item_cost > HPC_ITEM_COST_MAX))
+    return fail(HPC_ERR_ARG, "item_cost must be HPC_ITEM_COST_DEFAULT or 0 .. %d", HPC_ITEM_COST_MAX);
+  if (o->e4m3_kernel != HPC_E4M3_MMA && o->e4m3_kernel != HPC_E4M3_TCGEN05)
+    return fail(HPC_ERR_ARG, "e4m3_kernel must be HPC_E4M3_MMA or HPC_E4M3_TCGEN05");
+  if (!single_launch && (o->item_cost != HPC_ITEM_COST_DEFAULT || o->record))
+    return fail(HPC_ERR_ARG, "item_cost and record apply to the single-launch steps only");
+  if (o->record && (o->record_items < 0 || (reinterpret_cast<uintptr_t>(o->record) & 15)))
+    return fail(HPC_ERR_ARG, "record needs record_items >= 0 and 16-byte alignment");
+#ifndef HPC_TRACE
+  if (o->trace) return fail(HPC_ERR_ARG, "a trace buffer needs a library built with HPC_TRACE");
+#endif
+  if (o->trace && (reinterpret_cast<uintptr_t>(o->trace) & 7)) return fail(HPC_ERR_ALIGN, "trace must be 8-byte aligned");
+  out->item_cost = o->item_cost;
+  out->tc = o->e4m3_kernel == HPC_E4M3_TCGEN05;
+  out->record = static_cast<uint8_t*>(o->record);
+  out->record_items = o->record ? o->record_items : 0;
+  out->trace = o->trace;
+  return HPC_OK;
+}
 
 // Checks shared by the attention entry points; fills the tensor maps, launch shape and the
 // common kernel parameters.
@@ -966,10 +1060,12 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
 }
 
 template <bool FUSED, bool PRO = false, bool MULTI = false>
-int dispatch(int head_dim, bool fp8, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
-             int smem, cudaStream_t st) {
-  if (fp8 && !PRO && !MULTI && e4m3_on_tensor_cores() && tc_supported(head_dim, fp8, prm.group, prm.q_len, PRO))
+int dispatch(int head_dim, bool fp8, bool tc, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm,
+             int grid, int smem, cudaStream_t st) {
+  if (fp8 && !PRO && !MULTI && tc && tc_supported(head_dim, fp8, prm.group, prm.q_len, PRO)) {
+    if (prm.trace) return fail(HPC_ERR_ARG, "the tcgen05 kernel writes no trace");
     return launch_attention_tc(FUSED, mk, mv, prm, grid, st);
+  }
   if (fp8) return launch<128, true, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
   if (head_dim == 128) return launch<128, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
   return launch<64, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
@@ -1000,8 +1096,11 @@ extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const vo
                                     int32_t page_size, int32_t num_heads, int32_t kv_heads, int32_t head_dim,
                                     const int32_t* block_table, int32_t max_pages_per_req, const int32_t* seq_lens,
                                     const hpc_plan* plan, float sm_scale, float* partial_o, float* partial_ml,
-                                    void* out, hpc_dtype out_dtype, uint32_t* status, void* stream) {
+                                    void* out, hpc_dtype out_dtype, const hpc_step_options* options,
+                                    uint32_t* status, void* stream) {
   if (!plan || !partial_o || !partial_ml) return fail(HPC_ERR_ARG, "null pointer argument");
+  Options opt;
+  if (int rc = read_options(options, false, &opt)) return rc;
   if (plan->kv_heads != kv_heads || plan->num_ctas < 1) return fail(HPC_ERR_ARG, "plan does not match kv_heads");
   if (!aligned16(partial_o)) return fail(HPC_ERR_ALIGN, "partial_o must be 16-byte aligned");
   CUtensorMap mk, mv;
@@ -1017,9 +1116,56 @@ extern "C" int hpc_decode_attention(const void* q, const void* k_pages, const vo
   prm.partial_o = partial_o;
   prm.partial_ml = partial_ml;
   prm.batch = plan->batch;
-  return dispatch<false>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, plan->num_ctas, ls.smem,
+  prm.trace = opt.trace;
+  return dispatch<false>(head_dim, kv_dtype == HPC_E4M3, opt.tc, mk, mv, prm, plan->num_ctas, ls.smem,
                          static_cast<cudaStream_t>(stream));
 }
+
+namespace hpc {
+
+int step_three_launch(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                      const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                      int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                      int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
+                      int32_t num_ctas, float sm_scale, void* out, hpc_dtype out_dtype, uint32_t* status,
+                      void* plan_workspace, size_t plan_bytes, float* partial_o, size_t partial_o_bytes,
+                      float* partial_ml, size_t partial_ml_bytes, void* stream) {
+  // every check first: the attention's (shapes, dtypes, alignment, the int32 token bound, the
+  // tensor maps and launch shape), then the planner's, then the scratch sizes
+  CUtensorMap mk, mv;
+  LaunchShape ls;
+  AttnParams prm;
+  int rc = prepare(q, k_pages, v_pages, kv_dtype, HPC_HND, k_scale, v_scale, num_pages, page_size, num_heads,
+                   kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, tile_len, num_ctas, true, sm_scale,
+                   out, out_dtype, status, &mk, &mv, &ls, &prm);
+  if (rc) return rc;
+  hpc_plan plan;
+  rc = check_plan_args(seq_lens, batch, num_heads, kv_heads, tile_len, num_ctas, plan_workspace, &plan, status);
+  if (rc) return rc;
+  const size_t need_plan = hpc_plan_workspace_bytes(batch, kv_heads, num_ctas);
+  const int64_t max_items = static_cast<int64_t>(num_ctas) + static_cast<int64_t>(batch) * kv_heads;
+  const size_t rows = static_cast<size_t>(max_items) * (num_heads / kv_heads);
+  if (!partial_o || !partial_ml) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (!aligned16(partial_o)) return fail(HPC_ERR_ALIGN, "partial_o must be 16-byte aligned");
+  if (need_plan == 0 || plan_bytes < need_plan || partial_o_bytes < rows * head_dim * sizeof(float) ||
+      partial_ml_bytes < rows * 2 * sizeof(float))
+    return fail(HPC_ERR_CAPACITY, "scratch too small for the plan or the partial states");
+  // max_pages_per_req * page_size fits int32 (checked by prepare)
+  rc = hpc_decode_plan(seq_lens, batch, num_heads, kv_heads, tile_len, num_ctas, prm.max_seq_len, plan_workspace,
+                       plan_bytes, &plan, status, stream);
+  if (rc) return rc;
+  prm.items = plan.items;
+  prm.cta_indptr = plan.cta_indptr;
+  prm.partial_o = partial_o;
+  prm.partial_ml = partial_ml;
+  prm.batch = batch;
+  rc = dispatch<false>(head_dim, kv_dtype == HPC_E4M3, false, mk, mv, prm, num_ctas, ls.smem,
+                       static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  return hpc_merge_states(partial_o, partial_ml, &plan, num_heads, head_dim, out, out_dtype, status, stream);
+}
+
+}  // namespace hpc
 
 extern "C" size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads, int32_t kv_heads,
                                                   int32_t head_dim, int32_t num_ctas) {
@@ -1046,15 +1192,11 @@ struct PrologueArgs {
 // %globaltimer stamps on B200 put that cost near the time a CTA takes to stream 152 KB of KV
 // at its share of HBM (one new token), and 224 KB with several new tokens, where the
 // consumers are the bound. A CTA that starts many items (many short requests) therefore gets
-// fewer tiles. HPC_ITEM_COST (integer, 1/16 tile) overrides it; 0 splits by tiles alone, the
-// pages' rule.
-int item_cost_units(int head_dim, bool fp8, int tile_len, int q_len) {
-  constexpr int64_t kMax = 64 * kCostPerTile;
-  const char* e = getenv("HPC_ITEM_COST");
-  if (e && *e) {
-    const long v = strtol(e, nullptr, 10);
-    return static_cast<int>(v < 0 ? 0 : (v > kMax ? kMax : v));
-  }
+// fewer tiles. A caller's options->item_cost (1/16 tile) replaces it; 0 splits by tiles alone,
+// the pages' rule.
+int item_cost_units(int head_dim, bool fp8, int tile_len, int q_len, int32_t requested) {
+  constexpr int64_t kMax = HPC_ITEM_COST_MAX;
+  if (requested != HPC_ITEM_COST_DEFAULT) return requested;  // checked to lie in 0 .. kMax
   const int64_t tile_bytes = static_cast<int64_t>(tile_len) * head_dim * 2 * (fp8 ? 1 : 2);
   const int64_t item_bytes = (q_len > 1 ? 224 : 152) * 1024;
   const int64_t c = (kCostPerTile * item_bytes + tile_bytes / 2) / tile_bytes;
@@ -1065,9 +1207,12 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
               const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size, int32_t num_heads,
               int32_t kv_heads, int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
               const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas, float sm_scale,
-              void* workspace, size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
-              void* stream, const PrologueArgs* pro, int32_t q_len = 1, float* lse = nullptr) {
+              void* workspace, size_t workspace_bytes, void* out, hpc_dtype out_dtype,
+              const hpc_step_options* options, uint32_t* status, void* stream, const PrologueArgs* pro,
+              int32_t q_len = 1, float* lse = nullptr) {
   if (!workspace) return fail(HPC_ERR_ARG, "null pointer argument");
+  Options opt;
+  if (int rc = read_options(options, true, &opt)) return rc;
   if (lse && (q_len != 1 || pro)) return fail(HPC_ERR_ARG, "the log-sum-exp output is for the one-token step");
   if (q_len < 1 || q_len > 4) return fail(HPC_ERR_SHAPE, "q_len must be 1 to 4");
   if (pro && q_len != 1) return fail(HPC_ERR_SHAPE, "the folded prologue takes one new token per request");
@@ -1096,13 +1241,16 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
   prm.batch = batch;
   prm.lse = lse;
-  prm.item_cost = item_cost_units(head_dim, kv_dtype == HPC_E4M3, tile_len, q_len);
+  prm.item_cost = item_cost_units(head_dim, kv_dtype == HPC_E4M3, tile_len, q_len, opt.item_cost);
+  prm.record = opt.record;
+  prm.record_items = opt.record_items;
+  prm.trace = opt.trace;
+  const bool fp8 = kv_dtype == HPC_E4M3;
   if (!pro && q_len > 1)
-    return dispatch<true, false, true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
+    return dispatch<true, false, true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem,
                                        static_cast<cudaStream_t>(stream));
   if (!pro)
-    return dispatch<true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
-                          static_cast<cudaStream_t>(stream));
+    return dispatch<true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem, static_cast<cudaStream_t>(stream));
   prm.qkv = static_cast<const __nv_bfloat16*>(pro->qkv);
   prm.q_norm_w = pro->q_norm_w;
   prm.k_norm_w = pro->k_norm_w;
@@ -1110,7 +1258,7 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.rope_theta = static_cast<double>(pro->rope_theta);
   prm.k_pages_w = const_cast<void*>(k_pages);
   prm.v_pages_w = const_cast<void*>(v_pages);
-  return dispatch<true, true>(head_dim, kv_dtype == HPC_E4M3, mk, mv, prm, num_ctas, ls.smem,
+  return dispatch<true, true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem,
                               static_cast<cudaStream_t>(stream));
 }
 
@@ -1122,10 +1270,11 @@ extern "C" int hpc_decode_step(const void* q, const void* k_pages, const void* v
                                int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                                int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
                                int32_t num_ctas, float sm_scale, void* workspace, size_t workspace_bytes, void* out,
-                               hpc_dtype out_dtype, uint32_t* status, void* stream) {
+                               hpc_dtype out_dtype, const hpc_step_options* options, uint32_t* status,
+                               void* stream) {
   return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
-                   workspace, workspace_bytes, out, out_dtype, status, stream, nullptr);
+                   workspace, workspace_bytes, out, out_dtype, options, status, stream, nullptr);
 }
 
 extern "C" int hpc_decode_step_lse(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
@@ -1134,11 +1283,12 @@ extern "C" int hpc_decode_step_lse(const void* q, const void* k_pages, const voi
                                    int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
                                    const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
                                    float sm_scale, void* workspace, size_t workspace_bytes, void* out,
-                                   hpc_dtype out_dtype, float* lse, uint32_t* status, void* stream) {
+                                   hpc_dtype out_dtype, float* lse, const hpc_step_options* options,
+                                   uint32_t* status, void* stream) {
   if (!lse) return fail(HPC_ERR_ARG, "null pointer argument");
   return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
-                   workspace, workspace_bytes, out, out_dtype, status, stream, nullptr, 1, lse);
+                   workspace, workspace_bytes, out, out_dtype, options, status, stream, nullptr, 1, lse);
 }
 
 extern "C" size_t hpc_decode_step_multi_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_heads,
@@ -1154,11 +1304,11 @@ extern "C" int hpc_decode_step_multi(const void* q, int32_t q_len, const void* k
                                      int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
                                      int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch,
                                      int32_t tile_len, int32_t num_ctas, float sm_scale, void* workspace,
-                                     size_t workspace_bytes, void* out, hpc_dtype out_dtype, uint32_t* status,
-                                     void* stream) {
+                                     size_t workspace_bytes, void* out, hpc_dtype out_dtype,
+                                     const hpc_step_options* options, uint32_t* status, void* stream) {
   return step_impl(q, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
-                   workspace, workspace_bytes, out, out_dtype, status, stream, nullptr, q_len);
+                   workspace, workspace_bytes, out, out_dtype, options, status, stream, nullptr, q_len);
 }
 
 extern "C" int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, const float* k_norm_w, float eps,
@@ -1168,11 +1318,12 @@ extern "C" int hpc_decode_step_prologue(const void* qkv, const float* q_norm_w, 
                                         int32_t head_dim, const int32_t* block_table, int32_t max_pages_per_req,
                                         const int32_t* seq_lens, int32_t batch, int32_t tile_len, int32_t num_ctas,
                                         float sm_scale, void* workspace, size_t workspace_bytes, void* out,
-                                        hpc_dtype out_dtype, uint32_t* status, void* stream) {
+                                        hpc_dtype out_dtype, const hpc_step_options* options, uint32_t* status,
+                                        void* stream) {
   if (!qkv || !q_norm_w || !k_norm_w) return fail(HPC_ERR_ARG, "null pointer argument");
   if (!(rope_theta > 0.f) || !(eps >= 0.f)) return fail(HPC_ERR_ARG, "rope_theta must be > 0 and eps >= 0");
   const PrologueArgs pro{qkv, q_norm_w, k_norm_w, eps, rope_theta};
   return step_impl(qkv, k_pages, v_pages, kv_dtype, kv_layout, k_scale, v_scale, num_pages, page_size, num_heads,
                    kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len, num_ctas, sm_scale,
-                   workspace, workspace_bytes, out, out_dtype, status, stream, &pro);
+                   workspace, workspace_bytes, out, out_dtype, options, status, stream, &pro);
 }

@@ -58,7 +58,16 @@ struct AttnParams {
   void* v_pages_w;
   float eps;
   double rope_theta;
+  // single-launch step, on request: each CTA's record of its split (hpc_cta_record + items)
+  uint8_t* record;
+  int32_t record_items;
+  uint64_t* trace;  // HPC_TRACE builds: [grid][HPC_TRACE_WORDS] timestamps and counts
 };
+
+// Byte stride of one CTA's record: the header, then record_items work items.
+__host__ __device__ __forceinline__ size_t record_stride(int record_items) {
+  return sizeof(hpc_cta_record) + static_cast<size_t>(record_items) * sizeof(hpc_work_item);
+}
 
 // One work item as the producer and the consumers see it.
 struct ItemInfo {
@@ -189,6 +198,33 @@ template <>
 struct CursorOf<true> {
   using type = WalkCursor;
 };
+
+// The k-th item of CTA g's record (single-launch step, when a record buffer is given): the item
+// as the planner would list it, with HPC_ITEM_SECOND_SLOT for a split item in slot 2g + 1.
+__device__ __forceinline__ void record_item(const AttnParams& p, int64_t k, const ItemInfo& x) {
+  if (k >= p.record_items) return;
+  hpc_work_item w;
+  w.req = x.req;
+  w.kv_head = static_cast<int16_t>(x.kvh);
+  w.flags = static_cast<int16_t>(x.direct ? HPC_ITEM_DIRECT : ((x.slot & 1) ? HPC_ITEM_SECOND_SLOT : 0));
+  w.tile_begin = static_cast<int32_t>(x.tok0 / p.tile_len);
+  // tok1 = min(te * tile_len, L), and only the segment's last tile is clipped: te = ceil(tok1 / tile_len)
+  w.tile_end = static_cast<int32_t>((x.tok1 + p.tile_len - 1) / p.tile_len);
+  uint8_t* rec = p.record + static_cast<size_t>(blockIdx.x) * record_stride(p.record_items);
+  reinterpret_cast<hpc_work_item*>(rec + sizeof(hpc_cta_record))[k] = w;
+}
+
+// CTA g's record header: its unit run, the chunk and cost of the split, and its item count.
+__device__ __forceinline__ void record_header(const AttnParams& p, int64_t u0, int64_t u1, int64_t chunk,
+                                              int64_t n_items) {
+  hpc_cta_record h;
+  h.unit_begin = u0;
+  h.unit_end = u1;
+  h.chunk = chunk;
+  h.item_cost = p.item_cost;
+  h.n_items = static_cast<int32_t>(n_items);
+  *reinterpret_cast<hpc_cta_record*>(p.record + static_cast<size_t>(blockIdx.x) * record_stride(p.record_items)) = h;
+}
 
 // Where the single-launch step's split puts a unit. Unit u (tile t of segment S, the S-th
 // (request, kv head) with tiles, 1-based) sits at cost position W*u + c*S: every tile costs
@@ -380,7 +416,7 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
       float M = -INFINITY;
       for (int i = 0; i < n; ++i) M = fmaxf(M, s_m[i * grp + tid]);
       float L = 0.f;
-      for (int i = 0; i < n; ++i) L += expf(s_m[i * grp + tid] - M) * s_w[i * grp + tid];
+      for (int i = 0; i < n && M != -INFINITY; ++i) L += expf(s_m[i * grp + tid] - M) * s_w[i * grp + tid];
       s_M[tid] = M;
       s_iL[tid] = L > 0.f ? 1.f / L : 0.f;
       if (p.lse) {  // one new token per request: row tid is head kvh * group + tid
@@ -390,7 +426,7 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
     named_barrier_sync(1, nthr);
     for (int k = tid; k < n * grp; k += nthr) {
       const int h = k % grp;
-      s_w[k] = expf(s_m[k] - s_M[h]) * s_iL[h];
+      s_w[k] = s_iL[h] > 0.f ? expf(s_m[k] - s_M[h]) * s_iL[h] : 0.f;  // no live piece: zeros
     }
     named_barrier_sync(1, nthr);
     for (int idx = tid; idx < grp * D; idx += nthr) {
@@ -416,7 +452,7 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
     float M = -INFINITY;
     for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(p.partial_ml + 2 * (slot_of(i) * grp + h)));
     float Ls = 0.f, acc = 0.f;
-    for (int i = 0; i < n; ++i) {
+    for (int i = 0; i < n && M != -INFINITY; ++i) {
       const int64_t pi = slot_of(i) * grp + h;
       const float e = expf(__ldcg(p.partial_ml + 2 * pi) - M);
       Ls += e * __ldcg(p.partial_ml + 2 * pi + 1);
@@ -428,15 +464,6 @@ __device__ void merge_segment(const AttnParams& p, const ItemInfo& x, int64_t ch
     if (p.lse && idx - h * D == 0)
       p.lse[static_cast<int64_t>(x.req) * p.num_heads + x.kvh * p.group + h] = Ls > 0.f ? M + logf(Ls) : -INFINITY;
   }
-}
-
-// E4M3 caches run on the mma.sync kernel; HPC_E4M3_TCGEN05=1 in the environment selects the
-// tcgen05 kernel (attention_tc.cu) where it applies. Measured on the large-batch E4M3 workload
-// the mma.sync kernel is the faster one (775 against 1278 us per step): with N = 16 per product
-// and 128 tokens per stage, the tcgen05 pipeline is bound by its per-stage round trips.
-inline bool e4m3_on_tensor_cores() {
-  const char* e = getenv("HPC_E4M3_TCGEN05");
-  return e && e[0] == '1';
 }
 
 // The tcgen05 kernel for E4M3 caches (attention_tc.cu). It serves the one-token single-launch

@@ -13,7 +13,9 @@
 // Roles (320 threads):
 //  * warp 9, producer: streams 128-token stages (K then V, 16 KB each) into a ring by TMA,
 //    as the mma.sync kernel does, in boxes of up to 64 tokens that never cross a page.
-//    Boxes past an item's last token read an out-of-range page, which TMA fills with zeros.
+//    Boxes past an item's last token are not loaded: their rows hold whatever the slot held
+//    before, and the softmax masks those tokens and zeroes their V rows. A page id outside the
+//    pool is never handed to TMA either: page 0 stands in, and the box's tokens are masked.
 //  * warp 8, one lane issues the products. Per stage n:
 //      S^T[128 tokens x 16] = K[128 x 128] . Qhl^T          (tensor memory, buffer n % 2)
 //      O^T[128 d x 16]      = V^T[128 x 128 tokens] . Phl    (tensor memory, buffer n % 2)
@@ -155,6 +157,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ float s_qmax[4];                      // q amax of the warpgroup that writes Qhl
   __shared__ float s_sq[2];                        // q scale of each Qhl buffer
   __shared__ float s_xm[8], s_xl[8];               // warpgroup 1's (m, l) at an item end
+  __shared__ uint8_t s_badbox[16];                 // per ring slot: boxes whose page id was out of range
+  __shared__ int s_rec_n;                          // items this CTA has run (single-launch record)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stages = p.stages;
   uint8_t* ring = smem;
@@ -166,6 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t ring_u32 = smem_u32(ring);
 
   if (threadIdx.x == 0) {
+    s_rec_n = 0;
     for (int s = 0; s < stages; ++s) {
       mbar_init(bar.full(s), 1);
       mbar_init(bar.empty(s), 1);
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int64_t cb = 0; cb < nbox && ok; cb += 32) {
         const int nk = static_cast<int>(nbox - cb < 32 ? nbox - cb : 32);
         __syncwarp();
-        if (lane < nk) s_pages[lane] = cb + lane < nreal ? bt[(off0 + (cb + lane) * C) >> p_shift] : p.num_pages;
+        if (lane < nk) s_pages[lane] = cb + lane < nreal ? bt[(off0 + (cb + lane) * C) >> p_shift] : 0;
         __syncwarp();
         if (lane == 0) {
           for (int k = 0; k < nk; ++k) {
@@ -237,15 +242,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 bad |= HPC_DEV_TIMEOUT;
                 break;
               }
-              mbar_arrive_expect_tx(bar.full(slot), kTcStage);
+              // boxes of this stage that hold item tokens (the stage's boxes lie in this batch
+              // of page ids, as cps divides 32), and those whose page id is out of range
+              const int nb = static_cast<int>(nreal - bi < cps ? nreal - bi : cps);
+              uint32_t mask = 0;
+              for (int kk = 0; kk < nb; ++kk) {
+                const int32_t pg = s_pages[k + kk];
+                if (pg < 0 || pg >= p.num_pages) mask |= 1u << kk;
+              }
+              if (mask) bad |= HPC_DEV_BAD_PAGE;
+              s_badbox[slot] = static_cast<uint8_t>(mask);
+              mbar_arrive_expect_tx(bar.full(slot), static_cast<uint32_t>(nb) * 2u * C * 128u);
             }
-            const int32_t page = s_pages[k];
-            if (bi < nreal && (page < 0 || page >= p.num_pages)) bad |= HPC_DEV_BAD_PAGE;  // zeros are read there
-            const int off = static_cast<int>((off0 + bi * C) & (P - 1));
-            const int c1 = p.nhd ? x.kvh : off, c2 = p.nhd ? off : x.kvh;
-            const uint32_t dst = ring_u32 + slot * kTcStage + kc * C * 128;
-            tma_load_4d(dst, &tm_k, bar.full(slot), 0, c1, c2, page, policy);
-            tma_load_4d(dst + kTcHalf, &tm_v, bar.full(slot), 0, c1, c2, page, policy);
+            if (bi < nreal) {
+              int32_t page = s_pages[k];
+              if (page < 0 || page >= p.num_pages) page = 0;  // stand-in; the softmax masks the box
+              const int off = static_cast<int>((off0 + bi * C) & (P - 1));
+              const int c1 = p.nhd ? x.kvh : off, c2 = p.nhd ? off : x.kvh;
+              const uint32_t dst = ring_u32 + slot * kTcStage + kc * C * 128;
+              tma_load_4d(dst, &tm_k, bar.full(slot), 0, c1, c2, page, policy);
+              tma_load_4d(dst + kTcHalf, &tm_v, bar.full(slot), 0, c1, c2, page, policy);
+            }
             if (kc == cps - 1) {
               ++issued;
               if (++slot == stages) {
@@ -427,6 +444,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (w == 0 && have) build_q(x, 0);
     while (have) {
       const int kvh = x.kvh, head0 = kvh * p.group;
+      if (w == 0 && i == 0) {
+        if (FUSED && p.record) record_item(p, s_rec_n, x);
+        ++s_rec_n;
+      }
       const int64_t nst = stages_of(x);
       const int64_t n0 = n, n_end = n + nst;
       // the next item's Qhl is written right after warpgroup 0's last P of this item, so that
@@ -479,8 +500,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar.s_free(b));
+        // boxes with an out-of-range page id: the producer wrote the mask before the fill's
+        // arrive; this wait on the fill (already complete, since the S^T product read it) makes
+        // the mask visible. The slot cannot be refilled before this stage's P is written.
+        uint32_t badm = 0;
+        if (wait(bar.full(static_cast<int>(k % stages)), static_cast<uint32_t>((k / stages) & 1)))
+          badm = s_badbox[k % stages];
         const int64_t t = x.tok0 + (k - n0) * kTcTok + i;
-        const bool valid = t < x.tok1;
+        const bool valid = t < x.tok1 && !((badm >> (i / C)) & 1u);
         if (!valid) {
           // this token's V row may hold anything (even NaN codes): zero it, so 0 * v stays 0
           uint4* vrow = reinterpret_cast<uint4*>(ring + static_cast<size_t>(k % stages) * kTcStage + kTcHalf + i * 128);
@@ -493,9 +520,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         wg_reduce8<true>(sc, mx, s_red[w][(k >> 1) & 1], wq, lane, wbar);
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
-          const float mn = fmaxf(m_run[h], mx[h]);  // finite: every stage holds a live token
-          a[h] = exp2f(m_run[h] - mn);
-          pv[h] = exp2f(sc[h] - mn + 8.f);
+          const float mn = fmaxf(m_run[h], mx[h]);
+          const float mr = mn == -INFINITY ? 0.f : mn;  // no live token yet (bad pages): adds nothing
+          a[h] = exp2f(m_run[h] - mr);
+          pv[h] = exp2f(sc[h] - mr + 8.f);
           l_part[h] = l_part[h] * a[h] + pv[h];
           m_run[h] = mn;
         }
@@ -543,7 +571,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (h >= p.group) break;
           // a warpgroup without stages in this item has m = -inf and weighs 0
           const float m1 = s_xm[h], M = fmaxf(m_run[h], m1);
-          const float f0 = exp2f(m_run[h] - M), f1 = exp2f(m1 - M);
+          const float Mr = M == -INFINITY ? 0.f : M;  // neither warpgroup saw a live token
+          const float f0 = exp2f(m_run[h] - Mr), f1 = exp2f(m1 - Mr);
           const float Lh = L[h] * f0 + s_xl[h] * f1;
           const float oh = o_acc[h] * f0 + xo[i * 8 + h] * f1;
           if (x.direct) {
@@ -590,6 +619,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       named_barrier_sync(3, 2 * kSoftmax);  // the exchange, merge and scratch buffers are reused
       ++j;
       have = cursor.next(p, x);
+    }
+    if constexpr (FUSED) {
+      // s_walk still holds this CTA's unit run and the chunk from plan_in_kernel
+      if (p.record && w == 0 && i == 0) record_header(p, s_walk[0], s_walk[1], s_walk[7], s_rec_n);
     }
   }
 

@@ -28,6 +28,21 @@ struct PlanLayout {
 };
 PlanLayout plan_layout(int32_t batch, int32_t kv_heads, int32_t num_ctas, int32_t max_items);
 
+// Host checks of hpc_decode_plan's arguments (nothing is launched).
+int check_plan_args(const void* seq_lens, int32_t batch, int32_t num_heads, int32_t kv_heads, int32_t tile_len,
+                    int32_t ctas, const void* workspace, const void* plan, const void* status);
+
+// plan -> attention -> merge for one decode step (HND cache, default options) over scratch the
+// caller hands in: the plan workspace and the partial states. Every host check of the three
+// calls runs before the first launch, so a non-zero return means nothing was launched.
+int step_three_launch(const void* q, const void* k_pages, const void* v_pages, hpc_dtype kv_dtype,
+                      const float* k_scale, const float* v_scale, int32_t num_pages, int32_t page_size,
+                      int32_t num_heads, int32_t kv_heads, int32_t head_dim, const int32_t* block_table,
+                      int32_t max_pages_per_req, const int32_t* seq_lens, int32_t batch, int32_t tile_len,
+                      int32_t num_ctas, float sm_scale, void* out, hpc_dtype out_dtype, uint32_t* status,
+                      void* plan_workspace, size_t plan_bytes, float* partial_o, size_t partial_o_bytes,
+                      float* partial_ml, size_t partial_ml_bytes, void* stream);
+
 // Launch with programmatic dependent launch (PDL) allowed: the kernel may start while the
 // previous kernel on the stream is still running. It must call pdl_wait() before touching
 // memory that earlier work on the stream reads or writes.

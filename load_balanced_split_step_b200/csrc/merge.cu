@@ -50,15 +50,15 @@ __global__ void __launch_bounds__(kMergeThreads)
         const int h = threadIdx.x;
         float M = -INFINITY;
         for (int i = 0; i < n; ++i) M = fmaxf(M, s_m[i * group + h]);
-        float L = 0.f;
-        for (int i = 0; i < n; ++i) L += expf(s_m[i * group + h] - M) * s_w[i * group + h];
+        float L = 0.f;  // M = -inf: no part saw a live token (bad pages); the row is zero
+        for (int i = 0; i < n && M != -INFINITY; ++i) L += expf(s_m[i * group + h] - M) * s_w[i * group + h];
         s_M[h] = M;
         s_invL[h] = L > 0.f ? 1.f / L : 0.f;
       }
       __syncthreads();
       for (int k = threadIdx.x; k < n * group; k += blockDim.x) {
         const int h = k % group;
-        s_w[k] = expf(s_m[k] - s_M[h]) * s_invL[h];
+        s_w[k] = s_invL[h] > 0.f ? expf(s_m[k] - s_M[h]) * s_invL[h] : 0.f;
       }
       __syncthreads();
       const float* po = partial_o + static_cast<int64_t>(i0) * group * head_dim;
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         float M = -INFINITY;
         for (int i = i0; i < i1; ++i) M = fmaxf(M, partial_ml[2 * (static_cast<int64_t>(i) * group + h)]);
         float L = 0.f, acc = 0.f;
-        for (int i = i0; i < i1; ++i) {
+        for (int i = i0; i < i1 && M != -INFINITY; ++i) {
           const int64_t pi = static_cast<int64_t>(i) * group + h;
           const float e = expf(partial_ml[2 * pi] - M);
           L += e * partial_ml[2 * pi + 1];

@@ -19,10 +19,12 @@
 //    to start at zero: the planner rewrites every plan field on each call, and a partial
 //    slot is always written before it is read. Calls that overlap on the GPU race on the
 //    array. Issue them on one stream, or order them with events.
-//  * Host code cannot use the array's name as a device address. The first call on each
-//    device, with that device current, asks the runtime for the address
-//    (cudaGetSymbolAddress) and caches it. Make that first call before any stream
-//    capture begins.
+//  * Host code cannot use the array's name as a device address. The first call in each CUDA
+//    context (per device, and again after that device's context was reset and recreated) asks
+//    the runtime for the address (cudaGetSymbolAddress) with that device current, and caches
+//    it under the context's unique id. Make that first call before any stream capture begins.
+//  * Every host check (shapes, dtypes, alignment, sizes, the stream's device) runs before the
+//    first of the three launches, so a non-zero return means nothing was launched.
 #include <mutex>
 
 #include "hpc_common.cuh"
@@ -34,20 +36,57 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[HPC_NOALLOC_SCR
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};  // unique id of the context the address belongs to
 
-// Device address of g_noalloc_scratch on the current device (set-up on first use).
-int scratch_address(void** out) {
+// Unique id of the current CUDA context (never reused within the process), or 0 if the driver
+// does not report one; then the cache is keyed on the device ordinal alone.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch in the current context (looked up on first use there).
+// The stream must belong to the current device: the address is only valid in its context.
+int scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return hpc::fail(HPC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return hpc::fail(HPC_ERR_ARG, "device ordinal %d out of range", dev);
+  if (stream) {
+    int sdev = -1;
+    e = cudaStreamGetDevice(stream, &sdev);
+    if (e != cudaSuccess) return hpc::fail(HPC_ERR_CUDA, "cudaStreamGetDevice: %s", cudaGetErrorString(e));
+    if (sdev != dev)
+      return hpc::fail(HPC_ERR_ARG, "the stream belongs to device %d but device %d is current", sdev, dev);
+  }
+  // the caller's buffers live in the current context, so it exists (no cudaFree(0) here: that
+  // call is not allowed while a stream is being captured)
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return hpc::fail(HPC_ERR_CUDA, "cudaGetSymbolAddress(g_noalloc_scratch): %s", cudaGetErrorString(e));
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return HPC_OK;
@@ -67,6 +106,9 @@ extern "C" int hpc_decode_step_noalloc(const void* q, const void* k_pages, const
   if (batch < 1 || kv_heads < 1 || num_heads < 1 || num_ctas < 1 || head_dim < 1)
     return hpc::fail(HPC_ERR_ARG, "batch, heads, head_dim and num_ctas must be >= 1");
   if (num_heads % kv_heads) return hpc::fail(HPC_ERR_SHAPE, "num_heads %% kv_heads != 0");
+  if (max_pages_per_req < 1 || page_size < 1 ||
+      static_cast<int64_t>(max_pages_per_req) * static_cast<int64_t>(page_size) > INT32_MAX)
+    return hpc::fail(HPC_ERR_SHAPE, "max_pages_per_req * page_size must lie in 1 .. INT32_MAX");
   const size_t plan_bytes = hpc_plan_workspace_bytes(batch, kv_heads, num_ctas);
   if (plan_bytes == 0) return hpc::fail(HPC_ERR_ARG, "bad plan shape");
   const size_t max_items = static_cast<size_t>(num_ctas) + static_cast<size_t>(batch) * kv_heads;
@@ -80,20 +122,13 @@ extern "C" int hpc_decode_step_noalloc(const void* q, const void* k_pages, const
                      "use the entry points with caller-owned buffers",
                      need, static_cast<size_t>(HPC_NOALLOC_SCRATCH_BYTES));
   void* base = nullptr;
-  int rc = scratch_address(&base);
+  int rc = scratch_address(static_cast<cudaStream_t>(stream), &base);
   if (rc) return rc;
   char* s = static_cast<char*>(base);
-  void* plan_ws = s;
   float* partial_o = reinterpret_cast<float*>(s + up256(plan_bytes));
   float* partial_ml = reinterpret_cast<float*>(s + up256(plan_bytes) + up256(po_bytes));
-
-  hpc_plan plan;
-  rc = hpc_decode_plan(seq_lens, batch, num_heads, kv_heads, tile_len, num_ctas, max_pages_per_req * page_size,
-                       plan_ws, plan_bytes, &plan, status, stream);
-  if (rc) return rc;
-  rc = hpc_decode_attention(q, k_pages, v_pages, kv_dtype, HPC_HND, k_scale, v_scale, num_pages, page_size, num_heads,
-                            kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, &plan, sm_scale, partial_o,
-                            partial_ml, out, out_dtype, status, stream);
-  if (rc) return rc;
-  return hpc_merge_states(partial_o, partial_ml, &plan, num_heads, head_dim, out, out_dtype, status, stream);
+  return hpc::step_three_launch(q, k_pages, v_pages, kv_dtype, k_scale, v_scale, num_pages, page_size, num_heads,
+                                kv_heads, head_dim, block_table, max_pages_per_req, seq_lens, batch, tile_len,
+                                num_ctas, sm_scale, out, out_dtype, status, s, plan_bytes, partial_o, po_bytes,
+                                partial_ml, pml_bytes, stream);
 }

@@ -259,6 +259,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+}  // namespace
+
 int check_plan_args(const void* seq_lens, int32_t batch, int32_t num_heads, int32_t kv_heads, int32_t tile_len,
                     int32_t ctas, const void* workspace, const void* plan, const void* status) {
   if (!seq_lens || !workspace || !plan || !status) return fail(HPC_ERR_ARG, "null pointer argument");
@@ -272,6 +274,8 @@ int check_plan_args(const void* seq_lens, int32_t batch, int32_t num_heads, int3
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return fail(HPC_ERR_ALIGN, "workspace must be 256-byte aligned");
   return HPC_OK;
 }
+
+namespace {
 
 void bind_plan(void* ws, const PlanLayout& L, int32_t batch, int32_t kv_heads, int32_t tile_len, int32_t ctas,
                int32_t max_items, int32_t is_static, hpc_plan* plan) {

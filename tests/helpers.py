@@ -25,13 +25,13 @@ def to_device(case: W.DecodeCase, dev="cuda") -> dict:
 
 
 def run_attention(B, spec, dc, seq_lens=None, num_ctas=None, out_dtype=torch.float32, static_splits=None,
-                  q=None, tile_len=None):
+                  q=None, tile_len=None, e4m3_kernel="mma"):
     """plan -> attention -> merge through the binding. Returns (out, plan, status int)."""
     seq = dc["seq_lens"] if seq_lens is None else seq_lens
     out, p, st = B.decode_step(dc["q"] if q is None else q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq,
                                spec.num_heads, spec.kv_heads, tile_len or spec.tile_len, kv_dtype=spec.kv_dtype,
                                k_scale=dc["k_scale"], v_scale=dc["v_scale"], num_ctas=num_ctas,
-                               out_dtype=out_dtype, static_splits=static_splits)
+                               out_dtype=out_dtype, static_splits=static_splits, e4m3_kernel=e4m3_kernel)
     torch.cuda.synchronize()
     return out, p, int(st.item())
 

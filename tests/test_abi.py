@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 7
+    assert B._lib.hpc_abi_version() == 8
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -55,7 +55,7 @@ def test_host_argument_errors_return_codes(B):
     i32 = ctypes.c_int32
     # null pointers -> HPC_ERR_ARG before any CUDA call
     rc = B._lib.hpc_decode_attention(None, None, None, 0, 0, None, None, 1, 16, 8, 2, 64, None, 1, None,
-                                     ctypes.byref(P), 0.1, None, None, None, 1, None, None)
+                                     ctypes.byref(P), 0.1, None, None, None, 1, None, None, None)
     assert rc == B.HPC_ERR_ARG
     assert "null" in B._lib.hpc_last_error().decode()
     rc = B._lib.hpc_merge_states(None, None, ctypes.byref(P), 8, 64, None, 1, None, None)
@@ -63,22 +63,22 @@ def test_host_argument_errors_return_codes(B):
     # the single-launch step with the folded prologue: null qkv / norm weights, bad theta
     i32 = ctypes.c_int32
     rc = B._lib.hpc_decode_step_prologue(None, None, None, 1e-6, 1e6, None, None, 0, 0, None, None, 1, 16, 8, 2, 64,
-                                         None, 1, None, 1, 32, 4, 0.1, None, 0, None, 1, None, None)
+                                         None, 1, None, 1, 32, 4, 0.1, None, 0, None, 1, None, None, None)
     assert rc == B.HPC_ERR_ARG
     w = ctypes.c_void_p(16)  # never dereferenced: the argument checks fail first
     rc = B._lib.hpc_decode_step_prologue(w, w, w, 1e-6, -1.0, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1,
-                                         32, 4, 0.1, w, 0, w, 1, w, None)
+                                         32, 4, 0.1, w, 0, w, 1, None, w, None)
     assert rc == B.HPC_ERR_ARG and "rope_theta" in B._lib.hpc_last_error().decode()
     # several new tokens: q_len outside 1..4 and zero-size workspace queries
     rc = B._lib.hpc_decode_step_multi(w, 5, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1, 32, 4, 0.1, w, 1 << 20,
-                                      w, 1, w, None)
+                                      w, 1, None, w, None)
     assert rc == B.HPC_ERR_SHAPE and "q_len" in B._lib.hpc_last_error().decode()
     assert B._lib.hpc_decode_step_multi_workspace_bytes(4, 0, 8, 2, 64, 148) == 0
     assert (B._lib.hpc_decode_step_multi_workspace_bytes(4, 1, 8, 2, 64, 148)
             == B._lib.hpc_decode_step_workspace_bytes(4, 8, 2, 64, 148))
     # log-sum-exp step and merge: null outputs, bad sizes
     rc = B._lib.hpc_decode_step_lse(w, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1, 32, 4, 0.1, w, 1 << 20, w,
-                                    1, None, w, None)
+                                    1, None, None, w, None)
     assert rc == B.HPC_ERR_ARG
     assert B._lib.hpc_merge_lse(None, None, 2, 10, 64, None, None, None) == B.HPC_ERR_ARG
     assert B._lib.hpc_merge_lse(w, w, 0, 10, 64, w, None, None) == B.HPC_ERR_ARG
@@ -103,6 +103,59 @@ def test_host_argument_errors_return_codes(B):
     with pytest.raises(B.HpcError, match="num_heads"):
         B.plan_host(lens, 7, 2, 32, 4)
     assert B._lib.hpc_plan_workspace_bytes(0, 2, 4) == 0
+
+
+def test_options_are_checked_before_any_launch(B):
+    """Per-call options (ABI 8): out-of-range values, options that belong to the single-launch
+    step passed to the three-launch attention, and a trace buffer in a build without HPC_TRACE
+    all return HPC_ERR_ARG before any CUDA call (the pointers are never dereferenced)."""
+    w = ctypes.c_void_p(256)
+    P = B.CPlan()
+    P.kv_heads, P.num_ctas, P.tile_len = 2, 4, 32
+
+    def step(opt):
+        return B._lib.hpc_decode_step(w, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, 1, 32, 4, 0.1, w, 1 << 20,
+                                      w, 1, None if opt is None else ctypes.byref(opt), w, None)
+
+    def attention(opt):
+        return B._lib.hpc_decode_attention(w, w, w, 0, 0, None, None, 1, 16, 8, 2, 64, w, 1, w, ctypes.byref(P), 0.1,
+                                           w, w, w, 1, ctypes.byref(opt), w, None)
+
+    for kw, what in ((dict(item_cost=-2), "item_cost"), (dict(item_cost=B.ITEM_COST_MAX + 1), "item_cost"),
+                     (dict(e4m3_kernel="tcgen05"), None)):
+        o = B.options(**kw)
+        if what is None:
+            o.e4m3_kernel = 7
+            what = "e4m3_kernel"
+        assert step(o) == B.HPC_ERR_ARG and what in B._lib.hpc_last_error().decode()
+    o = B.options(item_cost=0)
+    assert attention(o) == B.HPC_ERR_ARG and "single-launch" in B._lib.hpc_last_error().decode()
+    o = B.COptions(B.ITEM_COST_DEFAULT, 0, None, 0, 0, 4096)
+    assert not (B.build_flags() & B.BUILD_TRACE)
+    assert step(o) == B.HPC_ERR_ARG and "HPC_TRACE" in B._lib.hpc_last_error().decode()
+    assert attention(o) == B.HPC_ERR_ARG
+    o = B.COptions(B.ITEM_COST_DEFAULT, 0, 24, 4, 0, None)  # a record buffer that is not 16-byte aligned
+    assert step(o) == B.HPC_ERR_ARG and "record" in B._lib.hpc_last_error().decode()
+    assert B._lib.hpc_step_record_bytes(148, 4) == 148 * (32 + 4 * 16)
+    assert B._lib.hpc_step_record_bytes(0, 4) == 0
+
+
+def test_noalloc_size_checks_come_first(B):
+    """The entry point without caller scratch rejects bad sizes, a token count beyond int32
+    (computed in 64 bits) and shapes too big for its array before any CUDA call."""
+    w = ctypes.c_void_p(256)
+
+    def call(num_pages=8, page_size=16, num_heads=8, kv_heads=2, head_dim=64, max_pages=4, batch=3, tile_len=32,
+             num_ctas=4):
+        return B._lib.hpc_decode_step_noalloc(w, w, w, 0, None, None, num_pages, page_size, num_heads, kv_heads,
+                                              head_dim, w, max_pages, w, batch, tile_len, num_ctas, 0.1, w, 1, w, None)
+
+    assert call(batch=0) == B.HPC_ERR_ARG
+    assert call(num_heads=7) == B.HPC_ERR_SHAPE
+    assert call(max_pages=1 << 20, page_size=1 << 12) == B.HPC_ERR_SHAPE  # 2^32 tokens: no int32 wrap
+    assert "INT32_MAX" in B._lib.hpc_last_error().decode()
+    assert call(max_pages=0) == B.HPC_ERR_SHAPE
+    assert call(batch=100000, kv_heads=8, num_heads=64, head_dim=128) == B.HPC_ERR_CAPACITY
 
 
 def test_launch_info(B):

@@ -2,7 +2,6 @@
 element (several tiles, ragged tails, every supported shape), the named workloads at full
 size on sampled requests, plus invariances (page permutation, run-to-run determinism,
 plan choice) and edge cases (L = 1, L = 0, NaN in unused slots, bad page ids)."""
-import os
 
 import numpy as np
 import pytest
@@ -68,48 +67,41 @@ def test_e4m3_shapes_ragged(B, Hq, Hkv, P, tl, consumer):
     spec, case = _case(lens, Hq, Hkv, 128, P, tl, seed=Hq + P + tl, kv="e4m3")
     dc = to_device(case)
     ref = oracle_out(case)
-    if consumer == "tcgen05":
-        os.environ["HPC_E4M3_TCGEN05"] = "1"
-    try:
-        for G in (5, 148):
-            out, _, st = run_attention(B, spec, dc, num_ctas=G)
-            assert st == 0
-            mx, _ = errors(out, ref)
-            assert mx <= 5e-2, (consumer, Hq, Hkv, P, tl, G, mx)
-            out, st_t, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
-                                               dc["seq_lens"], Hq, Hkv, tl, kv_dtype="e4m3", k_scale=dc["k_scale"],
-                                               v_scale=dc["v_scale"], num_ctas=G)
-            torch.cuda.synchronize()
-            assert int(st_t.item()) == 0
-            mx, _ = errors(out, ref)
-            assert mx <= 5e-2, (consumer, "fused", Hq, Hkv, P, tl, G, mx)
-    finally:
-        os.environ.pop("HPC_E4M3_TCGEN05", None)
+    kernel = "tcgen05" if consumer == "tcgen05" else "mma"
+    for G in (5, 148):
+        out, _, st = run_attention(B, spec, dc, num_ctas=G, e4m3_kernel=kernel)
+        assert st == 0
+        mx, _ = errors(out, ref)
+        assert mx <= 5e-2, (consumer, Hq, Hkv, P, tl, G, mx)
+        out, st_t, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
+                                           dc["seq_lens"], Hq, Hkv, tl, kv_dtype="e4m3", k_scale=dc["k_scale"],
+                                           v_scale=dc["v_scale"], num_ctas=G, e4m3_kernel=kernel)
+        torch.cuda.synchronize()
+        assert int(st_t.item()) == 0
+        mx, _ = errors(out, ref)
+        assert mx <= 5e-2, (consumer, "fused", Hq, Hkv, P, tl, G, mx)
 
 
 @pytest.mark.parametrize("path", ["split", "fused"])
 def test_e4m3_both_consumers(B, path):
-    """An E4M3 cache runs on the mma.sync kernel; HPC_E4M3_TCGEN05=1 selects the tcgen05
-    kernel. Both must meet the E4M3 tolerance on the same ragged batch, on both step paths."""
+    """An E4M3 cache runs on the mma.sync kernel by default; options.e4m3_kernel selects the
+    tcgen05 kernel. Both must meet the E4M3 tolerance on the same ragged batch, on both step
+    paths."""
     spec, case = _case((1, 2, 15, 16, 17, 127, 128, 129, 255, 256, 257, 4000), 32, 4, 128, 32, 64, seed=77,
                        kv="e4m3")
     dc = to_device(case)
     ref = oracle_out(case)
     outs = {}
     for consumer in ("tcgen05", "mma.sync"):
-        if consumer == "tcgen05":
-            os.environ["HPC_E4M3_TCGEN05"] = "1"
-        try:
-            if path == "split":
-                out, _, st = run_attention(B, spec, dc, num_ctas=37)
-            else:
-                out, st_t, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
-                                                   dc["seq_lens"], 32, 4, 64, kv_dtype="e4m3", k_scale=dc["k_scale"],
-                                                   v_scale=dc["v_scale"], num_ctas=37)
-                torch.cuda.synchronize()
-                st = int(st_t.item())
-        finally:
-            os.environ.pop("HPC_E4M3_TCGEN05", None)
+        kernel = "tcgen05" if consumer == "tcgen05" else "mma"
+        if path == "split":
+            out, _, st = run_attention(B, spec, dc, num_ctas=37, e4m3_kernel=kernel)
+        else:
+            out, st_t, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
+                                               dc["seq_lens"], 32, 4, 64, kv_dtype="e4m3", k_scale=dc["k_scale"],
+                                               v_scale=dc["v_scale"], num_ctas=37, e4m3_kernel=kernel)
+            torch.cuda.synchronize()
+            st = int(st_t.item())
         assert st == 0
         mx, mean = errors(out, ref)
         assert mx <= 5e-2, (consumer, mx)
@@ -189,16 +181,61 @@ def test_empty_request_and_nan_slack(B):
     assert_bf16_tol(out, ref, what="nan slack")
 
 
-def test_bad_page_is_flagged_without_fault(B):
-    spec, case = _case((40, 100), 8, 2, 64, 16, 32, seed=8)
+def _attention_without_pages(case, bt, kv):
+    """fp64 attention of every (request, head) over the tokens whose block-table entry is a page
+    of the pool: the kernels leave a bad page's tokens out of the softmax. Written from the
+    oracle's pieces (its pinned single-part softmax state) on the tokens that remain."""
+    from oracle import attention as OA
+    from oracle import merge as OM
+    spec = case.spec
+    P, grp = spec.page_size, spec.group
+    kp, vp = OA.to_f64(case.k_pages), OA.to_f64(case.v_pages)
+    if kv == "e4m3":
+        kp, vp = OF.decode_array(case.k_pages.numpy()), OF.decode_array(case.v_pages.numpy())
+        kp = kp * case.k_scale.double().numpy()[None, :, None, None]
+        vp = vp * case.v_scale.double().numpy()[None, :, None, None]
+    q = OA.to_f64(case.q)
+    out = np.zeros((spec.batch, spec.num_heads, spec.head_dim))
+    for r, L in enumerate(spec.seq_lens):
+        toks = [t for t in range(L) if 0 <= int(bt[r, t // P]) < case.num_pages]
+        for g in range(spec.kv_heads):
+            K = np.array([kp[int(bt[r, t // P]), g, t % P] for t in toks])
+            V = np.array([vp[int(bt[r, t // P]), g, t % P] for t in toks])
+            for h in range(g * grp, (g + 1) * grp):
+                m, lsum, o = OM.partial_state(spec.sm_scale * (K @ q[r, h]), V)
+                out[r, h] = o / lsum
+    return out
+
+
+@pytest.mark.parametrize("kv,kernel,tl", [("bf16", "mma", 32), ("bf16", "mma", 16), ("e4m3", "mma", 32),
+                                          ("e4m3", "tcgen05", 32), ("e4m3", "tcgen05", 16)])
+def test_bad_page_is_left_out_without_fault(B, kv, kernel, tl):
+    """A block-table entry outside the pool is never handed to the copy engine: page 0 stands in,
+    HPC_DEV_BAD_PAGE is set, and the page's tokens are left out of the request's softmax. The
+    outputs then equal attention over the remaining tokens, for every request, on both paths.
+    With 16-token tiles a split piece holds only a bad page (no live token) and must merge as
+    nothing."""
+    spec, case = _case((40, 100, 300), 8, 2, 128, 16, tl, seed=8, kv=kv)
     bt = case.block_table.clone()
     bt[1, 2] = case.num_pages + 5
     bt[0, 0] = -3
+    bt[2, 5] = case.num_pages
     dc = to_device(case)
     dc["block_table"] = bt.cuda()
-    out, _, st = run_attention(B, spec, dc, num_ctas=4)
-    assert st & B.DEV_STATUS["bad_page"]
-    assert torch.isfinite(out).all()
+    ref = _attention_without_pages(case, bt.numpy(), kv)
+    for G in (4, 148):
+        out, _, st = run_attention(B, spec, dc, num_ctas=G, e4m3_kernel=kernel)
+        fused, st_f, _ = B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"],
+                                             dc["seq_lens"], 8, 2, tl, kv_dtype=kv, k_scale=dc["k_scale"],
+                                             v_scale=dc["v_scale"], num_ctas=G, e4m3_kernel=kernel)
+        torch.cuda.synchronize()
+        for o, s_ in ((out, st), (fused, int(st_f.item()))):
+            assert s_ == B.DEV_STATUS["bad_page"]
+            assert torch.isfinite(o).all()
+            if kv == "bf16":
+                assert_bf16_tol(o, ref, what=f"bad pages, G={G}")
+            else:
+                assert errors(o, ref)[0] <= 5e-2
 
 
 def test_static_plan_matches_oracle(B):

@@ -18,12 +18,13 @@ def B():
     return binding
 
 
-def _fused(B, spec, dc, seq_lens=None, num_ctas=None, workspace=None, out_dtype=torch.float32, q=None):
+def _fused(B, spec, dc, seq_lens=None, num_ctas=None, workspace=None, out_dtype=torch.float32, q=None,
+           item_cost=None):
     out, st, ws = B.decode_step_fused(dc["q"] if q is None else q, dc["k_pages"], dc["v_pages"], dc["block_table"],
                                       dc["seq_lens"] if seq_lens is None else seq_lens, spec.num_heads,
                                       spec.kv_heads, spec.tile_len, kv_dtype=spec.kv_dtype, k_scale=dc["k_scale"],
                                       v_scale=dc["v_scale"], num_ctas=num_ctas, workspace=workspace,
-                                      out_dtype=out_dtype)
+                                      out_dtype=out_dtype, item_cost=item_cost)
     torch.cuda.synchronize()
     return out, int(st.item()), ws
 
@@ -61,27 +62,26 @@ def test_shapes_ragged(B, Hq, Hkv, D, P, tl):
         assert _tickets_zero(ws, spec.batch, spec.kv_heads)
 
 
-@pytest.mark.parametrize("cost", ["0", "16", "200", "1024"])
-def test_item_cost_split(B, monkeypatch, cost):
-    """The split of the single-launch step with a fixed cost per item (HPC_ITEM_COST, in 1/16 of
-    a tile; 0 is the pages' split by tiles alone). Whatever the cost, every tile lands in
+@pytest.mark.parametrize("cost", [0, 16, 200, 1024])
+def test_item_cost_split(B, cost):
+    """The split of the single-launch step with a fixed cost per item (options.item_cost, in 1/16
+    of a tile; 0 is the pages' split by tiles alone). Whatever the cost, every tile lands in
     exactly one CTA, every split segment's piece count and partial slots agree (the merge
     tickets end at zero) and the output equals the oracle, for CTA counts from 1 to 2 per SM."""
-    monkeypatch.setenv("HPC_ITEM_COST", cost)
     lens = (1, 15, 16, 17, 63, 64, 65, 129, 300, 1000, 2049, 0, 5000)
     spec = W.custom_spec(lens, 16, 4, 128, 64, 64, seed=61)
     case = W.make_case(spec)
     dc = to_device(case)
     ref = oracle_out(case)
     for G in (1, 3, 8, 37, 148, 296):
-        out, st, ws = _fused(B, spec, dc, num_ctas=G)
+        out, st, ws = _fused(B, spec, dc, num_ctas=G, item_cost=cost)
         assert st == 0
         assert_bf16_tol(out, ref, what=f"fused, item cost {cost}, G={G}")
         assert _tickets_zero(ws, spec.batch, spec.kv_heads)
 
 
 @pytest.mark.parametrize("D,Bmax", [(128, 4095), (64, 2047)])
-def test_largest_batch(B, monkeypatch, D, Bmax):
+def test_largest_batch(B, D, Bmax):
     """The single launch keeps the per-request prefix (tile and segment counts packed in one
     int64) in shared memory. Its largest batch, 4095 requests at head_dim 128 and 2047 at 64,
     runs with short ragged lengths and empty requests, with and without the item cost, and
@@ -94,12 +94,8 @@ def test_largest_batch(B, monkeypatch, D, Bmax):
     empty = [i for i, L in enumerate(lens) if L == 0][:3]
     rows = sorted(set([0, 1, 2, Bmax // 2, Bmax - 2, Bmax - 1] + empty + [int(x) for x in rng.integers(0, Bmax, 6)]))
     ref = oracle_out(W.make_case(spec, requests=rows))
-    for cost in ("0", None):
-        if cost is None:
-            monkeypatch.delenv("HPC_ITEM_COST", raising=False)
-        else:
-            monkeypatch.setenv("HPC_ITEM_COST", cost)
-        out, st, ws = _fused(B, spec, dc)
+    for cost in (0, None):
+        out, st, ws = _fused(B, spec, dc, item_cost=cost)
         assert st == 0
         assert_bf16_tol(out[rows], ref, what=f"largest batch {Bmax}, D {D}, cost {cost}")
         assert _tickets_zero(ws, spec.batch, spec.kv_heads)
@@ -130,9 +126,8 @@ def test_empty_and_invalid_requests(B):
     assert torch.all(out2[2] == 0) and torch.isfinite(out2).all()
 
 
-def test_matches_three_launch_path_and_is_deterministic(B, monkeypatch):
+def test_matches_three_launch_path_and_is_deterministic(B):
     # with no item cost the single launch splits the tiles exactly as the planner does
-    monkeypatch.setenv("HPC_ITEM_COST", "0")
     spec = W.custom_spec((5000, 40, 999, 131, 7777), 64, 8, 128, 64, 128, seed=52)
     case = W.make_case(spec)
     dc = to_device(case)
@@ -140,7 +135,7 @@ def test_matches_three_launch_path_and_is_deterministic(B, monkeypatch):
                                 128, num_ctas=148)
     outs, ws = [], None
     for _ in range(3):
-        o, st, ws = _fused(B, spec, dc, num_ctas=148, workspace=ws)
+        o, st, ws = _fused(B, spec, dc, num_ctas=148, workspace=ws, item_cost=0)
         assert st == 0
         outs.append(o.clone())
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])

@@ -32,7 +32,7 @@ def nhd(t):
     ("bf16", 8, 2, 64, 16, 32), ("bf16", 64, 8, 128, 64, 128), ("bf16", 16, 4, 128, 128, 128),
     ("e4m3", 64, 8, 128, 64, 128), ("e4m3", 16, 2, 128, 16, 32),
 ])
-def test_nhd_attention_both_paths(B, monkeypatch, kv, Hq, Hkv, D, P, tl):
+def test_nhd_attention_both_paths(B, kv, Hq, Hkv, D, P, tl):
     lens = (1, 17, 64, 65, 300, 1000, 2049)
     spec = W.custom_spec(lens, Hq, Hkv, D, P, tl, kv_dtype=kv, seed=61 + D + P)
     case = W.make_case(spec)
@@ -45,10 +45,8 @@ def test_nhd_attention_both_paths(B, monkeypatch, kv, Hq, Hkv, D, P, tl):
     split, _, st1 = B.decode_step(dc["q"], kn, vn, dc["block_table"], dc["seq_lens"], Hq, Hkv, tl, kv_layout="NHD",
                                   num_ctas=37, **common)
     # with no item cost the single launch cuts the tiles where the planner does: same sums
-    monkeypatch.setenv("HPC_ITEM_COST", "0")
     fused0, st2, _ = B.decode_step_fused(dc["q"], kn, vn, dc["block_table"], dc["seq_lens"], Hq, Hkv, tl,
-                                         kv_layout="NHD", num_ctas=37, **common)
-    monkeypatch.delenv("HPC_ITEM_COST")
+                                         kv_layout="NHD", num_ctas=37, item_cost=0, **common)
     fused, st3, _ = B.decode_step_fused(dc["q"], kn, vn, dc["block_table"], dc["seq_lens"], Hq, Hkv, tl,
                                         kv_layout="NHD", num_ctas=37, **common)
     torch.cuda.synchronize()
