@@ -66,8 +66,16 @@ def parse_args(argv=None):
     ap.add_argument("--shard", action="store_true",
                     help="request-sharded placement of ONE batch over the ranks (strong scaling): each rank runs its "
                          "parts, (out, lse) are all-gathered and split requests merged; default: independent replicas")
-    ap.add_argument("--no-extras", action="store_true", help="skip static split-k, e2e and CPU baseline legs")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the graph, distribution, static split-k, CPU baseline and other-workload legs")
+    ap.add_argument("--item-cost", type=int, default=None,
+                    help="single-launch split: cost of an item start in 1/16 tile (default: the library's)")
+    ap.add_argument("--e4m3-kernel", default="mma", choices=["mma", "tcgen05"], help="kernel for E4M3 caches")
+    ap.add_argument("--multi-kernel", default="default", choices=["default", "mma", "tcgen05"],
+                    help="kernel for several new tokens per request (--q-len > 1)")
+    ap.add_argument("--trace", action="store_true",
+                    help="run the HPC_TRACE build of the library and print a per-CTA load summary of the single "
+                         "launch (idle tail, plan and first-data latency) instead of the benchmark line")
     return ap.parse_args(argv)
 
 
@@ -171,8 +179,10 @@ class Step:
     """One decode step through the binding, with buffers allocated once."""
 
     def __init__(self, B, spec, dc, num_ctas, tile_len, static_splits=None, fused=False, layout="HND",
-                 folded=False):
+                 folded=False, item_cost=None, e4m3_kernel="mma", multi_kernel="default"):
         self.B, self.spec, self.dc = B, spec, dc
+        self.item_cost, self.e4m3_kernel, self.multi_kernel = item_cost, e4m3_kernel, multi_kernel
+        self.trace = None  # HPC_TRACE builds only: per-CTA stamps of the single-launch step
         self.layout = layout
         self.tl = tile_len
         self.fused = (fused or folded) and not static_splits
@@ -210,7 +220,8 @@ class Step:
                                    dc["block_table"], seq, s.num_heads, s.kv_heads, self.tl, kv_dtype=s.kv_dtype,
                                    kv_layout=self.layout, k_scale=dc["k_scale"], v_scale=dc["v_scale"],
                                    eps=s.rms_eps, rope_theta=s.rope_theta, num_ctas=self.num_ctas, out=self.out,
-                                   status=self.status, workspace=self.ws)
+                                   status=self.status, workspace=self.ws, item_cost=self.item_cost,
+                                   trace=self.trace)
             if ev is not None:
                 ev[1].record()
             return self.out
@@ -225,7 +236,8 @@ class Step:
             B.decode_step_multi(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, s.kv_heads, self.tl,
                                 kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                                 v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
-                                workspace=self.ws)
+                                workspace=self.ws, item_cost=self.item_cost, trace=self.trace,
+                                multi_kernel=self.multi_kernel)
             if ev is not None:
                 ev[1].record()
             return self.out
@@ -235,7 +247,8 @@ class Step:
             B.decode_step_fused(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, s.num_heads,
                                 s.kv_heads, self.tl, kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                                 v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
-                                workspace=self.ws)
+                                workspace=self.ws, item_cost=self.item_cost, e4m3_kernel=self.e4m3_kernel,
+                                trace=self.trace)
             if ev is not None:
                 ev[1].record()
             return self.out
@@ -249,7 +262,7 @@ class Step:
             ev[0].record()
         B.attention(self.q, dc["k_pages"], dc["v_pages"], dc["block_table"], seq, self.plan, kv_dtype=s.kv_dtype,
                     kv_layout=self.layout, k_scale=dc["k_scale"], v_scale=dc["v_scale"], out=self.out, partial_o=self.po,
-                    partial_ml=self.pml, status=self.status)
+                    partial_ml=self.pml, status=self.status, e4m3_kernel=self.e4m3_kernel)
         if ev is not None:
             ev[1].record()
         B.merge(self.plan, self.po, self.pml, self.out, s.num_heads, self.status)
@@ -263,10 +276,12 @@ class Step:
 
 class ShardStep:
     """The step of one batch placed over the ranks by request (load_balanced_split_step_b200.shard):
-    q rows of the local parts gathered (hpc_gather_rows), the parts through hpc_decode_step_lse,
-    one all-gather of (out, lse), every request formed from its parts (hpc_merge_lse_gather)."""
+    the placement follows this step's lengths (kept, or made again past the drift bound), the
+    rank's block-table view is rebuilt on the device (hpc_gather_pages), q rows of the local
+    parts gathered (hpc_gather_rows), the parts through hpc_decode_step_lse, one all-gather of
+    (out, lse), every request formed from its parts (hpc_merge_lse_gather)."""
 
-    def __init__(self, B, spec, dc, num_ctas, tile_len, rank, world):
+    def __init__(self, B, spec, dc, num_ctas, tile_len, rank, world, lens_dev):
         from load_balanced_split_step_b200 import shard as SH
         self.spec, self.dc, self.tl = spec, dc, tile_len
         self.status = torch.zeros(1, dtype=torch.int32, device=dc["seq_lens"].device)
@@ -274,21 +289,26 @@ class ShardStep:
                                      v_scale=dc["v_scale"], num_ctas=num_ctas, status=self.status)
         self.st = SH.ShardedStep(spec.seq_lens, world, rank, spec.page_size, spec.num_heads, spec.head_dim,
                                  compute=compute, merge=SH.library_merge(self.status),
-                                 gather=SH.library_gather(self.status))
+                                 gather=SH.library_gather(self.status), pages=SH.library_pages(self.status))
+        # the host knows each step's lengths (a serving loop's scheduler does): decode step i of the
+        # workload has seq_lens + i
+        self.host_lens = {id(t): [L + i for L in spec.seq_lens] for i, t in enumerate(lens_dev)}
         self.out = None
 
     def __call__(self, seq_lens=None, ev=None, q=None):
         d = self.dc
+        host = self.host_lens.get(id(seq_lens)) if seq_lens is not None else None
         if ev is not None:
             ev[0].record()
-        self.out = self.st.step(d["q"] if q is None else q, d["k_pages"], d["v_pages"], d["block_table"], self.tl)
+        self.out = self.st.step(d["q"] if q is None else q, d["k_pages"], d["v_pages"], d["block_table"], self.tl,
+                                seq_lens=host)
         if ev is not None:
             ev[1].record()
         return self.out
 
     @property
     def launches(self):
-        local = 2 if self.st.plan[self.st.rank] else 0  # q gather and the step, when the rank has parts
+        local = 3 if self.st.plan[self.st.rank] else 0  # page view, q gather and the step, when the rank has parts
         return local + 1  # then the indexed merge
 
 
@@ -411,7 +431,8 @@ def shard_e2e_leg(step, case, dc, steps, world):
     return t0.elapsed_time(t1), q_host.numel() * q_host.element_size(), hosts[0].numel() * hosts[0].element_size()
 
 
-def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND", folded=False):
+def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="HND", folded=False,
+            multi_kernel="default"):
     """Same metric through the public call, with per-step H2D of the step inputs (q or qkv,
     seq_lens, block_table) from pinned host memory and D2H of the output. The KV cache is
     device-resident decode state and is not copied. The step runs as a serving loop would:
@@ -467,7 +488,8 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
             elif fused and spec.q_len > 1:
                 B.decode_step_multi(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.kv_heads, tl,
                                     kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
-                                    v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws)
+                                    v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws,
+                                    multi_kernel=multi_kernel)
             elif fused:
                 B.decode_step_fused(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
                                     spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
@@ -497,50 +519,154 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
     return t0.elapsed_time(t1), h2d, d2h
 
 
-def cpu_baseline(spec, case, target_s):
-    """The fp64 oracle, as it stands, over whole passes of the workload on the host cores,
-    until target_s seconds have been spent. Returns (GB/s, description, threads)."""
-    from oracle import attention as OA
-    from oracle import prologue as OR
+# ------------------------------------------------------------------ CPU baseline (the oracle)
+#
+# The fp64 oracle, as it stands, on a fixed stratified sample of the workload: kv head g of
+# request r is in the sample when (g - r) % S == 0, S = min(4, kv_heads), so every request (the
+# 128K one of the extreme batch included) contributes the same fraction of its tokens. The
+# sample's (request, query head) pairs are the units of work. A pool of single-threaded worker
+# processes (started with spawn; BLAS and torch limited to one thread each) takes them from a
+# shared queue, longest first; the sample's pages sit in one shared-memory block that the
+# workers map without copying. The timed region is one pass over the units.
+
+_CPU = {}
+
+
+def _cpu_worker_init(shm_name, nbytes):
+    import torch
+    torch.set_num_threads(1)
     try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        from threadpoolctl import threadpool_limits
+        _CPU["limits"] = threadpool_limits(1)
     except Exception:
-        threads = os.cpu_count() or 1
-    bytes_step = W.algorithmic_bytes(spec)
-    # bounded sample: whole requests, drawn round-robin from the batch, until the target is met
-    order = list(range(spec.batch))
+        pass
+    from multiprocessing import shared_memory
+    shm = shared_memory.SharedMemory(name=shm_name)
+    _CPU["shm"] = shm
+    _CPU["buf"] = np.ndarray((nbytes,), dtype=np.uint8, buffer=shm.buf)
+    from oracle import attention  # noqa: F401  (imported before the timed pass)
+
+
+def _cpu_ready(_):
+    return os.getpid()
+
+
+def _cpu_unit(task):
+    """One (request, query head) of the sample through oracle.attention.decode_attention."""
+    import torch
+    from oracle import attention as OA
+    k_off, v_off, n_pages, P, D, L, kv_dtype, q_row, k_s, v_s, scale = task
+    buf = _CPU["buf"]
+    elt = 1 if kv_dtype == "e4m3" else 2
+    n = n_pages * P * D * elt
+    if kv_dtype == "e4m3":
+        kp = buf[k_off:k_off + n].reshape(n_pages, 1, P, D)
+        vp = buf[v_off:v_off + n].reshape(n_pages, 1, P, D)
+    else:
+        kp = torch.from_numpy(buf[k_off:k_off + n]).view(torch.bfloat16).reshape(n_pages, 1, P, D)
+        vp = torch.from_numpy(buf[v_off:v_off + n]).view(torch.bfloat16).reshape(n_pages, 1, P, D)
+    q = np.asarray(q_row, dtype=np.float64).reshape(1, 1, D)
+    bt = np.arange(n_pages, dtype=np.int64)[None, :]
     t0 = time.perf_counter()
-    done_bytes, n_req = 0, 0
-    per_req_kv = {r: spec.seq_lens[r] * spec.kv_heads * spec.head_dim * 2 * (1 if spec.kv_dtype == "e4m3" else 2)
-                  for r in order}
-    i = 0
-    while time.perf_counter() - t0 < target_s and n_req < 100000:
-        r = order[i % len(order)]
-        i += 1
+    OA.decode_attention(q, kp, vp, bt, np.array([L]), sm_scale=scale, kv_dtype=kv_dtype, k_scale=[k_s],
+                        v_scale=[v_s])
+    return time.perf_counter() - t0
+
+
+class CpuBaseline:
+    """The oracle on the host cores over a fixed stratified sample of one workload (see above)."""
+
+    def __init__(self, spec, case, max_workers=32):
+        from multiprocessing import shared_memory
+        Hkv, grp, D, P = spec.kv_heads, spec.group, spec.head_dim, spec.page_size
+        S = min(4, Hkv)
+        pairs = [(r, g) for r in range(spec.batch) for g in range(Hkv) if (g - r) % S == 0 and spec.seq_lens[r] > 0]
+        kp, vp, q, bt = case.k_pages, case.v_pages, case.q, case.block_table
+        self.prologue_note = ""
         if spec.prologue:
-            sub = W.extract_requests(case, [r])
-            kp, vp = sub.k_pages.numpy().copy(), sub.v_pages.numpy().copy()
-            q = OR.decode_prologue(sub.qkv, sub.q_norm_w, sub.k_norm_w, spec.rms_eps, spec.rope_theta,
-                                   sub.seq_lens.numpy(), sub.block_table.numpy(), kp, vp, spec.kv_dtype,
-                                   sub.k_scale, sub.v_scale, spec.num_heads, spec.kv_heads)[0]
-            OA.decode_attention(q, kp, vp, sub.block_table, sub.seq_lens, kv_dtype=spec.kv_dtype,
-                                k_scale=sub.k_scale, v_scale=sub.v_scale)
-        elif spec.q_len > 1:
-            OA.decode_attention_multi(case.q[r:r + 1], case.k_pages, case.v_pages, case.block_table[r:r + 1],
-                                      case.seq_lens[r:r + 1], kv_dtype=spec.kv_dtype, k_scale=case.k_scale,
-                                      v_scale=case.v_scale)
-        else:
-            OA.decode_attention(case.q[r:r + 1], case.k_pages, case.v_pages, case.block_table[r:r + 1],
-                                case.seq_lens[r:r + 1], kv_dtype=spec.kv_dtype, k_scale=case.k_scale,
-                                v_scale=case.v_scale)
-        done_bytes += per_req_kv[r] + spec.q_len * spec.num_heads * spec.head_dim * 6
-        n_req += 1
-    el = time.perf_counter() - t0
-    frac = done_bytes / bytes_step
-    desc = (f"{n_req} whole requests of the workload taken round-robin "
-            f"({frac:.2f} of one step's algorithmic bytes) in {el:.1f} s")
-    return done_bytes / el / 1e9, desc, threads, el
+            # q and the new token's K/V come from the oracle's own prologue, outside the timed pass
+            from oracle import prologue as OR
+            kpn, vpn = case.k_pages.numpy().copy(), case.v_pages.numpy().copy()
+            qo = OR.decode_prologue(case.qkv, case.q_norm_w, case.k_norm_w, spec.rms_eps, spec.rope_theta,
+                                    case.seq_lens.numpy(), case.block_table.numpy(), kpn, vpn, spec.kv_dtype,
+                                    case.k_scale, case.v_scale, spec.num_heads, Hkv)[0]
+            kp, vp, q = torch.from_numpy(kpn), torch.from_numpy(vpn), qo
+            self.prologue_note = "; q and the new token's K/V from the oracle's prologue, untimed (<1% of the work)"
+        qf = q.to(torch.float64).numpy() if isinstance(q, torch.Tensor) else np.asarray(q, dtype=np.float64)
+        elt = 1 if spec.kv_dtype == "e4m3" else 2
+        blocks, tasks, off = [], [], 0
+        ks = case.k_scale.double().numpy() if case.k_scale is not None else np.ones(Hkv)
+        vs = case.v_scale.double().numpy() if case.v_scale is not None else np.ones(Hkv)
+        self.bytes = 0
+        self.tokens = 0
+        for r, g in pairs:
+            L = spec.seq_lens[r]
+            npg = -(-L // P)
+            rows = bt[r, :npg].long()
+            kb = kp[rows, g].contiguous().view(torch.uint8).numpy().reshape(-1)
+            vb = vp[rows, g].contiguous().view(torch.uint8).numpy().reshape(-1)
+            blocks += [kb, vb]
+            for h in range(g * grp, (g + 1) * grp):
+                tasks.append((off, off + kb.size, npg, P, D, L, spec.kv_dtype, qf[r, h].tolist(), float(ks[g]),
+                              float(vs[g]), spec.sm_scale))
+            off += kb.size + vb.size
+            self.bytes += L * D * elt * 2 + grp * D * (2 + 4)
+            self.tokens += L
+        tasks.sort(key=lambda t: -t[5])  # longest first: the queue then balances the workers
+        self.tasks = tasks
+        self.pairs = len(pairs)
+        self.frac = self.bytes / W.algorithmic_bytes(spec)
+        self.nbytes = max(off, 1)
+        self.shm = shared_memory.SharedMemory(create=True, size=self.nbytes)
+        buf = np.ndarray((self.nbytes,), dtype=np.uint8, buffer=self.shm.buf)
+        pos = 0
+        for b in blocks:
+            buf[pos:pos + b.size] = b
+            pos += b.size
+        del buf
+        try:
+            avail = len(os.sched_getaffinity(0))
+        except AttributeError:
+            avail = os.cpu_count() or 1
+        self.workers = max(1, min(avail, max_workers, len(tasks)))
+        import multiprocessing as mp
+        self.pool = mp.get_context("spawn").Pool(self.workers, initializer=_cpu_worker_init,
+                                                 initargs=(self.shm.name, self.nbytes))
+        self.pool.map(_cpu_ready, range(4 * self.workers), chunksize=1)  # every worker up and imported
+        self.S = S
+
+    def run(self):
+        """One timed pass over the sample: (GB/s of algorithmic bytes, seconds)."""
+        t0 = time.perf_counter()
+        self.pool.map(_cpu_unit, self.tasks, chunksize=1)
+        el = time.perf_counter() - t0
+        return self.bytes / el / 1e9, el
+
+    def describe(self, el):
+        return (f"kv heads g of request r with (g - r) % {self.S} == 0: {self.pairs} (request, kv head) pairs, "
+                f"{len(self.tasks)} (request, query head) units, {self.frac:.3f} of one step's algorithmic bytes, "
+                f"every request in proportion; one pass in {el:.1f} s on {self.workers} single-threaded worker "
+                f"processes{self.prologue_note}")
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        self.shm.close()
+        self.shm.unlink()
+
+
+def cpu_baseline(spec, case, passes=3):
+    """The oracle on the host cores: the median of `passes` timed passes over the stratified
+    sample. Returns the cpu_baseline object of the JSON line."""
+    cb = CpuBaseline(spec, case)
+    try:
+        runs = sorted(cb.run() for _ in range(passes))
+        v, el = runs[len(runs) // 2]
+        return {"value": round(v, 4), "unit": "GB/s", "cores": cb.workers, "kind": "oracle",
+                "sample": cb.describe(el) + f"; median of {passes} passes", "cpu_model": cpu_model(),
+                "host_cores": os.cpu_count()}
+    finally:
+        cb.close()
 
 
 def qlen_text(args):
@@ -601,31 +727,19 @@ def load_traffic(workload):
         return None
 
 
-def run_ours(args, rank, world, local):
-    from load_balanced_split_step_b200 import binding as B
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    spec = workload_spec(args)
-    case = W.make_case(spec)
+def device_case(case, dev, layout="HND"):
     dc = {k: (getattr(case, k).to(dev) if getattr(case, k) is not None else None)
           for k in ("q", "qkv", "k_pages", "v_pages", "block_table", "seq_lens", "k_scale", "v_scale", "q_norm_w",
                     "k_norm_w")}
-    if args.layout == "NHD":  # same tokens, vLLM page layout [pages][P][Hkv][D]
+    if layout == "NHD":  # same tokens, vLLM page layout [pages][P][Hkv][D]
         dc["k_pages"] = dc["k_pages"].permute(0, 2, 1, 3).contiguous()
         dc["v_pages"] = dc["v_pages"].permute(0, 2, 1, 3).contiguous()
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    tl = args.tile_len or spec.tile_len
-    G = sms * args.ctas_per_sm
-    if args.shard:
-        if spec.prologue or spec.q_len != 1 or spec.steps != 1 or args.layout != "HND":
-            raise SystemExit("--shard runs one-step, one-token workloads without the prologue, HND cache")
-        step = ShardStep(B, spec, dc, G, tl, rank, world)
-    else:
-        step = Step(B, spec, dc, G, tl, fused=args.path == "fused", folded=args.path == "folded",
-                    layout=args.layout)
-    lens = step_lengths(dc, spec)
-    K, W_ = args.steps, max(3, args.warmup)
+    return dc
 
+
+def measure(step, spec, lens, K, W_, world, local, jobs=1, per_gpu_div=1):
+    """K back-to-back steps (the step time), then K more with events around the attention launch
+    (its own duration, for the roofline), with clocks sampled throughout. Returns a dict."""
     with ClockSampler(local) as clk:
         # the step as a user runs it: kernels back to back, chained by programmatic dependent launch
         total_ms, _ = time_steps(step, lens, K, W_, world, kernel_events=False)
@@ -639,14 +753,69 @@ def run_ours(args, rank, world, local):
     total_ms = max_over_ranks(total_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
     bytes_step = float(np.mean([W.algorithmic_bytes(spec, i % spec.steps) for i in range(spec.steps)]))
-    jobs = 1 if args.shard else world  # sharded: the ranks share one batch
-    value = jobs * bytes_step * K / (total_ms / 1e3) / 1e9
-    ms_step = total_ms / K
     peak, peak_kind = load_peaks()
-    achieved = bytes_step / (kern_ms / 1e3) / 1e9
-    if args.shard:  # per GPU: its share of the batch over the step, exchange and merge included
-        achieved = bytes_step / world / (kern_ms / 1e3) / 1e9
-    clocks = clk.summary()
+    achieved = bytes_step / per_gpu_div / (kern_ms / 1e3) / 1e9
+    return {"total_ms": total_ms, "kern_ms": kern_ms, "bytes_step": bytes_step, "K": K, "W": W_,
+            "value": jobs * bytes_step * K / (total_ms / 1e3) / 1e9, "ms_step": total_ms / K,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                         "frac_of_nominal_8000": round(achieved / 8000.0, 4), "kernel_us": round(1000 * kern_ms, 2)},
+            "clocks": clk.summary()}
+
+
+OTHER_WORKLOADS = ("uniform", "heavy", "fp8")
+
+
+def other_workload(B, args, name, dev, G, world, local):
+    """The same measurement on another named workload (single-launch path; the FP8 workload runs
+    the prologue kernel in front of it), for the workloads object of the JSON line."""
+    spec = W.config_spec(name)
+    case = W.make_case(spec)
+    dc = device_case(case, dev)
+    del case
+    step = Step(B, spec, dc, G, spec.tile_len, fused=True, item_cost=args.item_cost, e4m3_kernel=args.e4m3_kernel)
+    lens = step_lengths(dc, spec)
+    est_ms = W.algorithmic_bytes(spec) / 6.0e9
+    K = int(min(5000, max(64, round(1500.0 / est_ms))))
+    K -= K % spec.steps
+    m = measure(step, spec, lens, K, 20, world, local)
+    out = {"workload": WORKLOAD_TEXT[name], "steps": K, "warmup": 20, "us_per_step": round(1000 * m["ms_step"], 2),
+           "value": round(m["value"], 2), "unit": "GB/s",
+           "roofline": dict(m["roofline"], kernel="decode_attention_kernel<fused>", traffic=load_traffic(name)),
+           "clocks": m["clocks"], "gpu_launches": step.launches * K,
+           "path": "single launch" + (" after the prologue kernel (PDL)" if spec.prologue else "")}
+    if spec.steps > 1:
+        out["note"] = f"{spec.steps} decode steps cycled (lengths +1 per step, re-planned on the device each step)"
+    del step, dc
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local):
+    from load_balanced_split_step_b200 import binding as B
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec = workload_spec(args)
+    case = W.make_case(spec)
+    dc = device_case(case, dev, args.layout)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tl = args.tile_len or spec.tile_len
+    G = sms * args.ctas_per_sm
+    lens = step_lengths(dc, spec)
+    if args.shard:
+        if spec.prologue or spec.q_len != 1 or args.layout != "HND":
+            raise SystemExit("--shard runs one-token workloads without the prologue, HND cache")
+        step = ShardStep(B, spec, dc, G, tl, rank, world, lens)
+    else:
+        step = Step(B, spec, dc, G, tl, fused=args.path == "fused", folded=args.path == "folded",
+                    layout=args.layout, item_cost=args.item_cost, e4m3_kernel=args.e4m3_kernel,
+                    multi_kernel=args.multi_kernel)
+    K, W_ = args.steps, max(3, args.warmup)
+    jobs = 1 if args.shard else world  # sharded: the ranks share one batch
+    m = measure(step, spec, lens, K, W_, world, local, jobs=jobs, per_gpu_div=world if args.shard else 1)
+    total_ms, kern_ms, bytes_step = m["total_ms"], m["kern_ms"], m["bytes_step"]
+    value, ms_step = m["value"], m["ms_step"]
+    clocks = m["clocks"]
 
     extra = {}
     if not args.no_extras and not args.shard:
@@ -681,15 +850,21 @@ def run_ours(args, rank, world, local):
         e2e_ms, h2d, d2h = shard_e2e_leg(step, case, dc, e2e_steps, world)
     else:
         e2e_ms, h2d, d2h = e2e_leg(B, spec, case, dc, tl, G, e2e_steps, world, fused=args.path != "split",
-                                   layout=args.layout, folded=args.path == "folded")
+                                   layout=args.layout, folded=args.path == "folded", multi_kernel=args.multi_kernel)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_val = jobs * bytes_step * e2e_steps / (e2e_ms / 1e3) / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
-        v, desc, threads, _ = cpu_baseline(spec, case, args.cpu_seconds)
-        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "cpu_model": cpu_model(), "host_cores": os.cpu_count()}
+        cpu = cpu_baseline(spec, case)
+    others = None
+    if (world == 1 and not args.no_extras and not args.shard and args.workload == "extreme" and spec.q_len == 1
+            and not args.requests and args.path == "fused" and args.layout == "HND"):
+        del dc, case
+        if not isinstance(step, ShardStep):
+            step.dc = None
+        torch.cuda.empty_cache()
+        others = {name: other_workload(B, args, name, dev, G, world, local) for name in OTHER_WORKLOADS}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W_,
@@ -709,13 +884,10 @@ def run_ours(args, rank, world, local):
                    "parallelism": (f"one batch request-sharded over {world} GPU(s): one all-gather of (out, lse), "
                                    "log-sum-exp merge of split requests") if args.shard
                    else f"{world} independent replica(s), no collective"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "frac_of_nominal_8000": round(achieved / 8000.0, 4),
-                     "kernel": "decode_attention_kernel" + {"fused": "<fused>", "folded": "<fused, prologue>",
-                                                            "split": ""}[args.path],
-                     "kernel_us": round(1000 * kern_ms, 2),
-                     "traffic": load_traffic(args.workload)},
+        "roofline": dict(m["roofline"],
+                         kernel="decode_attention_kernel" + {"fused": "<fused>", "folded": "<fused, prologue>",
+                                                             "split": ""}[args.path],
+                         traffic=load_traffic(args.workload) if not (args.requests or args.q_len > 1) else None),
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": round(1000 * e2e_ms / e2e_steps, 2)},
@@ -723,42 +895,108 @@ def run_ours(args, rank, world, local):
         "clocks": clocks,
     }
     line.update(extra)
+    if others:
+        line["workloads"] = others
     return line
 
 
 def run_reference(args, rank, world):
-    """The reference arm: the fp64 CPU oracle as it stands, timed on the host cores."""
+    """The reference arm: the fp64 CPU oracle as it stands, timed on the host cores over the same
+    stratified sample as the cpu_baseline leg, one pass per step."""
     if rank != 0:
         return None
     spec = workload_spec(args)
     case = W.make_case(spec)
-    K, W_ = max(1, min(args.steps, 3)), 0
-    target = args.cpu_seconds
-    vals, descs, threads = [], [], 1
-    for _ in range(K):
-        v, desc, threads, _ = cpu_baseline(spec, case, target / K)
-        vals.append(v)
-        descs.append(desc)
-    v = float(np.mean(vals))
+    K, W_ = max(1, min(args.steps, 5)), min(max(args.warmup, 0), 1)
+    cb = CpuBaseline(spec, case)
+    try:
+        for _ in range(W_):
+            cb.run()
+        runs = [cb.run() for _ in range(K)]
+    finally:
+        cb.close()
+    el = sum(e for _, e in runs)
+    v = cb.bytes * K / el / 1e9
     bytes_step = W.algorithmic_bytes(spec)
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": W_, "ms_per_step": round(1000 * bytes_step / (v * 1e9), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload] + qlen_text(args), "tile_len": spec.tile_len,
-                   "plan": "none (exact)",
-                   "parallelism": "host cores"},
-        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": descs[0], "cpu_model": cpu_model(), "host_cores": os.cpu_count()},
+                   "plan": "none (exact)", "parallelism": f"{cb.workers} host processes"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cb.workers, "kind": "oracle",
+                         "sample": cb.describe(el / K) + f"; {K} timed passes", "cpu_model": cpu_model(),
+                         "host_cores": os.cpu_count()},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def run_trace(args, local):
+    """Per-CTA load evidence from the HPC_TRACE build: for each of R single-launch steps, every
+    CTA's entry, plan-ready, first-stage, last-item and producer-end stamps (%globaltimer, ns) with
+    its item and stage counts. Summarised per step: the launch span (first entry to last end),
+    each CTA's idle tail (span end minus its last item end, as a share of the span, averaged
+    over CTAs), the spread of CTA end times, the plan and first-data latencies. Stamps perturb
+    the kernel a little; the bench line, not this, gives the step time."""
+    from load_balanced_split_step_b200 import binding as B
+    from load_balanced_split_step_b200 import build as BLD
+    B.use_library(BLD.build_trace())
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec = workload_spec(args)
+    case = W.make_case(spec)
+    dc = device_case(case, dev, args.layout)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tl = args.tile_len or spec.tile_len
+    G = sms * args.ctas_per_sm
+    if args.path == "split":
+        raise SystemExit("--trace summarises the single-launch step")
+    step = Step(B, spec, dc, G, tl, fused=True, folded=args.path == "folded", layout=args.layout,
+                item_cost=args.item_cost, e4m3_kernel=args.e4m3_kernel)
+    trace = torch.zeros((G, B.TRACE_WORDS), dtype=torch.int64, device=dev)
+    step.trace = trace
+    lens = step_lengths(dc, spec)
+    for i in range(max(3, args.warmup)):
+        step(lens[i % len(lens)])
+    R = max(1, min(args.steps, 64))
+    per = []
+    for i in range(R):
+        trace.zero_()
+        step(lens[i % len(lens)])
+        torch.cuda.synchronize()
+        t = trace.cpu().numpy().astype(np.int64)
+        busy = t[:, 5] > 0
+        start = t[:, 1].min()  # the first CTA past the wait on the previous launch
+        end = max(t[:, 4].max(), t[busy, 3].max())
+        span = end - start
+        tail = (end - t[busy, 3]) / span  # idle after a CTA's last item, share of the span
+        per.append({"span_us": span / 1e3, "idle_tail_mean": float(tail.mean()),
+                    "idle_tail_p90": float(np.percentile(tail, 90)), "idle_tail_max": float(tail.max()),
+                    "end_spread_us": float((end - t[busy, 3].min()) / 1e3),
+                    "wait_and_plan_us_median": float(np.median(t[:, 1] - t[:, 0]) / 1e3),
+                    "plan_ready_spread_us": float((t[:, 1].max() - start) / 1e3),
+                    "first_data_us_median": float(np.median(t[busy, 2] - t[busy, 1]) / 1e3),
+                    "items_max": int(t[:, 5].max()), "items_median": float(np.median(t[busy, 5])),
+                    "stages_max": int(t[:, 6].max()), "stages_min_busy": int(t[busy, 6].min()),
+                    "ctas_busy": int(busy.sum())})
+    st = int(step.status.item())
+    if st:
+        raise RuntimeError(f"device status {st:#x}")
+    keys = per[0].keys()
+    summary = {k: round(float(np.median([p[k] for p in per])), 4) for k in keys}
+    return {"trace": summary, "steps": R, "workload": WORKLOAD_TEXT[args.workload] + qlen_text(args), "num_ctas": G,
+            "item_cost": args.item_cost if args.item_cost is not None else "default",
+            "note": "medians over the traced steps; span = first CTA past the wait on the previous launch to the last "
+                    "CTA's end; idle tail = (span end - a busy CTA's last item end) / span"}
 
 
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_init(args)
     try:
-        if args.impl == "reference":
+        if args.trace:
+            line = run_trace(args, local)
+        elif args.impl == "reference":
             line = run_reference(args, rank, world)
         else:
             line = run_ours(args, rank, world, local)

@@ -139,6 +139,9 @@ typedef struct {
 #define HPC_ITEM_COST_MAX 1024
 #define HPC_E4M3_MMA 0     /* E4M3 caches on the mma.sync consumers (the default) */
 #define HPC_E4M3_TCGEN05 1 /* E4M3 caches on the tcgen05 kernel, where it applies */
+#define HPC_MULTI_DEFAULT 0 /* several new tokens: the library's choice (see multi_kernel below) */
+#define HPC_MULTI_MMA 1     /* several new tokens on the mma.sync consumers */
+#define HPC_MULTI_TCGEN05 2 /* several new tokens on the tcgen05 kernel, where it applies */
 #define HPC_TRACE_WORDS 8  /* uint64 words per CTA in a trace buffer */
 #define HPC_BUILD_TRACE 1u /* hpc_build_flags(): the library was built with HPC_TRACE */
 
@@ -153,6 +156,10 @@ typedef struct {
  *   e4m3_kernel:  HPC_E4M3_MMA or HPC_E4M3_TCGEN05. The tcgen05 kernel serves E4M3 caches with
  *                 head_dim 128 in hpc_decode_attention, hpc_decode_step and hpc_decode_step_lse;
  *                 elsewhere the choice is ignored.
+ *   multi_kernel: HPC_MULTI_DEFAULT, HPC_MULTI_MMA or HPC_MULTI_TCGEN05: the kernel for
+ *                 hpc_decode_step_multi with q_len > 1. The tcgen05 kernel serves bf16 caches with
+ *                 head_dim 128 and q_len * (num_heads / kv_heads) <= 32; elsewhere the choice is
+ *                 ignored. The default is HPC_MULTI_MMA.
  *   record:       single-launch steps only: device buffer of hpc_step_record_bytes(num_ctas,
  *                 record_items) bytes that receives every CTA's hpc_cta_record, or NULL.
  *   trace:        device uint64 [num_ctas][HPC_TRACE_WORDS], or NULL. Only a library built with
@@ -161,17 +168,18 @@ typedef struct {
  *                 %globaltimer (ns): [0] entry, [1] plan ready (after the wait on the previous
  *                 kernel), [2] first stage consumed, [3] last item finished by the consumers,
  *                 [4] producer done; then [5] items, [6] pipeline stages, [7] SM id. Words [2]
- *                 and [3] stay 0 for a CTA without work. The mma.sync kernel writes it. */
+ *                 and [3] stay 0 for a CTA without work. The mma.sync kernels write it; with a
+ *                 tcgen05 kernel a trace buffer returns HPC_ERR_ARG. */
 typedef struct {
   int32_t item_cost;
   int32_t e4m3_kernel;
   void* record;
   int32_t record_items;
-  int32_t reserved;
+  int32_t multi_kernel;
   uint64_t* trace;
 } hpc_step_options;
 
-#define HPC_STEP_OPTIONS_INIT {HPC_ITEM_COST_DEFAULT, HPC_E4M3_MMA, NULL, 0, 0, NULL}
+#define HPC_STEP_OPTIONS_INIT {HPC_ITEM_COST_DEFAULT, HPC_E4M3_MMA, NULL, 0, HPC_MULTI_DEFAULT, NULL}
 
 /* Bytes of a record buffer for num_ctas CTAs with record_items entries each. */
 HPC_API size_t hpc_step_record_bytes(int32_t num_ctas, int32_t record_items);
@@ -372,6 +380,19 @@ HPC_API int hpc_merge_lse_gather(const float* outs, const float* lses, int64_t p
  * *status (device uint32, or NULL). */
 HPC_API int hpc_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* index, int64_t n,
                             void* dst, uint32_t* status, void* stream);
+
+/* Block-table view of the parts a request-sharded rank runs (each part is a page-aligned token
+ * range of one request; see hpc_merge_lse_gather): row i of the view lists the pages of request
+ * req[i] from column col0[i] on,
+ *   dst[i][j] = src[req[i]][col0[i] + j]  for j < width and col0[i] + j < src_cols, else -1,
+ * so that the rank's parts run as a batch of their own. Rebuilt every step on the device, it
+ * follows pages the caller appends to the table as requests grow. A req[i] outside
+ * [0, src_rows) or a negative col0[i] gives a row of -1 and sets HPC_DEV_BAD_INDEX.
+ *   src: device int32 [src_rows][src_cols]; req, col0: device int32 [n];
+ *   dst: device int32 [n][width]; status: device uint32 word or NULL. */
+HPC_API int hpc_gather_pages(const int32_t* src, int32_t src_rows, int32_t src_cols, const int32_t* req,
+                             const int32_t* col0, int32_t n, int32_t width, int32_t* dst, uint32_t* status,
+                             void* stream);
 
 /* ---- several new tokens per request ----------------------------------------------------- */
 

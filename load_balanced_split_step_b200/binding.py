@@ -29,6 +29,7 @@ RECORD_DTYPE = np.dtype([("unit_begin", "<i8"), ("unit_end", "<i8"), ("chunk", "
                          ("n_items", "<i4")])
 ITEM_COST_DEFAULT, ITEM_COST_MAX = -1, 1024
 E4M3_KERNELS = {"mma": 0, "tcgen05": 1}
+MULTI_KERNELS = {"default": 0, "mma": 1, "tcgen05": 2}
 TRACE_WORDS = 8
 BUILD_TRACE = 1
 
@@ -38,7 +39,7 @@ EXPORTS = ("hpc_step_record_bytes", "hpc_build_flags", "hpc_plan_workspace_bytes
            "hpc_status_string", "hpc_last_error", "hpc_abi_version", "hpc_decode_step_noalloc",
            "hpc_decode_step", "hpc_decode_step_workspace_bytes", "hpc_decode_step_prologue",
            "hpc_decode_step_multi", "hpc_decode_step_multi_workspace_bytes", "hpc_decode_step_lse",
-           "hpc_merge_lse", "hpc_wait_selftest", "hpc_merge_lse_gather", "hpc_gather_rows")
+           "hpc_merge_lse", "hpc_wait_selftest", "hpc_merge_lse_gather", "hpc_gather_rows", "hpc_gather_pages")
 
 
 class HpcError(RuntimeError):
@@ -55,7 +56,7 @@ class CPlan(ctypes.Structure):
 
 class COptions(ctypes.Structure):
     _fields_ = [("item_cost", ctypes.c_int32), ("e4m3_kernel", ctypes.c_int32), ("record", ctypes.c_void_p),
-                ("record_items", ctypes.c_int32), ("reserved", ctypes.c_int32), ("trace", ctypes.c_void_p)]
+                ("record_items", ctypes.c_int32), ("multi_kernel", ctypes.c_int32), ("trace", ctypes.c_void_p)]
 
 
 _path = LIB
@@ -109,6 +110,7 @@ def _load(path=LIB):
         "hpc_wait_selftest": (ctypes.c_int, [ctypes.c_uint64, i32, vp, vp, vp]),
         "hpc_merge_lse_gather": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, vp, vp, vp, vp]),
         "hpc_gather_rows": (ctypes.c_int, [vp, ctypes.c_int64, ctypes.c_int64, vp, ctypes.c_int64, vp, vp, vp]),
+        "hpc_gather_pages": (ctypes.c_int, [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp]),
         "hpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hpc_last_error": (ctypes.c_char_p, []),
         "hpc_abi_version": (ctypes.c_int, []),
@@ -336,18 +338,22 @@ def _out_code(out):
     return HPC_BF16 if out.dtype == torch.bfloat16 else HPC_FP32
 
 
-def options(item_cost=None, e4m3_kernel="mma", record=None, record_items=0, trace=None, device=None, num_ctas=None):
+def options(item_cost=None, e4m3_kernel="mma", record=None, record_items=0, trace=None, device=None, num_ctas=None,
+            multi_kernel="default"):
     """A ``hpc_step_options`` struct, or None when every option has its default.
     item_cost: 1/16 tile per item start (None: the library's default). e4m3_kernel: "mma" or
     "tcgen05". record: uint8 device tensor of ``record_bytes(num_ctas, record_items)`` bytes.
     trace: int64 device tensor [num_ctas, TRACE_WORDS] (HPC_TRACE builds only)."""
     if e4m3_kernel not in E4M3_KERNELS:
         raise HpcError(f"e4m3_kernel must be one of {list(E4M3_KERNELS)}")
-    if item_cost is None and e4m3_kernel == "mma" and record is None and trace is None:
+    if multi_kernel not in MULTI_KERNELS:
+        raise HpcError(f"multi_kernel must be one of {list(MULTI_KERNELS)}")
+    if item_cost is None and e4m3_kernel == "mma" and record is None and trace is None and multi_kernel == "default":
         return None
     o = COptions()
     o.item_cost = ITEM_COST_DEFAULT if item_cost is None else int(item_cost)
     o.e4m3_kernel = E4M3_KERNELS[e4m3_kernel]
+    o.multi_kernel = MULTI_KERNELS[multi_kernel]
     if record is not None:
         _need(record, "record", torch.uint8, device)
         o.record, o.record_items = record.data_ptr(), int(record_items)
@@ -551,10 +557,11 @@ def multi_workspace(batch, q_len, num_heads, kv_heads, head_dim, num_ctas, devic
 def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile_len, *, kv_dtype="bf16",
                       kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None,
                       out_dtype=torch.float32, status=None, workspace=None, item_cost=None, record=None,
-                      record_items=0, trace=None):
+                      record_items=0, trace=None, multi_kernel="default"):
     """q_len new tokens per request in one launch (``hpc_decode_step_multi``): q is
     [B, q_len, Hq, D]; query token t of request r sits at position L_r - q_len + t and
-    attends causally. Returns (out [B, q_len, Hq, D], status, workspace)."""
+    attends causally. multi_kernel: "default", "mma" or "tcgen05". Returns (out [B, q_len, Hq, D],
+    status, workspace)."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
     B, T, Hq, D = q.shape
@@ -567,7 +574,7 @@ def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile
     status = new_status(dev) if status is None else status
     workspace = _workspace(workspace, _lib.hpc_decode_step_multi_workspace_bytes(B, T, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    opt = options(item_cost, "mma", record, record_items, trace, dev, G)
+    opt = options(item_cost, "mma", record, record_items, trace, dev, G, multi_kernel)
     with torch.cuda.device(dev):
         _check(_lib.hpc_decode_step_multi(
             _ptr(q), T, _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv,
@@ -660,6 +667,27 @@ def gather_rows(src, index, out=None, status=None):
     with torch.cuda.device(dev):
         _check(_lib.hpc_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out), _ptr(status),
                                     _stream(dev)), "hpc_gather_rows")
+    return out
+
+
+def gather_pages(block_table, req, col0, width=None, out=None, status=None):
+    """``hpc_gather_pages``: out[i][j] = block_table[req[i]][col0[i] + j] (-1 past the table), the
+    block-table view of a request-sharded rank's parts. Returns out int32 [n, width]."""
+    _need(block_table, "block_table", torch.int32)
+    dev = block_table.device
+    _need(req, "req", torch.int32, dev)
+    _need(col0, "col0", torch.int32, dev)
+    if block_table.dim() != 2 or req.numel() != col0.numel():
+        raise HpcError("block_table must be 2-D and req / col0 of equal length")
+    n = req.numel()
+    width = block_table.shape[1] if width is None else int(width)
+    out = torch.empty((n, width), dtype=torch.int32, device=dev) if out is None else out
+    _need(out, "out", torch.int32, dev)
+    if tuple(out.shape) != (n, width):
+        raise HpcError("out must be [n, width]")
+    with torch.cuda.device(dev):
+        _check(_lib.hpc_gather_pages(_ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(req),
+                                     _ptr(col0), n, width, _ptr(out), _ptr(status), _stream(dev)), "hpc_gather_pages")
     return out
 
 

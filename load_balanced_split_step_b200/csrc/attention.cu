@@ -45,11 +45,13 @@ using namespace attn;
 
 // Online-softmax update of one warp's state with NB consecutive 16-token blocks of a stage.
 // K and V rows rb.. rb + 16*NB of the stage sit at kbase / vbase, in 128-byte swizzled
-// planes. Tokens tb.. of the request; tokens >= tok1 are masked. The NB blocks give
-// independent MMA chains, so the warp hides latency without more warps.
+// planes. Tokens tb.. of the request; tokens >= tok1 are masked, and so is the whole stage when
+// `bad` is set (its page id was out of range and page 0 stood in). The flag is applied with the
+// tail mask, after the QK^T products, so its shared-memory load does not hold them up. The NB
+// blocks give independent MMA chains, so the warp hides latency without more warps.
 template <int D, bool FP8, int NB>
 __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, uint32_t plane_bytes, int rb,
-                                               int64_t tb, int64_t tok1, const uint32_t (&qf)[D / 16][2],
+                                               int64_t tb, int64_t tok1, bool bad, const uint32_t (&qf)[D / 16][2],
                                                float score_scale, float& m0, float& m1, float& l0, float& l1,
                                                float (&o)[D / 16][4], int lane) {
   constexpr int KSTEPS = D / 16;
@@ -94,14 +96,15 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
   }
 
   // ---- online softmax (base 2) over these NB blocks, per head
-  const bool tail = tb + 16 * NB > tok1;
+  const bool tail = bad || tb + 16 * NB > tok1;
+  const int64_t lim = bad ? tb : tok1;  // a masked stage: no token is live
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) s[b][i] *= score_scale;
     if (tail) {
-      if (tb + 16 * b + g >= tok1) s[b][0] = s[b][1] = -INFINITY;
-      if (tb + 16 * b + g + 8 >= tok1) s[b][2] = s[b][3] = -INFINITY;
+      if (tb + 16 * b + g >= lim) s[b][0] = s[b][1] = -INFINITY;
+      if (tb + 16 * b + g + 8 >= lim) s[b][2] = s[b][3] = -INFINITY;
     }
   }
   float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
@@ -115,16 +118,19 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
   }
-  const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: every call has a live token
-  const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+  const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+  // -inf only when no token has been live yet (a masked stage): the reference 0 keeps every
+  // exponential at 0 instead of NaN
+  const float mr0 = mn0 == -INFINITY ? 0.f : mn0, mr1 = mn1 == -INFINITY ? 0.f : mn1;
+  const float al0 = exp2f(m0 - mr0), al1 = exp2f(m1 - mr1);
   float pr[NB][4];
   float add0 = 0.f, add1 = 0.f;
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    pr[b][0] = exp2f(s[b][0] - mn0);
-    pr[b][1] = exp2f(s[b][1] - mn1);
-    pr[b][2] = exp2f(s[b][2] - mn0);
-    pr[b][3] = exp2f(s[b][3] - mn1);
+    pr[b][0] = exp2f(s[b][0] - mr0);
+    pr[b][1] = exp2f(s[b][1] - mr1);
+    pr[b][2] = exp2f(s[b][2] - mr0);
+    pr[b][3] = exp2f(s[b][3] - mr1);
     add0 += pr[b][0] + pr[b][2];
     add1 += pr[b][1] + pr[b][3];
   }
@@ -169,8 +175,8 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
     mlo[b] = mhi[b] = 0xffffffffu;
     if (tail) {
       const int64_t t0 = tb + 16 * b;
-      mlo[b] = (t0 + 2 * c < tok1 ? 0x0000ffffu : 0u) | (t0 + 2 * c + 1 < tok1 ? 0xffff0000u : 0u);
-      mhi[b] = (t0 + 2 * c + 8 < tok1 ? 0x0000ffffu : 0u) | (t0 + 2 * c + 9 < tok1 ? 0xffff0000u : 0u);
+      mlo[b] = (t0 + 2 * c < lim ? 0x0000ffffu : 0u) | (t0 + 2 * c + 1 < lim ? 0xffff0000u : 0u);
+      mhi[b] = (t0 + 2 * c + 8 < lim ? 0x0000ffffu : 0u) | (t0 + 2 * c + 9 < lim ? 0xffff0000u : 0u);
     }
   }
 
@@ -668,18 +674,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (trace && warp == 0 && lane == 0 && trace[2] == 0) trace[2] = global_timer_ns();
 #endif
         const int64_t tb = t + 16 * my_first;
-        if (ok && t_live && tb < lim && !s_bad[stage]) {
+        if (ok && t_live && tb < lim) {
           const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
           const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
+          const bool bad_stage = s_bad[stage] != 0;
           if (FP8 && nb == 4)
-            consume_blocks<D, FP8, 4>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, qf, score_scale, m0, m1,
-                                      l0, l1, o, lane);
+            consume_blocks<D, FP8, 4>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, bad_stage, qf, score_scale,
+                                      m0, m1, l0, l1, o, lane);
           else if (nb == 2)
-            consume_blocks<D, FP8, 2>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, qf, score_scale, m0, m1,
-                                      l0, l1, o, lane);
+            consume_blocks<D, FP8, 2>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, bad_stage, qf, score_scale,
+                                      m0, m1, l0, l1, o, lane);
           else
-            consume_blocks<D, FP8, 1>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, qf, score_scale, m0, m1,
-                                      l0, l1, o, lane);
+            consume_blocks<D, FP8, 1>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, bad_stage, qf, score_scale,
+                                      m0, m1, l0, l1, o, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * stage);
@@ -960,6 +967,7 @@ namespace {
 struct Options {
   int32_t item_cost = HPC_ITEM_COST_DEFAULT;
   bool tc = false;
+  bool tcm = false;  // several new tokens on the tcgen05 kernel
   uint8_t* record = nullptr;
   int32_t record_items = 0;
   uint64_t* trace = nullptr;
@@ -972,6 +980,8 @@ int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
     return fail(HPC_ERR_ARG, "item_cost must be HPC_ITEM_COST_DEFAULT or 0 .. %d", HPC_ITEM_COST_MAX);
   if (o->e4m3_kernel != HPC_E4M3_MMA && o->e4m3_kernel != HPC_E4M3_TCGEN05)
     return fail(HPC_ERR_ARG, "e4m3_kernel must be HPC_E4M3_MMA or HPC_E4M3_TCGEN05");
+  if (o->multi_kernel != HPC_MULTI_DEFAULT && o->multi_kernel != HPC_MULTI_MMA && o->multi_kernel != HPC_MULTI_TCGEN05)
+    return fail(HPC_ERR_ARG, "multi_kernel must be HPC_MULTI_DEFAULT, HPC_MULTI_MMA or HPC_MULTI_TCGEN05");
   if (!single_launch && (o->item_cost != HPC_ITEM_COST_DEFAULT || o->record))
     return fail(HPC_ERR_ARG, "item_cost and record apply to the single-launch steps only");
   if (o->record && (o->record_items < 0 || (reinterpret_cast<uintptr_t>(o->record) & 15)))
@@ -982,6 +992,7 @@ int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
   if (o->trace && (reinterpret_cast<uintptr_t>(o->trace) & 7)) return fail(HPC_ERR_ALIGN, "trace must be 8-byte aligned");
   out->item_cost = o->item_cost;
   out->tc = o->e4m3_kernel == HPC_E4M3_TCGEN05;
+  out->tcm = o->multi_kernel == HPC_MULTI_TCGEN05;
   out->record = static_cast<uint8_t*>(o->record);
   out->record_items = o->record ? o->record_items : 0;
   out->trace = o->trace;
@@ -1061,10 +1072,14 @@ int prepare(const void* q, const void* k_pages, const void* v_pages, hpc_dtype k
 
 template <bool FUSED, bool PRO = false, bool MULTI = false>
 int dispatch(int head_dim, bool fp8, bool tc, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm,
-             int grid, int smem, cudaStream_t st) {
+             int grid, int smem, cudaStream_t st, bool tcm = false) {
   if (fp8 && !PRO && !MULTI && tc && tc_supported(head_dim, fp8, prm.group, prm.q_len, PRO)) {
     if (prm.trace) return fail(HPC_ERR_ARG, "the tcgen05 kernel writes no trace");
     return launch_attention_tc(FUSED, mk, mv, prm, grid, st);
+  }
+  if (FUSED && MULTI && tcm && tcm_supported(head_dim, fp8, prm.group, prm.q_len, PRO)) {
+    if (prm.trace) return fail(HPC_ERR_ARG, "the tcgen05 kernel writes no trace");
+    return launch_attention_tcm(mk, mv, prm, grid, st);
   }
   if (fp8) return launch<128, true, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
   if (head_dim == 128) return launch<128, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
@@ -1248,7 +1263,7 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   const bool fp8 = kv_dtype == HPC_E4M3;
   if (!pro && q_len > 1)
     return dispatch<true, false, true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem,
-                                       static_cast<cudaStream_t>(stream));
+                                       static_cast<cudaStream_t>(stream), opt.tcm);
   if (!pro)
     return dispatch<true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem, static_cast<cudaStream_t>(stream));
   prm.qkv = static_cast<const __nv_bfloat16*>(pro->qkv);

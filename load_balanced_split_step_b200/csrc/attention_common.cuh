@@ -475,5 +475,11 @@ int tc_threads();
 int launch_attention_tc(bool fused, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
                         cudaStream_t stream);
 
+// The tcgen05 kernel for several new tokens per request on a bf16 cache (attention_tcm.cu): the
+// single-launch step only, head_dim 128, q_len * group <= 32.
+bool tcm_supported(int head_dim, bool fp8, int group, int q_len, bool pro);
+int launch_attention_tcm(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
+                         cudaStream_t stream);
+
 }  // namespace attn
 }  // namespace hpc

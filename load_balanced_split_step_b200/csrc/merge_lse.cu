@@ -120,6 +120,31 @@ __global__ void __launch_bounds__(kMergeLseThreads)
   }
 }
 
+// Block-table view of the parts a request-sharded rank runs: row i holds the pages of request
+// req[i] from column col0[i] on, -1 past the table. One thread per entry.
+__global__ void __launch_bounds__(kMergeLseThreads)
+    gather_pages_kernel(const int32_t* __restrict__ src, int32_t src_rows, int32_t src_cols,
+                        const int32_t* __restrict__ req, const int32_t* __restrict__ col0, int32_t n, int32_t width,
+                        int32_t* __restrict__ dst, uint32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t total = static_cast<int64_t>(n) * width;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  bool bad = false;
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < total; k += stride) {
+    const int64_t i = k / width, j = k - i * width;
+    const int32_t r = req[i], c0 = col0[i];
+    int32_t v = -1;
+    if (r < 0 || r >= src_rows || c0 < 0) {
+      bad = true;
+    } else if (c0 + j < src_cols) {
+      v = src[static_cast<int64_t>(r) * src_cols + c0 + j];
+    }
+    dst[k] = v;
+  }
+  if (bad && status) atomicOr(status, HPC_DEV_BAD_INDEX);
+}
+
 }  // namespace
 }  // namespace hpc
 
@@ -181,4 +206,22 @@ extern "C" int hpc_gather_rows(const void* src, int64_t src_rows, int64_t row_by
                  static_cast<uint4*>(dst), status);
   if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "gather_rows_kernel: %s", cudaGetErrorString(e));
   return check_launch("gather_rows_kernel");
+}
+
+extern "C" int hpc_gather_pages(const int32_t* src, int32_t src_rows, int32_t src_cols, const int32_t* req,
+                                const int32_t* col0, int32_t n, int32_t width, int32_t* dst, uint32_t* status,
+                                void* stream) {
+  if (!src || !req || !col0 || !dst) return fail(HPC_ERR_ARG, "null pointer argument");
+  if (src_rows < 0 || src_cols < 1 || n < 0 || width < 1) return fail(HPC_ERR_ARG, "sizes out of range");
+  if (n == 0) return HPC_OK;
+  const int64_t total = static_cast<int64_t>(n) * width;
+  int64_t blocks = (total + kMergeLseThreads - 1) / kMergeLseThreads;
+  const int sms = device_sm_count();
+  const int64_t cap = sms > 0 ? static_cast<int64_t>(sms) * 8 : 1024;
+  if (blocks > cap) blocks = cap;
+  const cudaError_t e = launch_pdl(gather_pages_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kMergeLseThreads), 0,
+                                   static_cast<cudaStream_t>(stream), src, src_rows, src_cols, req, col0, n, width,
+                                   dst, status);
+  if (e != cudaSuccess) return fail(HPC_ERR_CUDA, "gather_pages_kernel: %s", cudaGetErrorString(e));
+  return check_launch("gather_pages_kernel");
 }

@@ -42,7 +42,7 @@ def _reference_worker(rank, world, port, q):
     import bench
     buf = io.StringIO()
     with redirect_stdout(buf):
-        bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--cpu-seconds", "0.3"])
+        bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1"])
     q.put((rank, buf.getvalue()))
 
 

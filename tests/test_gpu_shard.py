@@ -131,19 +131,49 @@ def test_gather_rows(B):
 @pytest.mark.parametrize("kv", ["bf16", "e4m3"])
 @pytest.mark.parametrize("world", [2, 3, 4])
 def test_sharded_batch_equals_unsharded(B, world, kv):
-    spec = W.custom_spec((9000, 64, 5, 130, 2047, 700), 32, 4, 128, 64, 128, kv_dtype=kv, seed=40 + world)
+    """Eight decode steps with lengths growing by 37 tokens per step (page boundaries crossed),
+    each rank's parts run through the library and merged, every step against the oracle. The
+    ranks are emulated one after the other on this GPU; each keeps its placement across steps
+    and rebuilds its block-table view on the device."""
+    steps_n, grow = 8, 37
+    spec = W.custom_spec((9000, 64, 5, 130, 2047, 700), 32, 4, 128, 64, 128, kv_dtype=kv, seed=40 + world,
+                         steps=steps_n * grow)
     case = W.make_case(spec)
     dc = to_device(case)
     compute = S.library_compute(32, 4, kv_dtype=kv, k_scale=dc["k_scale"], v_scale=dc["v_scale"], num_ctas=37)
     steps = [S.ShardedStep(spec.seq_lens, world, r, spec.page_size, 32, 128, compute=compute) for r in range(world)]
     assert sum(len(p) for p in steps[0].plan) > len(spec.seq_lens)  # the 9000-token request is split
-    local = [st.local(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"], spec.tile_len) for st in steps]
-    outs = torch.stack([o for o, _ in local])  # what the all-gather delivers to every rank
-    lses = torch.stack([l for _, l in local])
-    out = steps[0].assemble(outs, lses)
+    for i in range(steps_n):
+        lens = [L + grow * i for L in spec.seq_lens]
+        for st in steps:
+            st.update(lens)
+        local = [st.local(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"], spec.tile_len) for st in steps]
+        outs = torch.stack([o for o, _ in local])  # what the all-gather delivers to every rank
+        lses = torch.stack([l for _, l in local])
+        out = steps[0].assemble(outs, lses)
+        torch.cuda.synchronize()
+        ref = oracle_out(case, seq_lens=torch.tensor(lens, dtype=torch.int32))
+        if kv == "bf16":
+            assert_bf16_tol(out, ref, what=f"sharded over {world}, step {i}")
+        else:
+            assert errors(out, ref)[0] <= 5e-2
+    assert all(st.replacements == steps[0].replacements for st in steps)  # the ranks agree
+
+
+def test_gather_pages(B):
+    bt = torch.arange(40, dtype=torch.int32).reshape(4, 10).cuda()
+    req = torch.tensor([2, 0, 3], dtype=torch.int32, device="cuda")
+    col0 = torch.tensor([3, 0, 9], dtype=torch.int32, device="cuda")
+    st = B.new_status("cuda")
+    out = B.gather_pages(bt, req, col0, status=st)
     torch.cuda.synchronize()
-    ref = oracle_out(case)
-    if kv == "bf16":
-        assert_bf16_tol(out, ref, what=f"sharded over {world}")
-    else:
-        assert errors(out, ref)[0] <= 5e-2
+    want = torch.full((3, 10), -1, dtype=torch.int32)
+    want[0, :7] = bt.cpu()[2, 3:]
+    want[1] = bt.cpu()[0]
+    want[2, :1] = bt.cpu()[3, 9:]
+    assert int(st.item()) == 0 and torch.equal(out.cpu(), want)
+    req[1] = 4  # outside the table: a row of -1 and the status bit
+    out = B.gather_pages(bt, req, col0, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == B.DEV_STATUS["bad_index"] and torch.all(out[1] == -1)
+    assert torch.equal(out.cpu()[0], want[0])
