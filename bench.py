@@ -73,6 +73,10 @@ def parse_args(argv=None):
     ap.add_argument("--e4m3-kernel", default="mma", choices=["mma", "tcgen05"], help="kernel for E4M3 caches")
     ap.add_argument("--multi-kernel", default="default", choices=["default", "mma", "tcgen05"],
                     help="kernel for several new tokens per request (--q-len > 1)")
+    ap.add_argument("--record-traffic", default=None, metavar="CSV",
+                    help="write profiles/traffic.json's entry for --workload from an ncu CSV of one attention launch "
+                         "(dram__bytes_read.sum, dram__bytes_write.sum); with --requests N the capture covered the "
+                         "first N requests and is scaled to the full workload by algorithmic bytes")
     ap.add_argument("--trace", action="store_true",
                     help="run the HPC_TRACE build of the library and print a per-CTA load summary of the single "
                          "launch (idle tail, plan and first-data latency) instead of the benchmark line")
@@ -708,23 +712,46 @@ def kernel_source_hash():
 
 
 def load_traffic(workload):
-    """DRAM bytes per attention launch from the committed ncu summary, or None when the
-    kernel source has changed since those counters were taken."""
-    p = os.path.join(ROOT, "profiles", f"attention_{workload}_dram.md")
+    """DRAM bytes per attention launch at this workload's full size, from profiles/traffic.json
+    (written from an ncu capture; see profiles/attention_<workload>_dram.md for the command), or
+    None when the kernel source has changed since those counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    vals = {}
     with open(p) as f:
-        for line in f:
-            if ":" in line and not line.startswith(("#", "|", " ")):
-                k, v = line.split(":", 1)
-                vals[k.strip()] = v.strip()
-    if vals.get("source_sha256_16") != kernel_source_hash():
+        entry = json.load(f).get(workload)
+    if not entry or entry.get("source_sha256_16") != kernel_source_hash():
         return None
-    try:
-        return int(vals["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    return int(entry["traffic_bytes_per_launch"])
+
+
+def record_traffic(args):
+    """profiles/traffic.json entry of --workload from an ncu CSV (see --record-traffic)."""
+    import csv
+    units = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    got = {}
+    with open(args.record_traffic) as f:
+        rows = [ln for ln in f if ln.startswith('"')]
+    for row in csv.DictReader(rows):
+        name = row.get("Metric Name")
+        if name in ("dram__bytes_read.sum", "dram__bytes_write.sum") and name not in got:
+            got[name] = float(row["Metric Value"].replace(",", "")) * units.get(row["Metric Unit"], 1)
+    if len(got) != 2:
+        raise SystemExit(f"{args.record_traffic}: no dram__bytes_read.sum / dram__bytes_write.sum rows")
+    sample = workload_spec(args)
+    full = W.config_spec(args.workload)
+    scale = W.algorithmic_bytes(full) / W.algorithmic_bytes(sample)
+    traffic = (got["dram__bytes_read.sum"] + got["dram__bytes_write.sum"]) * scale
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    data = json.load(open(p)) if os.path.exists(p) else {}
+    data[args.workload] = {"traffic_bytes_per_launch": int(round(traffic)), "source_sha256_16": kernel_source_hash(),
+                           "read_bytes": int(got["dram__bytes_read.sum"]), "write_bytes": int(got["dram__bytes_write.sum"]),
+                           "captured_requests": sample.batch, "scale_to_full": round(scale, 6),
+                           "algorithmic_bytes_full": int(W.algorithmic_bytes(full))}
+    with open(p, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return {"workload": args.workload, **data[args.workload]}
 
 
 def device_case(case, dev, layout="HND"):
@@ -994,7 +1021,9 @@ def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_init(args)
     try:
-        if args.trace:
+        if args.record_traffic:
+            line = record_traffic(args)
+        elif args.trace:
             line = run_trace(args, local)
         elif args.impl == "reference":
             line = run_reference(args, rank, world)

@@ -121,7 +121,11 @@ __device__ __forceinline__ void consume_blocks(uint32_t kbase, uint32_t vbase, u
   const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
   // -inf only when no token has been live yet (a masked stage): the reference 0 keeps every
   // exponential at 0 instead of NaN
-  const float mr0 = mn0 == -INFINITY ? 0.f : mn0, mr1 = mn1 == -INFINITY ? 0.f : mn1;
+  float mr0 = mn0, mr1 = mn1;
+  if (tail) {  // only a tail call can have no live token at all
+    if (mn0 == -INFINITY) mr0 = 0.f;
+    if (mn1 == -INFINITY) mr1 = 0.f;
+  }
   const float al0 = exp2f(m0 - mr0), al1 = exp2f(m1 - mr1);
   float pr[NB][4];
   float add0 = 0.f, add1 = 0.f;
@@ -678,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kbase = ring_u32 + stage * p.stage_bytes;
           const uint32_t vbase = kbase + S::kPlanes * p.plane_bytes;
           const bool bad_stage = s_bad[stage] != 0;
-          if (FP8 && nb == 4)
+          if (nb == 4)
             consume_blocks<D, FP8, 4>(kbase, vbase, p.plane_bytes, 16 * my_first, tb, lim, bad_stage, qf, score_scale,
                                       m0, m1, l0, l1, o, lane);
           else if (nb == 2)

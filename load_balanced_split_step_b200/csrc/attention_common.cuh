@@ -83,9 +83,12 @@ struct ItemInfo {
 // 16-token blocks that one consumer warp takes from a stage of `bpc` blocks. Two blocks give
 // two independent MMA chains. An E4M3 stage carries half the bytes per token, so the fixed
 // per-call softmax work (row max across lanes, rescale factors) and the stage handshake weigh
-// twice as much per byte: there a warp takes up to four blocks, a whole 64-token stage.
+// twice as much per byte: there a warp takes up to four blocks, a whole 64-token stage. With
+// several new tokens on a bf16 cache a warp also takes four: the stage then needs q_pad warps
+// instead of 2 q_pad, so two stages are consumed at once instead of one, and each warp has four
+// independent chains (on the heavy-tailed batch with four new tokens: 1055 -> 590 us).
 __host__ __device__ __forceinline__ int blocks_per_warp(int bpc, bool fp8, int q_pad = 1) {
-  if (fp8 && bpc >= 4 && q_pad == 1) return 4;
+  if (bpc >= 4 && (fp8 ? q_pad == 1 : q_pad > 1)) return 4;
   return bpc >= 2 ? 2 : 1;
 }
 
