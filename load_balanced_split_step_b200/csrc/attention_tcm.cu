@@ -25,7 +25,8 @@
 //  * warp 9, producer: 128-token stages. K and V have rings of their own (2 and 3 slots of 32 KB),
 //    so that a K slot is refilled as soon as its S^T product is done. Boxes of up to 64 tokens never
 //    cross a page. Boxes past an item's last token are not loaded, and a page id outside the pool
-//    is never handed to TMA (page 0 stands in, and the softmax masks the box).
+//    is never handed to TMA (page 0 stands in; the softmax reads the page ids of its own tokens and
+//    leaves those tokens out).
 //  * warp 8, one lane issues the products in a non-blocking loop (mbarrier.test_wait).
 //  * warps 0-7, softmax: two warpgroups take alternate stages, each with its own running state
 //    for the item (row maxima, sums and rescale factors in shared memory, output in registers);
@@ -153,7 +154,6 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   __shared__ int s_flag;
   __shared__ int s_rec_n;
   __shared__ int32_t s_pages[32];
-  __shared__ uint8_t s_badbox[kTmVS];            // per V slot: boxes whose page id was out of range
   __shared__ __align__(16) float s_redmax[2][4][kTmN];  // per warpgroup: per-warp row maxima of a stage
   __shared__ __align__(16) float s_redsum[2][4][kTmN];  // per warpgroup: per-warp row sums of a stage
   __shared__ __align__(16) float s_m[2][kTmN];          // per warpgroup: running row maxima (log2 units)
@@ -209,19 +209,19 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   plan_in_kernel<kTmD>(p, reinterpret_cast<int64_t*>(kring), s_scan, s_walk, cursor, chunk);
   const int C = p.chunk_tokens;
   const int P = p.page_size;
+  const int p_shift = __ffs(P) - 1;
   const int cps = kTmTok / C;  // boxes per stage
 
   if (warp == kTmProducerWarp) {
     // ------------------------------------------------------------------ producer
     const uint64_t policy = l2_policy_evict_first();
-    const int p_shift = __ffs(P) - 1;
     int64_t n = 0;                  // stages begun
     int64_t filled[2] = {0, 0};     // fills issued: K, V
     bool ok = true;
     uint32_t bad = 0;
     ItemInfo x;
     while (ok && cursor.next(p, x)) {
-      const int32_t* bt = p.block_table + x.req * p.max_pages + (x.tok0 >> p_shift);
+      const int32_t* bt = p.block_table + static_cast<int64_t>(x.req) * p.max_pages + (x.tok0 >> p_shift);
       const int off0 = static_cast<int>(x.tok0 & (P - 1));
       const int64_t nreal = x.tok1 > x.tok0 ? (x.tok1 - x.tok0 + C - 1) / C : 0;  // boxes with item tokens
       const int64_t nbox = tm_stages(x) * cps;
@@ -236,12 +236,10 @@ __global__ void __launch_bounds__(kTmThreads, 1)
             const int64_t bi = cb + k;
             const int nb = static_cast<int>(nreal - bi < cps ? nreal - bi : cps);
             const uint32_t tx = static_cast<uint32_t>(nb) * 2u * C * 128u;
-            uint32_t mask = 0;
             for (int kk = 0; kk < nb; ++kk) {
               const int32_t pg = s_pages[k + kk];
-              if (pg < 0 || pg >= p.num_pages) mask |= 1u << kk;
+              if (pg < 0 || pg >= p.num_pages) bad |= HPC_DEV_BAD_PAGE;
             }
-            if (mask) bad |= HPC_DEV_BAD_PAGE;
             for (int half = 0; half < 2 && ok; ++half) {  // K, then V
               const int slot = static_cast<int>(half ? n % kTmVS : n % kTmKS);
               const int depth = half ? kTmVS : kTmKS;
@@ -252,13 +250,11 @@ __global__ void __launch_bounds__(kTmThreads, 1)
                 bad |= HPC_DEV_TIMEOUT;
                 break;
               }
-              // the softmax reads the mask after its wait on this stage's V fill
-              if (half) s_badbox[slot] = static_cast<uint8_t>(mask);
               mbar_arrive_expect_tx(full, tx);
               const uint32_t base = smem_u32(half ? vring : kring) + slot * kTmKV;
               for (int kk = 0; kk < nb; ++kk) {
                 int32_t page = s_pages[k + kk];
-                if (page < 0 || page >= p.num_pages) page = 0;  // stand-in; the softmax masks the box
+                if (page < 0 || page >= p.num_pages) page = 0;  // stand-in; the softmax leaves its tokens out
                 const int off = static_cast<int>((off0 + (bi + kk) * C) & (P - 1));
                 const int c1 = p.nhd ? x.kvh : off, c2 = p.nhd ? off : x.kvh;
                 const uint32_t dst = base + kk * C * 128;
@@ -482,6 +478,14 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         // P buffer b was last read by the O^T products of this warpgroup's previous stage, which
         // the issuing lane may start after this stage's S^T product: fold that stage first (its
         // wait covers the products' completion), before the buffer is overwritten below
+        // this thread's token: past the item, or on a page outside the pool, it is dead (the page id
+        // is read here, ahead of the waits, so that its latency is hidden)
+        const int64_t t = x.tok0 + (k - n0) * kTmTok + i;
+        bool tok_ok = t < x.tok1;
+        if (tok_ok) {
+          const int32_t pg = p.block_table[static_cast<int64_t>(x.req) * p.max_pages + (t >> p_shift)];
+          tok_ok = pg >= 0 && pg < p.num_pages;
+        }
         if (last_own >= 0) fold(last_own);
         float sv[kTmN];
         if (wait(bar.s_full(b), static_cast<uint32_t>((k >> 1) & 1))) {
@@ -494,35 +498,29 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar.s_free(b));
-        // the V fill of this stage: its slot is refilled only after this stage's O^T product,
-        // which waits for the P^T written below, so the phase cannot have moved on
-        const int vs = static_cast<int>(k % kTmVS);
-        uint32_t badm = 0;
-        if (wait(bar.v_full(vs), static_cast<uint32_t>((k / kTmVS) & 1))) badm = s_badbox[vs];
-        const int64_t t = x.tok0 + (k - n0) * kTmTok + i;
-        const bool tok_ok = t < x.tok1 && !((badm >> (i / C)) & 1u);
-        if (!tok_ok) {
-          // this token's V row may hold anything (even NaN): zero it, so 0 * v stays 0
-          uint8_t* vrow = vring + vs * kTmKV + i * 128;
+        // A dead token's V row may hold anything (even NaN): it is zeroed, so that 0 * v stays 0.
+        // Only a warp with a dead token waits for the stage's V fill (its slot is refilled only after
+        // this stage's O^T product, which waits for the P^T written below, so the phase cannot have
+        // moved on); the others never wait on V.
+        if (__any_sync(0xffffffffu, !tok_ok)) {
+          const int vs = static_cast<int>(k % kTmVS);
+          if (wait(bar.v_full(vs), static_cast<uint32_t>((k / kTmVS) & 1)) && !tok_ok) {
+            uint8_t* vrow = vring + vs * kTmKV + i * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            reinterpret_cast<uint4*>(vrow)[c] = make_uint4(0u, 0u, 0u, 0u);
-            reinterpret_cast<uint4*>(vrow + kTmPlane)[c] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-        // row c is query token c / group: it sits at L - q_len + c / group and sees tokens up to it
-        {
-          const int64_t lim0 = L - q_len;
-          int tq = 0, h = 0;
-#pragma unroll
-          for (int c = 0; c < kTmN; ++c) {
-            const bool live = tok_ok && c < rows && t <= lim0 + tq;
-            sv[c] = live ? sv[c] * p.score_scale : -INFINITY;
-            if (++h == group) {
-              h = 0;
-              ++tq;
+            for (int c = 0; c < 8; ++c) {
+              reinterpret_cast<uint4*>(vrow)[c] = make_uint4(0u, 0u, 0u, 0u);
+              reinterpret_cast<uint4*>(vrow + kTmPlane)[c] = make_uint4(0u, 0u, 0u, 0u);
             }
           }
+        }
+        // row c is query token c / group: it sits at L - q_len + c / group and sees tokens up to
+        // it, so token t is live for the rows c in [c_lo, rows) with c_lo = group * (t - (L - q_len))
+        {
+          const int64_t behind = t - (L - q_len);  // query tokens this token is ahead of (<= 0: all see it)
+          const int c_lo = behind <= 0 ? 0 : (behind >= q_len ? kTmN : static_cast<int>(behind) * group);
+          const int c_hi = tok_ok ? rows : 0;
+#pragma unroll
+          for (int c = 0; c < kTmN; ++c) sv[c] = (c >= c_lo && c < c_hi) ? sv[c] * p.score_scale : -INFINITY;
         }
         // row maxima over the warpgroup's 128 tokens; lane c of warp 0 sets row c's new maximum
         // and rescale factor
@@ -530,6 +528,9 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         named_barrier_sync(wbar, kTmSoftmax);
         float* a_k = s_a[w][(k >> 1) & 1];
         if (wq == 0) {
+          if (last_own >= 0)  // the previous own stage's row sums, with that stage's rescale factor
+            s_l[w][lane] = s_l[w][lane] * s_a[w][(last_own >> 1) & 1][lane] +
+                           ((s_redsum[w][0][lane] + s_redsum[w][1][lane]) + (s_redsum[w][2][lane] + s_redsum[w][3][lane]));
           const float mx = fmaxf(fmaxf(s_redmax[w][0][lane], s_redmax[w][1][lane]),
                                  fmaxf(s_redmax[w][2][lane], s_redmax[w][3][lane]));
           const float mo = s_m[w][lane], mn = fmaxf(mo, mx);
@@ -562,17 +563,20 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar.p_full(b));
-        // row sums of p over the 128 tokens; warp 0 folds them into the running sums
+        // row sums of p over the 128 tokens; warp 0 folds them into the running sums during this
+        // warpgroup's next stage (or at the item end)
         s_redsum[w][wq][lane] = warp_reduce32<false>(sv, lane);
-        named_barrier_sync(wbar, kTmSoftmax);
-        if (wq == 0)
-          s_l[w][lane] = s_l[w][lane] * a_k[lane] + ((s_redsum[w][0][lane] + s_redsum[w][1][lane]) +
-                                                     (s_redsum[w][2][lane] + s_redsum[w][3][lane]));
         if (w == 0 && have_next && k + 2 >= n_end) build_next();
         last_own = k;
       }
       if (w == 0 && have_next && !built_next) build_next();  // no stage of this item here
-      if (last_own >= 0) fold(last_own);
+      if (last_own >= 0) {
+        fold(last_own);
+        named_barrier_sync(wbar, kTmSoftmax);  // the last stage's row sums are written
+        if (wq == 0)
+          s_l[w][lane] = s_l[w][lane] * s_a[w][(last_own >> 1) & 1][lane] +
+                         ((s_redsum[w][0][lane] + s_redsum[w][1][lane]) + (s_redsum[w][2][lane] + s_redsum[w][3][lane]));
+      }
       n = n_end;
 
       // ---- item end: the two warpgroups' states combined by log-sum-exp. The exchange and merge
