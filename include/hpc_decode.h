@@ -159,7 +159,8 @@ typedef struct {
  *   multi_kernel: HPC_MULTI_DEFAULT, HPC_MULTI_MMA or HPC_MULTI_TCGEN05: the kernel for
  *                 hpc_decode_step_multi with q_len > 1. The tcgen05 kernel serves bf16 caches with
  *                 head_dim 128 and q_len * (num_heads / kv_heads) <= 32; elsewhere the choice is
- *                 ignored. The default is HPC_MULTI_MMA.
+ *                 ignored. The default takes the tcgen05 kernel for q_len >= 3 where it applies
+ *                 and the mma.sync consumers otherwise.
  *   record:       single-launch steps only: device buffer of hpc_step_record_bytes(num_ctas,
  *                 record_items) bytes that receives every CTA's hpc_cta_record, or NULL.
  *   trace:        device uint64 [num_ctas][HPC_TRACE_WORDS], or NULL. Only a library built with

@@ -971,7 +971,7 @@ namespace {
 struct Options {
   int32_t item_cost = HPC_ITEM_COST_DEFAULT;
   bool tc = false;
-  bool tcm = false;  // several new tokens on the tcgen05 kernel
+  int32_t multi_kernel = HPC_MULTI_DEFAULT;  // several new tokens: which kernel
   uint8_t* record = nullptr;
   int32_t record_items = 0;
   uint64_t* trace = nullptr;
@@ -996,7 +996,7 @@ int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
   if (o->trace && (reinterpret_cast<uintptr_t>(o->trace) & 7)) return fail(HPC_ERR_ALIGN, "trace must be 8-byte aligned");
   out->item_cost = o->item_cost;
   out->tc = o->e4m3_kernel == HPC_E4M3_TCGEN05;
-  out->tcm = o->multi_kernel == HPC_MULTI_TCGEN05;
+  out->multi_kernel = o->multi_kernel;
   out->record = static_cast<uint8_t*>(o->record);
   out->record_items = o->record ? o->record_items : 0;
   out->trace = o->trace;
@@ -1265,9 +1265,13 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.record_items = opt.record_items;
   prm.trace = opt.trace;
   const bool fp8 = kv_dtype == HPC_E4M3;
-  if (!pro && q_len > 1)
+  if (!pro && q_len > 1) {
+    // by default three or four new tokens go to the tcgen05 kernel (one product per stage for
+    // all of them), two to the mma.sync consumers, where they are faster
+    const bool tcm = opt.multi_kernel == HPC_MULTI_TCGEN05 || (opt.multi_kernel == HPC_MULTI_DEFAULT && q_len >= 3);
     return dispatch<true, false, true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem,
-                                       static_cast<cudaStream_t>(stream), opt.tcm);
+                                       static_cast<cudaStream_t>(stream), tcm);
+  }
   if (!pro)
     return dispatch<true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem, static_cast<cudaStream_t>(stream));
   prm.qkv = static_cast<const __nv_bfloat16*>(pro->qkv);

@@ -46,12 +46,15 @@ def _check(out, ref, kv, what):
         assert mx <= 5e-2, (what, mx)
 
 
+@pytest.mark.parametrize("mk", ["default", "mma"])
 @pytest.mark.parametrize("T", [1, 2, 3, 4])
 @pytest.mark.parametrize("kv,Hq,Hkv,D,P,tl", [
     ("bf16", 8, 2, 64, 16, 32), ("bf16", 64, 8, 128, 64, 128), ("bf16", 16, 4, 128, 32, 32),
     ("e4m3", 64, 8, 128, 64, 128), ("e4m3", 16, 2, 128, 16, 48),
 ])
-def test_matches_oracle(B, T, kv, Hq, Hkv, D, P, tl):
+def test_matches_oracle(B, T, kv, Hq, Hkv, D, P, tl, mk):
+    """The default kernel (tcgen05 for three or four tokens on a bf16 cache with head_dim 128)
+    and the mma.sync consumers, against the oracle."""
     if tl % P and P % tl:
         pytest.skip("tile/page combination not supported")
     lens = (T, T + 1, 15, 16, 17, 64, 65, 129, 300, 1000, 2049)
@@ -60,9 +63,9 @@ def test_matches_oracle(B, T, kv, Hq, Hkv, D, P, tl):
     dc = to_device(case)
     ref = _oracle(case)
     for G in (5, 148):
-        out, st, _ = _run(B, spec, dc, G)
+        out, st, _ = _run(B, spec, dc, G, multi_kernel=mk)
         assert st == 0
-        _check(out, ref, kv, f"q_len {T} {kv} {(Hq, Hkv, D, P, tl)} G={G}")
+        _check(out, ref, kv, f"q_len {T} {kv} {(Hq, Hkv, D, P, tl)} G={G} {mk}")
 
 
 def test_one_token_is_the_single_launch_step(B):
