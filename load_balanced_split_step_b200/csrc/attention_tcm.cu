@@ -17,9 +17,10 @@
 // M = 64 accumulator takes the lower half of each 32-lane subpartition (row m at lane
 // m % 16 + 32 (m / 16)); the upper halves hold a second one. Stages therefore go in pairs: the
 // even stage of a pair in the lower halves, the odd one in the upper halves, both in the same
-// columns. Query rows 0..15 live in subpartition 0 and rows 16..31 in subpartition 1, so warps 0
-// and 1 run the softmax, each thread one (row, stage) with its 128 scores: no reduction across
-// threads. P (a bf16 high part and residual, two bf16 per 32-bit column) is written over the
+// columns. Query rows 0..15 live in subpartition 0 and rows 16..31 in subpartition 1; each of
+// the two is worked by two warps (warp % 4 is the subpartition a warp reaches), one per half of
+// the 128 token columns, so a thread holds one (row, stage) with 64 scores and only the two
+// warps' row maxima and sums are exchanged. P (a bf16 high part and residual, two bf16 per 32-bit column) is written over the
 // stage's own S columns and is the A operand of the O product straight from tensor memory; V is
 // an MN-major B operand read from its swizzled TMA tile. Shared memory then holds only Q and the
 // K and V rings (three 32 KB slots each), the bytes a CTA keeps in flight. A new S is issued into
@@ -33,16 +34,16 @@
 // p), and computes every exponential and then selects: a branch per token cost several times the
 // whole pass.
 //
-// Roles (160 threads): warps 0-1 softmax (and Q tiles, item ends, merges); warp 2, one lane issues
-// the products in a non-blocking loop; warps 3 and 4 the TMA producers of K and of V. Every wait is
-// bounded (2 s) and ends in HPC_DEV_TIMEOUT; tensor memory is freed on every path.
+// Roles (224 threads): warps 0, 1, 4, 5 softmax (and Q tiles, item ends, merges); warp 2, one lane
+// issues the products in a non-blocking loop; warps 3 and 6 the TMA producers of K and of V. Every
+// wait is bounded (2 s) and ends in HPC_DEV_TIMEOUT; tensor memory is freed on every path.
 #include "attention_common.cuh"
 
 namespace hpc {
 namespace attn {
 namespace {
 
-constexpr int kTmThreads = 160;
+constexpr int kTmThreads = 224;
 constexpr int kTmTok = 128;               // tokens per stage: N of the S product, K of the O product
 constexpr int kTmD = 128;                 // head_dim
 constexpr int kTmN = 32;                  // query rows read back (q_len x group <= 32)
@@ -53,8 +54,8 @@ constexpr int kTmQPlane = kTmN * 128;     // one plane of the Q tile: 4 KB
 constexpr int kTmQ = 2 * kTmQPlane;       // Q tile: 8 KB
 constexpr uint32_t kTmCols = 512;         // S[2] at 0 and 128 (P over S), O at 256
 constexpr int kTmSB = 2;                  // S buffers: pair p uses buffer p % 2
-constexpr int kTmSoftThreads = 64;        // warps 0 and 1
-constexpr int kTmMmaWarp = 2, kTmProducerWarp = 3;  // producers: warp 3 K, warp 4 V
+constexpr int kTmSoftThreads = 128;       // warps 0, 1, 4, 5
+constexpr int kTmMmaWarp = 2, kTmProducerK = 3, kTmProducerV = 6;
 constexpr float kTmMove = 8.f;            // the running maximum moves when exceeded by more (log2 units)
 // instruction descriptors: fp32 accumulate, bf16 x bf16, M = 64, N = 128; the O product reads V
 // (its B) MN-major
@@ -146,6 +147,8 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   __shared__ int s_rec_n;
   __shared__ int32_t s_pages[2][32];
   __shared__ __align__(16) float s_merge[1024];
+  __shared__ float s_px[2][2][2][32];  // softmax: [pair parity][subpartition][column half][lane] partial maxima
+  __shared__ float s_pl[2][2][32];     // softmax, item end: [subpartition][column half][lane] partial sums
   __shared__ uint32_t s_tmem;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qt = smem;
@@ -154,6 +157,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   const TmBars bar{smem_u32(smem + kTmOffBar)};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q_len = p.q_len, group = p.group, rows = q_len * group;  // rows <= kTmN (checked on the host)
+#ifdef HPC_TRACE
+  uint64_t* trace = p.trace ? p.trace + static_cast<size_t>(blockIdx.x) * HPC_TRACE_WORDS : nullptr;
+  if (trace && threadIdx.x == 0) {
+    trace[0] = global_timer_ns();
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    trace[7] = smid;
+    trace[2] = trace[3] = 0;
+  }
+#endif
 
   if (threadIdx.x == 0) {
     s_rec_n = 0;
@@ -168,16 +181,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
     for (int b = 0; b < kTmSB; ++b) mbar_init(bar.buf_free(b), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar.s_full(b), 1);
-      mbar_init(bar.p_full(b), 2);
+      mbar_init(bar.p_full(b), 4);
       mbar_init(bar.o_done(b), 1);
-      mbar_init(bar.q_full(b), 2);
+      mbar_init(bar.q_full(b), 4);
       mbar_init(bar.q_free(b), 1);
     }
     mbar_init(bar.done(), 1);
     fence_barrier_init();
   }
   if (warp == kTmMmaWarp) tmem_alloc(smem_u32(&s_tmem), kTmCols);
-  if (warp == kTmProducerWarp && lane == 0) {
+  if (warp == kTmProducerK && lane == 0) {
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
   }
@@ -192,17 +205,20 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   int64_t chunk = 0;
   // the per-request tile prefix lives in the K ring until the first TMA copy is issued
   plan_in_kernel<kTmD>(p, reinterpret_cast<int64_t*>(kring), s_scan, s_walk, cursor, chunk);
+#ifdef HPC_TRACE
+  if (trace && threadIdx.x == 0) trace[1] = global_timer_ns();
+#endif
   const int C = p.chunk_tokens;
   const int P = p.page_size;
   const int p_shift = __ffs(P) - 1;
   const int cps = kTmTok / C;  // boxes per stage
   const int c_shift = __ffs(C) - 1;
 
-  if (warp >= kTmProducerWarp) {
+  if (warp == kTmProducerK || warp == kTmProducerV) {
     // ------------------------------------------------------------------ producers
     // Warp 3 fills the K ring and warp 4 the V ring, each on its own, so that a K fill never waits
     // behind a V slot (a V slot is held until its stage's O product, after the softmax).
-    const int half = warp - kTmProducerWarp;  // 0: K, 1: V
+    const int half = warp == kTmProducerV ? 1 : 0;  // 0: K, 1: V
     const int depth = half ? kTmVS : kTmKS;
     const CUtensorMap* tmap = half ? &tm_v : &tm_k;
     uint8_t* ring = half ? vring : kring;
@@ -265,6 +281,12 @@ __global__ void __launch_bounds__(kTmThreads, 1)
           bad |= HPC_DEV_TIMEOUT;
       }
       if (bad) atomicOr(p.status, bad);
+#ifdef HPC_TRACE
+      if (trace && !half) {  // the K producer: its end and the 128-token stages it filled
+        trace[4] = global_timer_ns();
+        trace[6] = static_cast<uint64_t>(n);
+      }
+#endif
     }
   } else if (warp == kTmMmaWarp) {
     // ------------------------------------------------------------------ products
@@ -388,16 +410,21 @@ __global__ void __launch_bounds__(kTmThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ softmax (warps 0 and 1)
-    // Thread (warp w, lane l) owns query row r = 16 w + l % 16 of the stages of half h = l / 16:
-    // tensor-memory lane 32 w + l of every S, P and O. Control flow is uniform within each warp;
-    // per-lane waits (a half's O product) are bounded and do not diverge the collective calls.
-    const int w = warp, h = lane >> 4;
-    const int r = 16 * w + (lane & 15);
-    const int tid = threadIdx.x;  // 0 .. 63
+    // ------------------------------------------------------------------ softmax (warps 0, 1, 4, 5)
+    // Warp w works on subpartition sp = w % 4 and on column half hb = w / 4 of every stage (tokens
+    // 64 hb .. 64 hb + 63, and the same d columns of O). Thread (w, lane l) owns query row
+    // r = 16 sp + l % 16 of the stages of half h = l / 16: tensor-memory lane 32 sp + l. The two
+    // warps of a subpartition exchange their row maxima once per pair (shared memory and a named
+    // barrier of 64 threads) and their row sums at the item end. Control flow is uniform within
+    // each warp; per-lane waits (a half's O product) are bounded and do not diverge the collective
+    // calls.
+    const int sp = warp & 3, hb = warp >> 2, h = lane >> 4;
+    const int r = 16 * sp + (lane & 15);
+    const int tid = 64 * hb + 32 * sp + lane;  // 0 .. 127
+    const int pbar = 2 + sp;                   // named barrier of the subpartition's two warps
     const bool row_live = r < rows;
     const int tq = r / group, hd = r - tq * group;
-    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * w) << 16);  // this warp's lanes
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * sp) << 16);  // this warp's lanes
     zero_empty_requests<kTmD>(p, tid, kTmSoftThreads);
     bool ok = true;
     auto fail_wait = [&]() {
@@ -415,15 +442,15 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       return got;
     };
-    // Q tile of item y into buffer jy % 2 (warps 0 and 1). Row c = t * group + g holds query token
-    // t of head kv_head * group + g; rows past q_len * group are zero. Thread tid writes 16-byte
-    // chunks tid, tid + 64, ... of the 32 x 256-byte tile.
+    // Q tile of item y into buffer jy % 2 (the four softmax warps). Row c = t * group + g holds
+    // query token t of head kv_head * group + g; rows past q_len * group are zero. Thread tid
+    // writes 16-byte chunks tid, tid + 128, tid + 256, tid + 384 of the 32 x 256-byte tile.
     auto build_q = [&](const ItemInfo& y, int jy) {
       const int qb = jy & 1;
       if (jy >= 2) wait_warp(bar.q_free(qb), static_cast<uint32_t>(((jy >> 1) - 1) & 1));
       uint8_t* qtile = qt + qb * kTmQ;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 4; ++k) {
         const int qi = tid + kTmSoftThreads * k, c = qi >> 4, cc = qi & 15;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (c < rows) {
@@ -503,16 +530,23 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         };
         wait_warp(bar.s_full(buf), static_cast<uint32_t>((gp >> 1) & 1));
         tc_fence_after();
-        // two passes over the stage's 128 scores (32 at a time): the maximum, then p
+#ifdef HPC_TRACE
+        if (trace && tid == 0 && trace[2] == 0) trace[2] = global_timer_ns();
+#endif
+        // two passes over this warp's 64 scores of the stage (32 at a time): the maximum (combined
+        // with the other column half's through shared memory), then p
         float mx = -INFINITY;
 #pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c4 = 2 * hb; c4 < 2 * hb + 2; ++c4) {
           const uint32_t lv = chunk_live(c4);
           float v[32];
           tmem_ld32(tl + 128u * buf + 32 * c4, v);
 #pragma unroll
           for (int c = 0; c < 32; ++c) mx = fmaxf(mx, ((lv >> c) & 1u) ? v[c] * p.score_scale : -INFINITY);
         }
+        s_px[gp & 1][sp][hb][lane] = mx;
+        named_barrier_sync(pbar, 64);
+        mx = fmaxf(mx, s_px[gp & 1][sp][hb ^ 1][lane]);
         // the running maximum: set by the first stage of the half, or by a live stage before which
         // the half saw no live token (its O holds zeros); afterwards moved only past the margin,
         // with O and the sum rescaled
@@ -534,7 +568,7 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         const float mr = m_used == -INFINITY ? 0.f : m_used;
         float add = 0.f;
 #pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c4 = 2 * hb; c4 < 2 * hb + 2; ++c4) {
           const uint32_t lv = chunk_live(c4);
           float v[32];
           tmem_ld32(tl + 128u * buf + 32 * c4, v);
@@ -564,7 +598,7 @@ __global__ void __launch_bounds__(kTmThreads, 1)
           ok = __all_sync(0xffffffffu, ok);
           tc_fence_after();
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c4 = 2 * hb; c4 < 2 * hb + 2; ++c4) {  // this warp's 64 columns of O
             float v[32];
             tmem_ld32(tl + 256 + 32 * c4, v);
             uint32_t o0[16], o1[16];
@@ -578,16 +612,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
           }
         }
         // tokens dead for every row (past the item, or on a page outside the pool): their V rows
-        // may hold anything (even NaN) and are zeroed, so that 0 * v stays 0. The 32 threads of a
-        // half take tokens q, q + 32, q + 64, q + 96 (q = 16 w + l % 16) of their stage.
+        // may hold anything (even NaN) and are zeroed, so that 0 * v stays 0. The 64 threads of a
+        // half take tokens q and q + 64 (q = 16 (2 hb + sp) + l % 16) of their stage.
         if (__any_sync(0xffffffffu, dead_any)) {
           if (dead_any) {
             const int vs = static_cast<int>(k % kTmVS);
             if (mbar_wait(bar.v_full(vs), static_cast<uint32_t>((k / kTmVS) & 1))) {
-              const int q0 = 16 * w + (lane & 15);
+              const int q0 = 16 * (2 * hb + sp) + (lane & 15);
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int c = q0 + 32 * u;
+              for (int u = 0; u < 2; ++u) {
+                const int c = q0 + 64 * u;
                 if (t0 + c >= x.tok1 || ((badm >> (c >> c_shift)) & 1u)) {
                   uint8_t* vrow = vring + vs * kTmKV + c * 128;
 #pragma unroll
@@ -617,7 +651,11 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       pair0 += npairs;
 
       // ---- item end: the two halves combined by log-sum-exp (lanes l and l ^ 16 hold the same
-      // row), once each half's last O product is complete
+      // row), once each half's last O product is complete. A row's sum is split over the two
+      // column halves' warps.
+      s_pl[sp][hb][lane] = l_sum;
+      named_barrier_sync(pbar, 64);
+      l_sum += s_pl[sp][hb ^ 1][lane];
       if (had && !mbar_wait(bar.o_done(h), static_cast<uint32_t>((pv_cnt - 1) & 1))) fail_wait();
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
@@ -630,7 +668,7 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       const float Lt = (had ? l_sum * f_s : 0.f) + (had_o ? l_o * f_p : 0.f);
       const int64_t head = static_cast<int64_t>(x.kvh) * group + hd;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c4 = 2 * hb; c4 < 2 * hb + 2; ++c4) {  // this warp's 64 columns of O
         float v[32];
         tmem_ld32(tl + 256 + 32 * c4, v);
         float mine[16];
@@ -696,6 +734,12 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       have = cur.next(p, x);
     }
     if (p.record && tid == 0) record_header(p, s_walk[0], s_walk[1], s_walk[7], s_rec_n);
+#ifdef HPC_TRACE
+    if (trace && tid == 0) {
+      if (s_rec_n > 0) trace[3] = global_timer_ns();
+      trace[5] = static_cast<uint64_t>(s_rec_n);
+    }
+#endif
   }
 
   tc_fence_before();

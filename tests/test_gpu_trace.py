@@ -106,3 +106,36 @@ def test_default_build_refuses_a_trace_buffer():
     with pytest.raises(B.HpcError, match="HPC_TRACE"):
         B.decode_step_fused(dc["q"], dc["k_pages"], dc["v_pages"], dc["block_table"], dc["seq_lens"], 8, 2, 32,
                             num_ctas=8, trace=trace)
+
+
+def test_trace_several_tokens_tcgen05(BT):
+    """Four new tokens per request on the tcgen05 kernel (the default for three or four): the
+    same stamps, with the stage count in its 128-token stages."""
+    spec = W.custom_spec((4, 17, 300, 1000, 2049, 5000, 64, 129), 32, 4, 128, 64, 128, seed=93, q_len=4)
+    case = W.make_case(spec)
+    dc = to_device(case)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    q = dc["q"] if dc["q"].dim() == 4 else dc["q"].unsqueeze(1).contiguous()
+    for G in (5, sms):
+        trace = torch.zeros((G, BT.TRACE_WORDS), dtype=torch.int64, device="cuda")
+        ri = spec.batch * spec.kv_heads + 1
+        rec = torch.zeros(BT.record_bytes(G, ri), dtype=torch.uint8, device="cuda")
+        out, st, _ = BT.decode_step_multi(q, dc["k_pages"], dc["v_pages"], dc["block_table"], dc["seq_lens"],
+                                          spec.kv_heads, spec.tile_len, num_ctas=G, trace=trace, record=rec,
+                                          record_items=ri)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        used = int(BT.read_record(rec, G, ri)[0]["item_cost"][0])
+        split = OP.plan_cost_split(spec.seq_lens, spec.kv_heads, spec.tile_len, G, used)
+        n_items = [len(split.items[g]) for g in range(G)]
+        n_stages = [_chunks_of(split.items[g], spec.seq_lens, spec.tile_len, 128) for g in range(G)]
+        _check_stamps(trace.cpu().numpy(), n_items, n_stages, sms)
+
+
+def _chunks_of(items, lens, tl, C):
+    n = 0
+    for it in items:
+        L = lens[int(it["req"])]
+        t0, t1 = int(it["tile_begin"]) * tl, min(int(it["tile_end"]) * tl, L)
+        n += -(-(t1 - t0) // C)
+    return n
