@@ -169,8 +169,10 @@ typedef struct {
  *                 %globaltimer (ns): [0] entry, [1] plan ready (after the wait on the previous
  *                 kernel), [2] first stage consumed, [3] last item finished by the consumers,
  *                 [4] producer done; then [5] items, [6] pipeline stages, [7] SM id. Words [2]
- *                 and [3] stay 0 for a CTA without work. The mma.sync kernels write it; with a
- *                 tcgen05 kernel a trace buffer returns HPC_ERR_ARG. */
+ *                 and [3] stay 0 for a CTA without work. The mma.sync kernels and the
+ *                 several-token tcgen05 kernel write it (the latter counts 128-token stages in
+ *                 [6], filled by its K producer); with the E4M3 tcgen05 kernel a trace buffer
+ *                 returns HPC_ERR_ARG. */
 typedef struct {
   int32_t item_cost;
   int32_t e4m3_kernel;

@@ -1081,10 +1081,8 @@ int dispatch(int head_dim, bool fp8, bool tc, const CUtensorMap& mk, const CUten
     if (prm.trace) return fail(HPC_ERR_ARG, "the tcgen05 kernel writes no trace");
     return launch_attention_tc(FUSED, mk, mv, prm, grid, st);
   }
-  if (FUSED && MULTI && tcm && tcm_supported(head_dim, fp8, prm.group, prm.q_len, PRO)) {
-    if (prm.trace) return fail(HPC_ERR_ARG, "the tcgen05 kernel writes no trace");
-    return launch_attention_tcm(mk, mv, prm, grid, st);
-  }
+  if (FUSED && MULTI && tcm && tcm_supported(head_dim, fp8, prm.group, prm.q_len, PRO))
+    return launch_attention_tcm(mk, mv, prm, grid, st);  // stamps the trace in 128-token stages
   if (fp8) return launch<128, true, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
   if (head_dim == 128) return launch<128, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
   return launch<64, false, FUSED, PRO, MULTI>(mk, mv, prm, grid, smem, st);
