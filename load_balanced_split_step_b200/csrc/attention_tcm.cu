@@ -20,12 +20,13 @@
 // columns. Query rows 0..15 live in subpartition 0 and rows 16..31 in subpartition 1; each of
 // the two is worked by two warps (warp % 4 is the subpartition a warp reaches), one per half of
 // the 128 token columns, so a thread holds one (row, stage) with 64 scores and only the two
-// warps' row maxima and sums are exchanged. P (a bf16 high part and residual, two bf16 per 32-bit column) is written over the
-// stage's own S columns and is the A operand of the O product straight from tensor memory; V is
-// an MN-major B operand read from its swizzled TMA tile. Shared memory then holds only Q and the
-// K and V rings (three 32 KB slots each), the bytes a CTA keeps in flight. A new S is issued into
-// a buffer only once the O products that read the P there have completed: the tensor pipe does
-// not hold a later product's write to those columns behind an earlier product's read of them.
+// warps' row maxima and sums are exchanged. P (a bf16 high part and residual, two bf16 per
+// 32-bit column) is written over the stage's own S columns and is the A operand of the O product
+// straight from tensor memory; V is an MN-major B operand read from its swizzled TMA tile.
+// Shared memory then holds only Q and the K and V rings (three 32 KB slots each), the bytes a CTA
+// keeps in flight. A new S is issued into a buffer only once the O products that read the P
+// there have completed: the tensor pipe does not hold a later product's write to those columns
+// behind an earlier product's read of them.
 //
 // The running maximum per (row, half) moves only when a stage's maximum exceeds it by more than
 // 2^8 (log2 units); p = 2^(s - m) then stays below 256, and O in tensor memory is rescaled only on
@@ -328,8 +329,8 @@ __global__ void __launch_bounds__(kTmThreads, 1)
           const int64_t pair = pq0 + (iq >> 1);
           const int ks = static_cast<int>(nq % kTmKS);
           if (q_ready && pair < pairs_o + 2 &&
-              (pair < kTmSB ||
-               mbar_test(bar.buf_free(static_cast<int>(pair % kTmSB)), static_cast<uint32_t>((pair / kTmSB - 1) & 1))) &&
+              (pair < kTmSB || mbar_test(bar.buf_free(static_cast<int>(pair % kTmSB)),
+                                         static_cast<uint32_t>((pair / kTmSB - 1) & 1))) &&
               mbar_test(bar.k_full(ks), static_cast<uint32_t>((nq / kTmKS) & 1))) {
             tc_fence_after();
             const int half = static_cast<int>(iq & 1);
@@ -370,8 +371,8 @@ __global__ void __launch_bounds__(kTmThreads, 1)
             const uint32_t vbase = smem_u32(vring) + vs * kTmKV;
 #pragma unroll
             for (int kk = 0; kk < kTmTok / 16; ++kk)  // 16 tokens per product: high part of P
-              umma_bf16_ts(od, pa + 32 * (kk >> 1) + 8 * (kk & 1), umma_desc(vbase + 2048 * kk, kTmPlane, 1024, 2), kTmIdO,
-                           (iv >= 2 || kk > 0) ? 1u : 0u);
+              umma_bf16_ts(od, pa + 32 * (kk >> 1) + 8 * (kk & 1), umma_desc(vbase + 2048 * kk, kTmPlane, 1024, 2),
+                           kTmIdO, (iv >= 2 || kk > 0) ? 1u : 0u);
 #pragma unroll
             for (int kk = 0; kk < kTmTok / 16; ++kk)  // residual of P
               umma_bf16_ts(od, pa + 32 * (kk >> 1) + 16 + 8 * (kk & 1), umma_desc(vbase + 2048 * kk, kTmPlane, 1024, 2),
@@ -758,7 +759,8 @@ bool tcm_supported(int head_dim, bool fp8, int group, int q_len, bool pro) {
 
 int launch_attention_tcm(const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm, int grid,
                          cudaStream_t stream) {
-  if (prm.chunk_tokens < 16 || kTmTok % prm.chunk_tokens) return fail(HPC_ERR_SHAPE, "box of %d tokens", prm.chunk_tokens);
+  if (prm.chunk_tokens < 16 || kTmTok % prm.chunk_tokens)
+    return fail(HPC_ERR_SHAPE, "box of %d tokens", prm.chunk_tokens);
   if (prm.q_len * prm.group > kTmN) return fail(HPC_ERR_SHAPE, "q_len x group above %d", kTmN);
   static int configured[64] = {0};
   int dev = 0;
