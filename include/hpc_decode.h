@@ -152,7 +152,8 @@ typedef struct {
  *                 units over CTAs, in 1/16 of a tile, 0 .. HPC_ITEM_COST_MAX. 0 splits by tiles
  *                 alone (exactly hpc_decode_plan's CTA ranges). HPC_ITEM_COST_DEFAULT: the time
  *                 one item start takes, as KV bytes a CTA streams meanwhile: 152 KB with one new
- *                 token, 224 KB with several, converted to tiles of the call's shape (rounded).
+ *                 token; with several, 320 KB on the mma.sync consumers and 224 KB on the tcgen05
+ *                 kernel; converted to tiles of the call's shape (rounded).
  *   e4m3_kernel:  HPC_E4M3_MMA or HPC_E4M3_TCGEN05. The tcgen05 kernel serves E4M3 caches with
  *                 head_dim 128 in hpc_decode_attention, hpc_decode_step and hpc_decode_step_lse;
  *                 elsewhere the choice is ignored.
@@ -284,7 +285,8 @@ HPC_API size_t hpc_decode_step_workspace_bytes(int32_t batch, int32_t num_heads,
  *    with a closed form over the same tiles and unit order as hpc_decode_plan. The CTAs take
  *    contiguous unit runs of equal cost, where a tile costs 16 and each (request, kv head)
  *    segment start adds the fixed cost of an item: 152 KB worth of KV streaming with one new
- *    token, 224 KB with several (2.4 tiles of bf16 KV at tile_len 128, head_dim 128).
+ *    token (2.4 tiles of bf16 KV at tile_len 128, head_dim 128); with several, 320 KB on the
+ *    mma.sync consumers and 224 KB on the tcgen05 kernel.
  *    options->item_cost (1/16 of a tile, 0 .. HPC_ITEM_COST_MAX) sets it per call; 0 assigns
  *    exactly hpc_decode_plan's ranges (ceil(T / num_ctas) units per CTA).
  *  - options: NULL for the defaults, or see hpc_step_options (item cost, E4M3 kernel, per-CTA

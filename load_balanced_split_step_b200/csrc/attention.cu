@@ -1207,15 +1207,15 @@ struct PrologueArgs {
 // state, take the merge ticket (and merge), and load the next item's q; the ring keeps
 // streaming, but only a few stages beyond what covers the memory latency. Per-CTA
 // %globaltimer stamps on B200 put that cost near the time a CTA takes to stream 152 KB of KV
-// at its share of HBM (one new token), and 224 KB with several new tokens, where the
-// consumers are the bound. A CTA that starts many items (many short requests) therefore gets
-// fewer tiles. A caller's options->item_cost (1/16 tile) replaces it; 0 splits by tiles alone,
-// the pages' rule.
-int item_cost_units(int head_dim, bool fp8, int tile_len, int q_len, int32_t requested) {
+// at its share of HBM (one new token). With several new tokens a sweep of the cost put it at
+// 320 KB on the mma.sync consumers and 224 KB on the tcgen05 kernel. A CTA that starts many
+// items (many short requests) therefore gets fewer tiles. A caller's options->item_cost
+// (1/16 tile) replaces it; 0 splits by tiles alone, the pages' rule.
+int item_cost_units(int head_dim, bool fp8, int tile_len, int q_len, int32_t requested, bool tcm) {
   constexpr int64_t kMax = HPC_ITEM_COST_MAX;
   if (requested != HPC_ITEM_COST_DEFAULT) return requested;  // checked to lie in 0 .. kMax
   const int64_t tile_bytes = static_cast<int64_t>(tile_len) * head_dim * 2 * (fp8 ? 1 : 2);
-  const int64_t item_bytes = (q_len > 1 ? 224 : 152) * 1024;
+  const int64_t item_bytes = (q_len == 1 ? 152 : (tcm ? 224 : 320)) * 1024;
   const int64_t c = (kCostPerTile * item_bytes + tile_bytes / 2) / tile_bytes;
   return static_cast<int>(c > kMax ? kMax : c);
 }
@@ -1258,18 +1258,18 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.partial_ml = reinterpret_cast<float*>(ws + L.partial_ml);
   prm.batch = batch;
   prm.lse = lse;
-  prm.item_cost = item_cost_units(head_dim, kv_dtype == HPC_E4M3, tile_len, q_len, opt.item_cost);
+  const bool fp8 = kv_dtype == HPC_E4M3;
+  // by default three or four new tokens go to the tcgen05 kernel (one product per stage for all
+  // of them), two to the mma.sync consumers, where they are faster
+  const bool tcm = !pro && q_len > 1 && tcm_supported(head_dim, fp8, prm.group, q_len, false) &&
+                   (opt.multi_kernel == HPC_MULTI_TCGEN05 || (opt.multi_kernel == HPC_MULTI_DEFAULT && q_len >= 3));
+  prm.item_cost = item_cost_units(head_dim, fp8, tile_len, q_len, opt.item_cost, tcm);
   prm.record = opt.record;
   prm.record_items = opt.record_items;
   prm.trace = opt.trace;
-  const bool fp8 = kv_dtype == HPC_E4M3;
-  if (!pro && q_len > 1) {
-    // by default three or four new tokens go to the tcgen05 kernel (one product per stage for
-    // all of them), two to the mma.sync consumers, where they are faster
-    const bool tcm = opt.multi_kernel == HPC_MULTI_TCGEN05 || (opt.multi_kernel == HPC_MULTI_DEFAULT && q_len >= 3);
+  if (!pro && q_len > 1)
     return dispatch<true, false, true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem,
                                        static_cast<cudaStream_t>(stream), tcm);
-  }
   if (!pro)
     return dispatch<true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem, static_cast<cudaStream_t>(stream));
   prm.qkv = static_cast<const __nv_bfloat16*>(pro->qkv);

@@ -47,11 +47,14 @@ def _expected_record(B, split, record_items):
     return buf
 
 
-def _default_cost(tile_len, head_dim, kv_dtype, q_len):
+def _default_cost(tile_len, head_dim, kv_dtype, q_len, group):
     """The documented default: the time of one item start as KV bytes streamed meanwhile, 152 KB
-    with one new token and 224 KB with several, in 1/16 of a tile of this shape, rounded."""
+    with one new token; with several, 224 KB on the tcgen05 kernel (the default for three or four
+    tokens on a bf16 cache with head_dim 128 and q_len * group <= 32) and 320 KB on the mma.sync
+    consumers; in 1/16 of a tile of this shape, rounded."""
     tile_bytes = tile_len * head_dim * 2 * (1 if kv_dtype == "e4m3" else 2)
-    item_bytes = (224 if q_len > 1 else 152) * 1024
+    tcm = q_len >= 3 and kv_dtype == "bf16" and head_dim == 128 and q_len * group <= 32
+    item_bytes = (152 if q_len == 1 else (224 if tcm else 320)) * 1024
     return min(1024, (16 * item_bytes + tile_bytes // 2) // tile_bytes)
 
 
@@ -85,7 +88,7 @@ def _run(B, lens, Hq, Hkv, D, P, tl, kv, G, cost, q_len=1, seed=0, e4m3_kernel="
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     used = int(B.read_record(rec, G, record_items)[0]["item_cost"][0])
-    want_cost = _default_cost(tl, D, kv, q_len) if cost is None else cost
+    want_cost = _default_cost(tl, D, kv, q_len, Hq // Hkv) if cost is None else cost
     assert used == want_cost
     split = OP.plan_cost_split(lens, Hkv, tl, G, used)
     assert rec.cpu().numpy().tobytes() == _expected_record(B, split, record_items).tobytes()
