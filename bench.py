@@ -790,25 +790,34 @@ def measure(step, spec, lens, K, W_, world, local, jobs=1, per_gpu_div=1):
             "clocks": clk.summary()}
 
 
-OTHER_WORKLOADS = ("uniform", "heavy", "fp8")
+OTHER_WORKLOADS = ("uniform", "heavy", "fp8", "heavy_q4")
 
 
 def other_workload(B, args, name, dev, G, world, local):
     """The same measurement on another named workload (single-launch path; the FP8 workload runs
-    the prologue kernel in front of it), for the workloads object of the JSON line."""
-    spec = W.config_spec(name)
+    the prologue kernel in front of it), for the workloads object of the JSON line. heavy_q4 is
+    the heavy-tailed batch with four new tokens per request, on the library's default kernel for
+    them (the tcgen05 several-token kernel)."""
+    from dataclasses import replace
+    q_len = 4 if name == "heavy_q4" else 1
+    base = "heavy" if name == "heavy_q4" else name
+    spec = W.config_spec(base)
+    if q_len > 1:
+        spec = replace(spec, q_len=q_len, name=f"{spec.name}, {q_len} new tokens per request")
     case = W.make_case(spec)
     dc = device_case(case, dev)
     del case
     step = Step(B, spec, dc, G, spec.tile_len, fused=True, item_cost=args.item_cost, e4m3_kernel=args.e4m3_kernel)
     lens = step_lengths(dc, spec)
-    est_ms = W.algorithmic_bytes(spec) / 6.0e9
+    est_ms = W.algorithmic_bytes(spec) / (6.0e9 if q_len == 1 else 4.0e9)
     K = int(min(5000, max(64, round(1500.0 / est_ms))))
     K -= K % spec.steps
     m = measure(step, spec, lens, K, 20, world, local)
-    out = {"workload": WORKLOAD_TEXT[name], "steps": K, "warmup": 20, "us_per_step": round(1000 * m["ms_step"], 2),
+    text = WORKLOAD_TEXT[base] + (f"; {q_len} new tokens per request, causal among themselves" if q_len > 1 else "")
+    kernel = "decode_attention_tcm_kernel (tcgen05)" if q_len > 1 else "decode_attention_kernel<fused>"
+    out = {"workload": text, "steps": K, "warmup": 20, "us_per_step": round(1000 * m["ms_step"], 2),
            "value": round(m["value"], 2), "unit": "GB/s",
-           "roofline": dict(m["roofline"], kernel="decode_attention_kernel<fused>", traffic=load_traffic(name)),
+           "roofline": dict(m["roofline"], kernel=kernel, traffic=load_traffic(name) if q_len == 1 else None),
            "clocks": m["clocks"], "gpu_launches": step.launches * K,
            "path": "single launch" + (" after the prologue kernel (PDL)" if spec.prologue else "")}
     if spec.steps > 1:
