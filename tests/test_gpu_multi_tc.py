@@ -1,8 +1,9 @@
 """Several new tokens per request on the tcgen05 kernel (options.multi_kernel = HPC_MULTI_TCGEN05),
 through the C ABI, against the fp64 oracle's causal multi-token attention: every q_len from 1 to
 4, GQA groups of 8, 4 and 1, ragged lengths (including L = q_len, requests too short for q_len,
-and empty ones), several grid sizes, both page layouts, pages outside the pool, the in-kernel
-split's record, and a full-size heavy-tailed batch with four new tokens on sampled requests."""
+and empty ones), several grid sizes (up to twice the SM count), both page layouts, pages outside
+the pool, the in-kernel split's record, and a full-size heavy-tailed batch with four new tokens on
+sampled requests."""
 import numpy as np
 import pytest
 import torch
@@ -48,7 +49,7 @@ def test_matches_oracle(B, T, Hq, Hkv, P, tl):
     case = W.make_case(spec)
     dc = to_device(case)
     ref = _oracle(case)
-    for G in (1, 5, 148):
+    for G in (1, 5, 148, 296):  # 296: more CTAs than SMs (one CTA per SM is resident at a time)
         out, st, ws = _run(B, spec, dc, G)
         assert st == 0
         assert_bf16_tol(out, ref, what=f"tcgen05 q_len {T} {(Hq, Hkv, P, tl)} G={G}")
