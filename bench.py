@@ -713,7 +713,7 @@ def kernel_source_hash():
 
 def load_traffic(workload):
     """DRAM bytes per attention launch at this workload's full size, from profiles/traffic.json
-    (written from an ncu capture; see profiles/attention_<workload>_dram.md for the command), or
+    (written by --record-traffic from a 1-pass ncu capture of dram bytes), or
     None when the kernel source has changed since those counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
