@@ -134,6 +134,7 @@ constexpr int kTmOffK = 2 * kTmQ;
 constexpr int kTmOffV = kTmOffK + kTmKS * kTmKV;
 constexpr int kTmOffBar = kTmOffV + kTmVS * kTmKV;
 constexpr int kTmSmem = kTmOffBar + TmBars::kCount * 8 + 1024;  // + alignment slack
+static_assert(kTmVS >= 2, "the softmax's wait on a V fill needs the slot's previous fill landed");
 
 __device__ __forceinline__ int64_t tm_stages(const ItemInfo& x) {
   return x.tok1 > x.tok0 ? (x.tok1 - x.tok0 + kTmTok - 1) / kTmTok : 0;
@@ -616,7 +617,16 @@ __global__ void __launch_bounds__(kTmThreads, 1)
         // may hold anything (even NaN) and are zeroed, so that 0 * v stays 0. The 64 threads of a
         // half take tokens q and q + 64 (q = 16 (2 hb + sp) + l % 16) of their stage.
         if (__any_sync(0xffffffffu, dead_any)) {
-          if (dead_any) {
+          // The wait on the stage's V fill is by phase parity, which is exact only once the slot's
+          // previous fill (stage k - kTmVS) has landed. Nothing orders that before this point (the
+          // S of this pair implies only the O products of pair gp - 2), so the O products of pair
+          // gp - 1 are waited for first: they read every V fill through stage k - 2. Their commit
+          // is buf_free, whose phase before (pair gp - 3) completed before this pair's S was written.
+          if (dead_any && gp >= 1 &&
+              !mbar_wait(bar.buf_free(static_cast<int>((gp - 1) % kTmSB)),
+                         static_cast<uint32_t>(((gp - 1) / kTmSB) & 1)))
+            fail_wait();
+          if (dead_any && ok) {
             const int vs = static_cast<int>(k % kTmVS);
             if (mbar_wait(bar.v_full(vs), static_cast<uint32_t>((k / kTmVS) & 1))) {
               const int q0 = 16 * (2 * hb + sp) + (lane & 15);
@@ -652,12 +662,18 @@ __global__ void __launch_bounds__(kTmThreads, 1)
       pair0 += npairs;
 
       // ---- item end: the two halves combined by log-sum-exp (lanes l and l ^ 16 hold the same
-      // row), once each half's last O product is complete. A row's sum is split over the two
+      // row), once every O product of the item is complete. A row's sum is split over the two
       // column halves' warps.
       s_pl[sp][hb][lane] = l_sum;
       named_barrier_sync(pbar, 64);
       l_sum += s_pl[sp][hb ^ 1][lane];
-      if (had && !mbar_wait(bar.o_done(h), static_cast<uint32_t>((pv_cnt - 1) & 1))) fail_wait();
+      // The item's last pair gp = pair0 - 1: its buf_free commit follows every O product through
+      // it. Its phase before, pair gp - 2, completed before the S of pair gp was written, so the
+      // parity wait is exact. (A half's own o_done would not do: its phase before is the O
+      // product of pair gp - 1, which nothing here orders.)
+      if (npairs > 0 && !mbar_wait(bar.buf_free(static_cast<int>((pair0 - 1) % kTmSB)),
+                                   static_cast<uint32_t>(((pair0 - 1) / kTmSB) & 1)))
+        fail_wait();
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       const float m_o = __shfl_xor_sync(0xffffffffu, m_used, 16);
