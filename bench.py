@@ -702,10 +702,28 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+def uses_tcgen05_multi(spec, multi_kernel):
+    """Whether a several-token step runs the tcgen05 kernel: asked for, or the library's default
+    for three or four tokens on a bf16 cache with head_dim 128 and q_len x group <= 32."""
+    if spec.q_len == 1:
+        return False
+    fits = spec.kv_dtype == "bf16" and spec.head_dim == 128 and spec.q_len * (spec.num_heads // spec.kv_heads) <= 32
+    return fits and (multi_kernel == "tcgen05" or (multi_kernel == "default" and spec.q_len >= 3))
+
+
+def traffic_key(workload, q_len):
+    """profiles/traffic.json key: the workload name, with _q<T> for T new tokens per request."""
+    return workload if q_len == 1 else f"{workload}_q{q_len}"
+
+
+def kernel_source_hash(key="extreme"):
+    """Hash of the sources of the kernel that the traffic entry `key` measured: the several-token
+    tcgen05 kernel for the four-token entry (its default kernel), the single-launch kernel for
+    the others."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("attention.cu", "attention_common.cuh", "hpc_common.cuh"):
+    main = "attention_tcm.cu" if key.endswith(("_q3", "_q4")) else "attention.cu"
+    for name in (main, "attention_common.cuh", "hpc_common.cuh"):
         with open(os.path.join(ROOT, "load_balanced_split_step_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -720,7 +738,7 @@ def load_traffic(workload):
         return None
     with open(p) as f:
         entry = json.load(f).get(workload)
-    if not entry or entry.get("source_sha256_16") != kernel_source_hash():
+    if not entry or entry.get("source_sha256_16") != kernel_source_hash(workload):
         return None
     return int(entry["traffic_bytes_per_launch"])
 
@@ -738,20 +756,26 @@ def record_traffic(args):
             got[name] = float(row["Metric Value"].replace(",", "")) * units.get(row["Metric Unit"], 1)
     if len(got) != 2:
         raise SystemExit(f"{args.record_traffic}: no dram__bytes_read.sum / dram__bytes_write.sum rows")
+    from dataclasses import replace
     sample = workload_spec(args)
     full = W.config_spec(args.workload)
+    if args.q_len > 1:
+        full = replace(full, q_len=args.q_len)
     scale = W.algorithmic_bytes(full) / W.algorithmic_bytes(sample)
     traffic = (got["dram__bytes_read.sum"] + got["dram__bytes_write.sum"]) * scale
     p = os.path.join(ROOT, "profiles", "traffic.json")
     data = json.load(open(p)) if os.path.exists(p) else {}
-    data[args.workload] = {"traffic_bytes_per_launch": int(round(traffic)), "source_sha256_16": kernel_source_hash(),
+    key = traffic_key(args.workload, args.q_len)
+    if args.q_len > 1 and args.multi_kernel != "default":
+        raise SystemExit("--record-traffic with --q-len > 1 records the default kernel only")
+    data[key] = {"traffic_bytes_per_launch": int(round(traffic)), "source_sha256_16": kernel_source_hash(key),
                            "read_bytes": int(got["dram__bytes_read.sum"]), "write_bytes": int(got["dram__bytes_write.sum"]),
                            "captured_requests": sample.batch, "scale_to_full": round(scale, 6),
                            "algorithmic_bytes_full": int(W.algorithmic_bytes(full))}
     with open(p, "w") as f:
         json.dump(data, f, indent=1, sort_keys=True)
         f.write("\n")
-    return {"workload": args.workload, **data[args.workload]}
+    return {"workload": key, **data[key]}
 
 
 def device_case(case, dev, layout="HND"):
@@ -817,7 +841,7 @@ def other_workload(B, args, name, dev, G, world, local):
     kernel = "decode_attention_tcm_kernel (tcgen05)" if q_len > 1 else "decode_attention_kernel<fused>"
     out = {"workload": text, "steps": K, "warmup": 20, "us_per_step": round(1000 * m["ms_step"], 2),
            "value": round(m["value"], 2), "unit": "GB/s",
-           "roofline": dict(m["roofline"], kernel=kernel, traffic=load_traffic(name) if q_len == 1 else None),
+           "roofline": dict(m["roofline"], kernel=kernel, traffic=load_traffic(traffic_key(base, q_len))),
            "clocks": m["clocks"], "gpu_launches": step.launches * K,
            "path": "single launch" + (" after the prologue kernel (PDL)" if spec.prologue else "")}
     if spec.steps > 1:
@@ -921,9 +945,11 @@ def run_ours(args, rank, world, local):
                                    "log-sum-exp merge of split requests") if args.shard
                    else f"{world} independent replica(s), no collective"},
         "roofline": dict(m["roofline"],
-                         kernel="decode_attention_kernel" + {"fused": "<fused>", "folded": "<fused, prologue>",
-                                                             "split": ""}[args.path],
-                         traffic=load_traffic(args.workload) if not (args.requests or args.q_len > 1) else None),
+                         kernel="decode_attention_tcm_kernel (tcgen05)" if uses_tcgen05_multi(spec, args.multi_kernel)
+                         else "decode_attention_kernel" + {"fused": "<fused>", "folded": "<fused, prologue>",
+                                                           "split": ""}[args.path],
+                         traffic=load_traffic(traffic_key(args.workload, args.q_len))
+                         if not args.requests and (args.q_len == 1 or args.multi_kernel == "default") else None),
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": round(1000 * e2e_ms / e2e_steps, 2)},
