@@ -225,7 +225,7 @@ class Step:
                                    kv_layout=self.layout, k_scale=dc["k_scale"], v_scale=dc["v_scale"],
                                    eps=s.rms_eps, rope_theta=s.rope_theta, num_ctas=self.num_ctas, out=self.out,
                                    status=self.status, workspace=self.ws, item_cost=self.item_cost,
-                                   trace=self.trace)
+                                   trace=self.trace, seq_lens_ready=True)
             if ev is not None:
                 ev[1].record()
             return self.out
@@ -241,7 +241,7 @@ class Step:
                                 kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                                 v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
                                 workspace=self.ws, item_cost=self.item_cost, trace=self.trace,
-                                multi_kernel=self.multi_kernel)
+                                multi_kernel=self.multi_kernel, seq_lens_ready=True)
             if ev is not None:
                 ev[1].record()
             return self.out
@@ -252,7 +252,7 @@ class Step:
                                 s.kv_heads, self.tl, kv_dtype=s.kv_dtype, kv_layout=self.layout, k_scale=dc["k_scale"],
                                 v_scale=dc["v_scale"], num_ctas=self.num_ctas, out=self.out, status=self.status,
                                 workspace=self.ws, item_cost=self.item_cost, e4m3_kernel=self.e4m3_kernel,
-                                trace=self.trace)
+                                trace=self.trace, seq_lens_ready=True)
             if ev is not None:
                 ev[1].record()
             return self.out
@@ -481,7 +481,7 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
                                        d["block_table"], d["seq_lens"], spec.num_heads, spec.kv_heads, tl,
                                        kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
                                        v_scale=d["v_scale"], eps=spec.rms_eps, rope_theta=spec.rope_theta,
-                                       num_ctas=num_ctas, out=outs[b], workspace=ws)
+                                       num_ctas=num_ctas, out=outs[b], workspace=ws, seq_lens_ready=True)
             elif spec.prologue:
                 q = B.prologue(d["qkv"], d["q_norm_w"], d["k_norm_w"], d["k_pages"], d["v_pages"], d["block_table"],
                                d["seq_lens"], spec.num_heads, spec.kv_heads, kv_dtype=spec.kv_dtype, kv_layout=layout,
@@ -493,11 +493,12 @@ def e2e_leg(B, spec, case, dc, tl, num_ctas, steps, world, fused=True, layout="H
                 B.decode_step_multi(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.kv_heads, tl,
                                     kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
                                     v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws,
-                                    multi_kernel=multi_kernel)
+                                    multi_kernel=multi_kernel, seq_lens_ready=True)
             elif fused:
                 B.decode_step_fused(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
                                     spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
-                                    v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws)
+                                    v_scale=d["v_scale"], num_ctas=num_ctas, out=outs[b], workspace=ws,
+                                    seq_lens_ready=True)
             else:
                 B.decode_step(q, d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"], spec.num_heads,
                               spec.kv_heads, tl, kv_dtype=spec.kv_dtype, kv_layout=layout, k_scale=d["k_scale"],
@@ -933,7 +934,9 @@ def run_ours(args, rank, world, local):
         "dtype": "bf16" if spec.kv_dtype == "bf16" else "e4m3/f16",
         "data": "synthetic (seeded N(0,1), bf16-rounded; random page permutation)",
         "config": {"workload": WORKLOAD_TEXT[args.workload] + qlen_text(args), "tile_len": tl, "num_ctas": G,
-                   "plan": "dynamic (re-planned on the device every step)",
+                   "plan": "dynamic (re-planned on the device every step)"
+                   + ("; the single launch plans while the previous step's kernel finishes (seq_lens_ready: no "
+                      "kernel writes the lengths)" if args.path in ("fused", "folded") and not args.shard else ""),
                    "path": ({"fused": "single launch: in-kernel plan, attention, ticket merge"
                                       + (" (after the prologue kernel, PDL)" if spec.prologue else ""),
                              "folded": "single launch: prologue, in-kernel plan, attention, ticket merge",

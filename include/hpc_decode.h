@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define HPC_DECODE_ABI_VERSION 8
+#define HPC_DECODE_ABI_VERSION 9
 
 /* Symbols of the library are hidden by default; the entry points below are exported. */
 #if defined(__GNUC__)
@@ -121,7 +121,7 @@ typedef struct {
   int32_t* merge_list;
 } hpc_plan;
 
-/* ---- per-call options (ABI 8) ----------------------------------------------------------- */
+/* ---- per-call options (ABI 9) ----------------------------------------------------------- */
 
 /* Record of one CTA's share of a single-launch step, written when a caller asks for it (tests,
  * debugging). CTA g writes the record at byte offset g * hpc_step_record_bytes(1, record_items):
@@ -167,13 +167,20 @@ typedef struct {
  *   trace:        device uint64 [num_ctas][HPC_TRACE_WORDS], or NULL. Only a library built with
  *                 HPC_TRACE (hpc_build_flags() & HPC_BUILD_TRACE) accepts it; the default build
  *                 returns HPC_ERR_ARG, and its kernels carry no trace code. Per CTA, from
- *                 %globaltimer (ns): [0] entry, [1] plan ready (after the wait on the previous
- *                 kernel), [2] first stage consumed, [3] last item finished by the consumers,
+ *                 %globaltimer (ns): [0] entry, [1] plan ready and the previous kernel on the
+ *                 stream finished, [2] first stage consumed, [3] last item finished by the consumers,
  *                 [4] producer done; then [5] items, [6] pipeline stages, [7] SM id. Words [2]
  *                 and [3] stay 0 for a CTA without work. The mma.sync kernels and the
  *                 several-token tcgen05 kernel write it (the latter counts 128-token stages in
  *                 [6], filled by its K producer); with the E4M3 tcgen05 kernel a trace buffer
- *                 returns HPC_ERR_ARG. */
+ *                 returns HPC_ERR_ARG.
+ *   seq_lens_ready: single-launch steps only, 0 or 1. 1 promises that the kernel launched just
+ *                 before this call on the stream does not write seq_lens (they were copied from
+ *                 the host, or written earlier). The kernel then reads them and plans its split
+ *                 while that kernel finishes (programmatic dependent launch), before it waits
+ *                 for it; everything else (q, the cache, the block table, the outputs) is still
+ *                 touched only after the wait. With 0 (the default) the plan follows the wait.
+ *                 A step whose previous kernel writes seq_lens must pass 0. */
 typedef struct {
   int32_t item_cost;
   int32_t e4m3_kernel;
@@ -181,9 +188,10 @@ typedef struct {
   int32_t record_items;
   int32_t multi_kernel;
   uint64_t* trace;
+  int32_t seq_lens_ready;
 } hpc_step_options;
 
-#define HPC_STEP_OPTIONS_INIT {HPC_ITEM_COST_DEFAULT, HPC_E4M3_MMA, NULL, 0, HPC_MULTI_DEFAULT, NULL}
+#define HPC_STEP_OPTIONS_INIT {HPC_ITEM_COST_DEFAULT, HPC_E4M3_MMA, NULL, 0, HPC_MULTI_DEFAULT, NULL, 0}
 
 /* Bytes of a record buffer for num_ctas CTAs with record_items entries each. */
 HPC_API size_t hpc_step_record_bytes(int32_t num_ctas, int32_t record_items);

@@ -56,7 +56,8 @@ class CPlan(ctypes.Structure):
 
 class COptions(ctypes.Structure):
     _fields_ = [("item_cost", ctypes.c_int32), ("e4m3_kernel", ctypes.c_int32), ("record", ctypes.c_void_p),
-                ("record_items", ctypes.c_int32), ("multi_kernel", ctypes.c_int32), ("trace", ctypes.c_void_p)]
+                ("record_items", ctypes.c_int32), ("multi_kernel", ctypes.c_int32), ("trace", ctypes.c_void_p),
+                ("seq_lens_ready", ctypes.c_int32)]
 
 
 _path = LIB
@@ -339,18 +340,22 @@ def _out_code(out):
 
 
 def options(item_cost=None, e4m3_kernel="mma", record=None, record_items=0, trace=None, device=None, num_ctas=None,
-            multi_kernel="default"):
+            multi_kernel="default", seq_lens_ready=False):
     """A ``hpc_step_options`` struct, or None when every option has its default.
     item_cost: 1/16 tile per item start (None: the library's default). e4m3_kernel: "mma" or
     "tcgen05". record: uint8 device tensor of ``record_bytes(num_ctas, record_items)`` bytes.
-    trace: int64 device tensor [num_ctas, TRACE_WORDS] (HPC_TRACE builds only)."""
+    trace: int64 device tensor [num_ctas, TRACE_WORDS] (HPC_TRACE builds only).
+    seq_lens_ready: the kernel launched just before on the stream does not write seq_lens, so the
+    single-launch step may plan before waiting for it."""
     if e4m3_kernel not in E4M3_KERNELS:
         raise HpcError(f"e4m3_kernel must be one of {list(E4M3_KERNELS)}")
     if multi_kernel not in MULTI_KERNELS:
         raise HpcError(f"multi_kernel must be one of {list(MULTI_KERNELS)}")
-    if item_cost is None and e4m3_kernel == "mma" and record is None and trace is None and multi_kernel == "default":
+    if (item_cost is None and e4m3_kernel == "mma" and record is None and trace is None and multi_kernel == "default"
+            and not seq_lens_ready):
         return None
     o = COptions()
+    o.seq_lens_ready = 1 if seq_lens_ready else 0
     o.item_cost = ITEM_COST_DEFAULT if item_cost is None else int(item_cost)
     o.e4m3_kernel = E4M3_KERNELS[e4m3_kernel]
     o.multi_kernel = MULTI_KERNELS[multi_kernel]
@@ -483,10 +488,11 @@ def _workspace(ws, nbytes, dev):
 def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *,
                       kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None,
                       out=None, out_dtype=torch.float32, status=None, workspace=None, item_cost=None,
-                      e4m3_kernel="mma", record=None, record_items=0, trace=None):
+                      e4m3_kernel="mma", record=None, record_items=0, trace=None, seq_lens_ready=False):
     """One decode step in a single launch (``hpc_decode_step``): in-kernel planning, attention
     and ticket merge. Returns (out, status, workspace); pass the workspace back on later calls.
-    item_cost, e4m3_kernel, record / record_items and trace are the call's options."""
+    item_cost, e4m3_kernel, record / record_items, trace and seq_lens_ready are the call's
+    options."""
     _need(q, "q", torch.bfloat16)
     dev = q.device
     B, Hq, D = q.shape
@@ -501,7 +507,7 @@ def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_
     status = new_status(dev) if status is None else status
     workspace = _workspace(workspace, _lib.hpc_decode_step_workspace_bytes(B, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    opt = options(item_cost, e4m3_kernel, record, record_items, trace, dev, G)
+    opt = options(item_cost, e4m3_kernel, record, record_items, trace, dev, G, seq_lens_ready=seq_lens_ready)
     with torch.cuda.device(dev):
         _check(_lib.hpc_decode_step(
             _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,
@@ -514,7 +520,8 @@ def decode_step_fused(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_
 def decode_step_prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads,
                          tile_len, *, kv_dtype="bf16", kv_layout="HND", k_scale=None, v_scale=None, eps=1e-6,
                          rope_theta=1e6, num_ctas=None, sm_scale=None, out=None, out_dtype=torch.float32,
-                         status=None, workspace=None, item_cost=None, record=None, record_items=0, trace=None):
+                         status=None, workspace=None, item_cost=None, record=None, record_items=0, trace=None,
+                         seq_lens_ready=False):
     """One decode step in a single launch with the prologue folded in
     (``hpc_decode_step_prologue``): the new token's K/V go into the cache and q is formed from
     qkv inside the attention kernel. Returns (out, status, workspace)."""
@@ -536,7 +543,7 @@ def decode_step_prologue(qkv, q_norm_w, k_norm_w, k_pages, v_pages, block_table,
     status = new_status(dev) if status is None else status
     workspace = _workspace(workspace, _lib.hpc_decode_step_workspace_bytes(B, num_heads, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    opt = options(item_cost, "mma", record, record_items, trace, dev, G)
+    opt = options(item_cost, "mma", record, record_items, trace, dev, G, seq_lens_ready=seq_lens_ready)
     with torch.cuda.device(dev):
         _check(_lib.hpc_decode_step_prologue(
             _ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta), _ptr(k_pages), _ptr(v_pages),
@@ -557,7 +564,7 @@ def multi_workspace(batch, q_len, num_heads, kv_heads, head_dim, num_ctas, devic
 def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile_len, *, kv_dtype="bf16",
                       kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None,
                       out_dtype=torch.float32, status=None, workspace=None, item_cost=None, record=None,
-                      record_items=0, trace=None, multi_kernel="default"):
+                      record_items=0, trace=None, multi_kernel="default", seq_lens_ready=False):
     """q_len new tokens per request in one launch (``hpc_decode_step_multi``): q is
     [B, q_len, Hq, D]; query token t of request r sits at position L_r - q_len + t and
     attends causally. multi_kernel: "default", "mma" or "tcgen05". Returns (out [B, q_len, Hq, D],
@@ -574,7 +581,7 @@ def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile
     status = new_status(dev) if status is None else status
     workspace = _workspace(workspace, _lib.hpc_decode_step_multi_workspace_bytes(B, T, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    opt = options(item_cost, "mma", record, record_items, trace, dev, G, multi_kernel)
+    opt = options(item_cost, "mma", record, record_items, trace, dev, G, multi_kernel, seq_lens_ready)
     with torch.cuda.device(dev):
         _check(_lib.hpc_decode_step_multi(
             _ptr(q), T, _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv,
@@ -586,7 +593,7 @@ def decode_step_multi(q, k_pages, v_pages, block_table, seq_lens, kv_heads, tile
 
 def decode_step_lse(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_heads, tile_len, *, kv_dtype="bf16",
                     kv_layout="HND", k_scale=None, v_scale=None, num_ctas=None, sm_scale=None, out=None, lse=None,
-                    status=None, workspace=None, item_cost=None, e4m3_kernel="mma"):
+                    status=None, workspace=None, item_cost=None, e4m3_kernel="mma", seq_lens_ready=False):
     """``hpc_decode_step_lse``: the single-launch step, plus the natural-log log-sum-exp of
     every output row. Returns (out fp32 [B, Hq, D], lse fp32 [B, Hq], status, workspace)."""
     _need(q, "q", torch.bfloat16)
@@ -607,7 +614,7 @@ def decode_step_lse(q, k_pages, v_pages, block_table, seq_lens, num_heads, kv_he
     status = new_status(dev) if status is None else status
     workspace = _workspace(workspace, _lib.hpc_decode_step_workspace_bytes(B, Hq, Hkv, D, G), dev)
     scale = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    opt = options(item_cost, e4m3_kernel, device=dev)
+    opt = options(item_cost, e4m3_kernel, device=dev, seq_lens_ready=seq_lens_ready)
     with torch.cuda.device(dev):
         _check(_lib.hpc_decode_step_lse(
             _ptr(q), _ptr(k_pages), _ptr(v_pages), code, lay, _ptr(k_scale), _ptr(v_scale), num_pages, P, Hq, Hkv, D,

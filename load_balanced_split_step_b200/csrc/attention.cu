@@ -450,14 +450,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   // Everything above overlaps the previous kernel's tail under programmatic dependent launch;
-  // the plan, seq_lens, q and the output buffers are touched only after it has finished.
-  pdl_wait();
-  pdl_launch_dependents();
+  // seq_lens, q, the cache and the output buffers are touched only after it has finished. The
+  // single launch's plan reads seq_lens alone, and runs before the wait when the caller says
+  // the previous kernel does not write them (plan_early).
+  const bool early = FUSED && p.plan_early;
+  if (!early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   Cursor cursor;
   int64_t chunk = 0;
   if constexpr (FUSED) {
     plan_in_kernel<D>(p, reinterpret_cast<int64_t*>(red_o), s_scan, s_walk, cursor, chunk);
+    if (early) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
   } else {
     cursor.it = p.cta_indptr[blockIdx.x];
     cursor.it_end = p.cta_indptr[blockIdx.x + 1];
@@ -975,6 +984,7 @@ struct Options {
   uint8_t* record = nullptr;
   int32_t record_items = 0;
   uint64_t* trace = nullptr;
+  int32_t seq_lens_ready = 0;  // single launch: plan before waiting for the previous kernel
 };
 
 int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
@@ -986,8 +996,9 @@ int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
     return fail(HPC_ERR_ARG, "e4m3_kernel must be HPC_E4M3_MMA or HPC_E4M3_TCGEN05");
   if (o->multi_kernel != HPC_MULTI_DEFAULT && o->multi_kernel != HPC_MULTI_MMA && o->multi_kernel != HPC_MULTI_TCGEN05)
     return fail(HPC_ERR_ARG, "multi_kernel must be HPC_MULTI_DEFAULT, HPC_MULTI_MMA or HPC_MULTI_TCGEN05");
-  if (!single_launch && (o->item_cost != HPC_ITEM_COST_DEFAULT || o->record))
-    return fail(HPC_ERR_ARG, "item_cost and record apply to the single-launch steps only");
+  if (o->seq_lens_ready != 0 && o->seq_lens_ready != 1) return fail(HPC_ERR_ARG, "seq_lens_ready must be 0 or 1");
+  if (!single_launch && (o->item_cost != HPC_ITEM_COST_DEFAULT || o->record || o->seq_lens_ready))
+    return fail(HPC_ERR_ARG, "item_cost, record and seq_lens_ready apply to the single-launch steps only");
   if (o->record && (o->record_items < 0 || (reinterpret_cast<uintptr_t>(o->record) & 15)))
     return fail(HPC_ERR_ARG, "record needs record_items >= 0 and 16-byte alignment");
 #ifndef HPC_TRACE
@@ -1000,6 +1011,7 @@ int read_options(const hpc_step_options* o, bool single_launch, Options* out) {
   out->record = static_cast<uint8_t*>(o->record);
   out->record_items = o->record ? o->record_items : 0;
   out->trace = o->trace;
+  out->seq_lens_ready = o->seq_lens_ready;
   return HPC_OK;
 }
 
@@ -1267,6 +1279,7 @@ int step_impl(const void* q, const void* k_pages, const void* v_pages, hpc_dtype
   prm.record = opt.record;
   prm.record_items = opt.record_items;
   prm.trace = opt.trace;
+  prm.plan_early = opt.seq_lens_ready;
   if (!pro && q_len > 1)
     return dispatch<true, false, true>(head_dim, fp8, opt.tc, mk, mv, prm, num_ctas, ls.smem,
                                        static_cast<cudaStream_t>(stream), tcm);

@@ -49,6 +49,7 @@ struct AttnParams {
   int32_t batch, kv_heads, max_seq_len;
   int32_t* tickets;  // [batch * kv_heads], zero between steps
   int32_t item_cost;  // cost of starting an item, in 1/kCostPerTile of a tile (0: split by tiles alone)
+  int32_t plan_early;  // seq_lens are not the previous kernel's output: plan before waiting for it
   // single-launch step with the prologue folded in: q comes from qkv through RMSNorm and RoPE,
   // and the new token's K/V are written into the cache
   const __nv_bfloat16* qkv;  // [batch][num_heads + 2 kv_heads][D]

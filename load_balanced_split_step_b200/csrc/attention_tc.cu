@@ -196,14 +196,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  pdl_wait();
-  pdl_launch_dependents();
+  // the single launch's plan reads seq_lens alone: before the wait on the previous kernel when
+  // that kernel does not write them (plan_early), after it otherwise
+  const bool early = FUSED && p.plan_early;
+  if (!early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   Cursor cursor;
   int64_t chunk = 0;
   if constexpr (FUSED) {
     // the per-request tile prefix lives in the ring until the first TMA copy is issued
     plan_in_kernel<kTcD>(p, reinterpret_cast<int64_t*>(ring), s_scan, s_walk, cursor, chunk);
+    if (early) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
   } else {
     cursor.it = p.cta_indptr[blockIdx.x];
     cursor.it_end = p.cta_indptr[blockIdx.x + 1];

@@ -200,13 +200,21 @@ __global__ void __launch_bounds__(kTmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  pdl_wait();
-  pdl_launch_dependents();
+  // the plan reads seq_lens alone: before the wait on the previous kernel when that kernel does
+  // not write them (plan_early), after it otherwise
+  if (!p.plan_early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   WalkCursor cursor;
   int64_t chunk = 0;
   // the per-request tile prefix lives in the K ring until the first TMA copy is issued
   plan_in_kernel<kTmD>(p, reinterpret_cast<int64_t*>(kring), s_scan, s_walk, cursor, chunk);
+  if (p.plan_early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 #ifdef HPC_TRACE
   if (trace && threadIdx.x == 0) trace[1] = global_timer_ns();
 #endif

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(B):
 
 
 def test_abi_version_and_strings(B):
-    assert B._lib.hpc_abi_version() == 8
+    assert B._lib.hpc_abi_version() == 9
     assert B.status_string(0) == "ok"
     assert B.status_string(6) == "buffer too small"
 
@@ -106,7 +106,7 @@ def test_host_argument_errors_return_codes(B):
 
 
 def test_options_are_checked_before_any_launch(B):
-    """Per-call options (ABI 8): out-of-range values, options that belong to the single-launch
+    """Per-call options (ABI 9): out-of-range values, options that belong to the single-launch
     step passed to the three-launch attention, and a trace buffer in a build without HPC_TRACE
     all return HPC_ERR_ARG before any CUDA call (the pointers are never dereferenced)."""
     w = ctypes.c_void_p(256)
@@ -130,6 +130,12 @@ def test_options_are_checked_before_any_launch(B):
         assert step(o) == B.HPC_ERR_ARG and what in B._lib.hpc_last_error().decode()
     o = B.options(item_cost=0)
     assert attention(o) == B.HPC_ERR_ARG and "single-launch" in B._lib.hpc_last_error().decode()
+    o = B.options(seq_lens_ready=True)
+    assert o.seq_lens_ready == 1
+    assert attention(o) == B.HPC_ERR_ARG and "single-launch" in B._lib.hpc_last_error().decode()
+    o.seq_lens_ready = 2
+    assert step(o) == B.HPC_ERR_ARG and "seq_lens_ready" in B._lib.hpc_last_error().decode()
+    assert B.options(seq_lens_ready=False) is None
     o = B.COptions(B.ITEM_COST_DEFAULT, 0, None, 0, 0, 4096)
     assert not (B.build_flags() & B.BUILD_TRACE)
     assert step(o) == B.HPC_ERR_ARG and "HPC_TRACE" in B._lib.hpc_last_error().decode()
