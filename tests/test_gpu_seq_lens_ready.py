@@ -2,8 +2,9 @@
 and plan their split before they wait for the previous kernel on the stream, which the caller
 promises does not write seq_lens. Checked: the same output bytes and the same record of the
 split as without it, on the one-token kernel (bf16; E4M3 on both E4M3 kernels), on both kernels
-for several new tokens and on the log-sum-exp step; and steps launched back to back, each on
-lengths written before the first launch, against the fp64 oracle."""
+for several new tokens, on the log-sum-exp step and with the prologue folded in (there also the
+same cache bytes); and steps launched back to back, each on lengths written before the first
+launch, against the fp64 oracle."""
 import pytest
 import torch
 
@@ -97,3 +98,25 @@ def test_back_to_back_steps(B):
         ref = oracle_out(case, seq_lens=case.seq_lens + s)
         assert_bf16_tol(outs[s], ref, what=f"back-to-back step {s}")
     assert bool(torch.all(ws[: len(LENS) * 8 * 4] == 0).item())  # merge tickets left at zero
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3"])
+def test_folded_prologue_same_bytes(B, kv_dtype):
+    """The single launch with the prologue folded in: the same output, cache bytes and split
+    record with and without the option (each run on its own copy of the cache, since the step
+    writes the new token into it)."""
+    spec = W.custom_spec(LENS, 64, 8, 128, 64, 128, kv_dtype=kv_dtype, prologue=True, seed=305)
+    case = W.make_case(spec)
+    got = []
+    for ready in (False, True):
+        d = to_device(case)
+        rec = torch.zeros(B.record_bytes(G, 8), dtype=torch.uint8, device="cuda")
+        out, st, _ = B.decode_step_prologue(d["qkv"], d["q_norm_w"], d["k_norm_w"], d["k_pages"], d["v_pages"],
+                                            d["block_table"], d["seq_lens"], 64, 8, 128, kv_dtype=kv_dtype,
+                                            k_scale=d["k_scale"], v_scale=d["v_scale"], num_ctas=G, record=rec,
+                                            record_items=8, seq_lens_ready=ready)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        got.append((out.clone(), d["k_pages"].clone(), d["v_pages"].clone(), rec.clone()))
+    for a, b in zip(got[0], got[1]):
+        assert torch.equal(a, b)
