@@ -180,7 +180,8 @@ typedef struct {
  *                 while that kernel finishes (programmatic dependent launch), before it waits
  *                 for it; everything else (q, the cache, the block table, the outputs) is still
  *                 touched only after the wait. With 0 (the default) the plan follows the wait.
- *                 A step whose previous kernel writes seq_lens must pass 0. */
+ *                 A step whose previous kernel writes seq_lens must pass 0: with 1 its split
+ *                 would be planned on lengths being written, and its results are undefined. */
 typedef struct {
   int32_t item_cost;
   int32_t e4m3_kernel;
